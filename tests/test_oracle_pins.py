@@ -139,6 +139,9 @@ def test_lk_hybrid_weighting_at_known_alpha():
         kl = a * math.log(a / b) + (1 - a) * math.log((1 - a) / (1 - b))
         lam = math.exp(-3 * alpha)
         assert abs(t["alpha"][0] - alpha) < 1e-14
+        # S = sum of q over the tokens where the draft is below the target.
+        S = (b if b < a else 0.0) + ((1 - b) if (1 - b) < (1 - a) else 0.0)
+        assert abs(t["S"][0] - S) < 1e-14
         assert abs(t["loss"][0] - (lam * kl + (1 - lam) * (1 - alpha))) < 1e-14
         assert abs(orc.token_terms("tv", zq, zp)["loss"][0] - 0.5 * (abs(a - b) * 2)) < 1e-14
         assert abs(orc.token_terms("nla", zq, zp)["loss"][0] + math.log(alpha)) < 1e-14
