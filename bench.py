@@ -1,0 +1,434 @@
+#!/usr/bin/env python
+"""Benchmark of the streaming LM-head loss: one step = forward + backward of the whole path
+(loss, per-token statistics, dH and dW) over one batch of synthetic tokens.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--kind KIND]
+                    [--impl ours|reference]
+
+Default workload: the Llama-3.1-8B-shaped forward KL(p||q): N=16384 tokens, d=4096,
+V=128256 (bf16 inputs, fp32 accumulation).  Prints one JSON line on rank 0.
+
+For N > 1 (torchrun, one rank per GPU) every rank streams its own batch of N tokens
+(weak scaling) and the ranks combine the result the way data-parallel training does: an
+all-reduce of (loss_sum, n_valid) before the backward normalises by the global valid
+count, and an all-reduce of dW after it.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "LM-head+loss fwd+bwd tokens/s (d=4096,V=128256); % of BF16 tensor peak"
+DEFAULT_WORKLOAD = "llama8b_kl"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = ["lm_head_loss_streaming_b200/csrc/slm_kernels.cu",
+                  "lm_head_loss_streaming_b200/csrc/sm100.cuh",
+                  "lm_head_loss_streaming_b200/csrc/slm_internal.h"]
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--kind", default=None)
+    ap.add_argument("--tokens", type=int, default=None, help="override N (tokens per GPU)")
+    ap.add_argument("--chunk-tokens", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-sample-rows", type=int, default=0)
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------------------
+# Algorithmic work.
+# ---------------------------------------------------------------------------------------
+def gemm_passes(kind):
+    """Number of N x V x d logit-sized GEMMs per token in fwd + bwd (each 2NVd flops):
+    CE: fwd 1 + recompute 1 + dH 1 + dW 1 = 4;  KL: 2 + 2 + 1 + 1 = 6;
+    alpha losses: 2 + 2 (second pass) + 2 + 1 + 1 = 8."""
+    return {"ce": 4, "kl_div": 6}.get(kind, 8)
+
+
+def fwd_gemm_passes(kind):
+    return 1 if kind == "ce" else 2
+
+
+def launches_per_step(kind, N, d, chunk_tokens):
+    """Kernels of libslm.so launched by one forward + backward (memsets excluded)."""
+    if N == 0:
+        return 1 + 1
+    fwd = 3 if kind in ("ce", "kl_div") else 5  # GEMM, combine, [alpha GEMM, combine], finalize
+    C = chunk_tokens if chunk_tokens > 0 else ((2 * d + 127) // 128) * 128
+    C = max(1, min(C, N))
+    chunks = (N + C - 1) // C
+    return fwd + 3 * chunks
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha1()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:12]
+
+
+def traffic_for(workload, kind, kernel):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, or None when the
+    kernel sources changed since the counters were taken."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    cur = kernel_source_hash()
+    with open(TRAFFIC_FILE) as f:
+        for line in f:
+            parts = line.split()
+            if len(parts) >= 5 and not line.startswith("#"):
+                wl, kd, kn, sha, nbytes = parts[:5]
+                if (wl, kd, kn, sha) == (workload, kind, kernel, cur):
+                    return float(nbytes)
+    return None
+
+
+# ---------------------------------------------------------------------------------------
+# Clock sampling during the timed region.
+# ---------------------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", str(self.gpu)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            c = [x.strip() for x in line.split(",")]
+            if len(c) < 9:
+                continue
+            try:
+                sm.append(float(c[1]))
+                mx = float(c[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, c[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        sm.sort()
+        med = sm[len(sm) // 2] if sm else None
+        return {"sm_mhz": med, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------------------
+# CPU baseline: the float64 oracle on a bounded sample of the same workload.
+# ---------------------------------------------------------------------------------------
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else None
+    except Exception:
+        return None
+
+
+def oracle_sample(workload, kind, rows, steps, warmup):
+    """Time the oracle's forward + backward on `rows` token rows of the workload's shape
+    (same V, d and value distributions; CPU-drawn inputs).  Returns tokens/s and details."""
+    import oracle
+    from lm_head_loss_streaming_b200 import synthetic
+
+    inp = synthetic.workload(workload, kind=kind, N=rows, seed=1234, device="cpu")
+    times = []
+    for it in range(warmup + steps):
+        t0 = time.perf_counter()
+        oracle.forward(kind, inp.Hq, inp.W, inp.labels, inp.Hp, inp.ignore_index)
+        oracle.backward(kind, inp.Hq, inp.W, inp.labels, inp.Hp, None, inp.ignore_index)
+        dt = time.perf_counter() - t0
+        if it >= warmup:
+            times.append(dt)
+    t = sum(times) / len(times)
+    return rows / t, t
+
+
+def cpu_baseline_block(workload, kind, rows):
+    tps, t = oracle_sample(workload, kind, rows, 1, 0)
+    return {"value": round(tps, 3), "unit": "tokens/s", "cores": blas_threads() or cpu_cores(),
+            "kind": "oracle",
+            "sample": f"float64 NumPy oracle, fwd+bwd of {rows} token rows of the "
+                      f"{workload} shape (V, d full) in {t:.1f} s on host cores"}
+
+
+# ---------------------------------------------------------------------------------------
+# Our implementation.
+# ---------------------------------------------------------------------------------------
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from lm_head_loss_streaming_b200 import synthetic
+    from lm_head_loss_streaming_b200.loss import (FwdResult, lm_head_loss_bwd,
+                                                  lm_head_loss_fwd, workspace_bytes)
+    from lm_head_loss_streaming_b200 import _lib
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=dev)
+
+    cfg = synthetic.WORKLOADS[args.workload]
+    kind = args.kind or cfg["kinds"][0]
+    N = args.tokens or cfg["N"]
+    inp = synthetic.workload(args.workload, kind=kind, seed=rank, device=dev, N=N)
+    d, V = inp.d, inp.V
+    Hq, W, Hp, lab = inp.Hq, inp.W, inp.Hp, inp.labels
+    k = _lib.KIND[kind]
+    ws = torch.empty(workspace_bytes(kind, N, d, V, args.chunk_tokens), dtype=torch.uint8,
+                     device=dev)
+    nk = _lib.slm_stats_floats(k)
+    res = FwdResult(k, torch.empty(1, device=dev), torch.empty(1, dtype=torch.float64, device=dev),
+                    torch.empty(1, dtype=torch.int64, device=dev), torch.empty(N, device=dev),
+                    torch.empty(N, device=dev) if k >= 2 else None,
+                    torch.empty(nk, N, device=dev), ws)
+    dH = torch.empty(N, d, dtype=torch.bfloat16, device=dev)
+    dW = torch.empty(V, d, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        lm_head_loss_fwd(kind, Hq, W, lab, Hp, inp.ignore_index, workspace=ws,
+                         chunk_tokens=args.chunk_tokens, out=res)
+        if ev is not None:
+            ev[1].record(stream)
+        if world > 1:
+            dist.all_reduce(res.n_valid)
+        lm_head_loss_bwd(res, Hq, W, lab, Hp, inp.ignore_index, dH=dH, dW=dW,
+                         chunk_tokens=args.chunk_tokens)
+        if world > 1:
+            dist.all_reduce(dW)
+            dist.all_reduce(res.loss_sum)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st = _lib.slm_device_status(ws.data_ptr(), stream.cuda_stream)
+    if st != 0:
+        raise RuntimeError(f"device status after warm-up: {_lib.status_string(st)}")
+
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    t0.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    total_ms = t0.elapsed_time(t1)
+    fwd_ms = sum(a.elapsed_time(b) for a, b in evs) / len(evs)
+    if world > 1:
+        tt = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    ms_step = total_ms / args.steps
+    tokens_per_s = world * N / (ms_step / 1e3)
+
+    # End to end through the public API with host buffers: each step copies the inputs
+    # from pinned host memory and reads the loss back.
+    e2e = None
+    if not args.no_e2e:
+        hHq = Hq.cpu().pin_memory()
+        hW = W.cpu().pin_memory()
+        hHp = Hp.cpu().pin_memory() if Hp is not None else None
+        hlab = lab.cpu().pin_memory() if lab is not None else None
+        dHq, dWt = torch.empty_like(Hq), torch.empty_like(W)
+        dHp = torch.empty_like(Hp) if Hp is not None else None
+        dlab = torch.empty_like(lab) if lab is not None else None
+        hloss = torch.empty(1, dtype=torch.float32).pin_memory()
+        h2d = hHq.numel() * 2 + hW.numel() * 2 + (hHp.numel() * 2 if hHp is not None else 0) \
+            + (hlab.numel() * 4 if hlab is not None else 0)
+
+        def e2e_step():
+            dHq.copy_(hHq, non_blocking=True)
+            dWt.copy_(hW, non_blocking=True)
+            if dHp is not None:
+                dHp.copy_(hHp, non_blocking=True)
+            if dlab is not None:
+                dlab.copy_(hlab, non_blocking=True)
+            lm_head_loss_fwd(kind, dHq, dWt, dlab, dHp, inp.ignore_index, workspace=ws,
+                             chunk_tokens=args.chunk_tokens, out=res)
+            if world > 1:
+                dist.all_reduce(res.n_valid)
+            lm_head_loss_bwd(res, dHq, dWt, dlab, dHp, inp.ignore_index, dH=dH, dW=dW,
+                             chunk_tokens=args.chunk_tokens)
+            if world > 1:
+                dist.all_reduce(dW)
+                dist.all_reduce(res.loss_sum)
+            hloss.copy_(res.loss_mean, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        ksteps = max(1, min(args.steps, 5))
+        if world > 1:
+            dist.barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(ksteps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        e_ms = a.elapsed_time(b) / ksteps
+        if world > 1:
+            tt = torch.tensor([e_ms], device=dev)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            e_ms = float(tt.item())
+        e2e = {"value": round(world * N / (e_ms / 1e3), 1), "unit": "tokens/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": 4,
+               "ms_per_step": round(e_ms, 3)}
+
+    peaks, peak_src = load_peaks()
+    flops_step = gemm_passes(kind) * 2.0 * N * V * d
+    base_flops = 8.0 * N * V * d
+    fwd_flops = fwd_gemm_passes(kind) * 2.0 * N * V * d
+    achieved = fwd_flops / (fwd_ms / 1e3) / 1e12
+    peak = peaks["bf16_tflops_sustained"]
+    traffic = traffic_for(args.workload, kind, "fwd_gemm")
+    out = {
+        "metric": METRIC,
+        "value": round(tokens_per_s, 1),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded; no weights or datasets)",
+        "config": {"workload": args.workload, "kind": kind, "tokens_per_gpu": N, "d": d,
+                   "V": V, "global_batch_tokens": world * N, "parallelism": f"dp{world}",
+                   "chunk_tokens": args.chunk_tokens or "auto",
+                   "l2": "inputs larger than L2 (W alone is %.2f GB)" % (V * d * 2 / 1e9)},
+        "tflops": round(flops_step / (ms_step / 1e3) / 1e12, 1),
+        "frac_bf16_peak": round(flops_step / (ms_step / 1e3) / 1e12 / peaks["bf16_tflops"], 4),
+        "frac_bf16_peak_8NVd": round(base_flops / (ms_step / 1e3) / 1e12 / peaks["bf16_tflops"], 4),
+        "peak_source": f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback",
+        "roofline": {"bound": "tensor", "kernel": "forward statistics GEMM",
+                     "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak, 4), "traffic": traffic,
+                     "fwd_ms": round(fwd_ms, 3), "peak_kind": "sustained bf16, " + peak_src},
+        "gpu_launches": launches_per_step(kind, N, d, args.chunk_tokens) * args.steps,
+        "clocks": clocks,
+        "e2e": e2e,
+        "kernel_sha": kernel_source_hash(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rows = args.cpu_sample_rows or 128
+        out["cpu_baseline"] = cpu_baseline_block(args.workload, kind, rows)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def run_reference(args):
+    """The oracle as it stands, on host cores, on a bounded sample of the same workload."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from lm_head_loss_streaming_b200 import synthetic
+    cfg = synthetic.WORKLOADS[args.workload]
+    kind = args.kind or cfg["kinds"][0]
+    rows = args.cpu_sample_rows or 32
+    tps, t = oracle_sample(args.workload, kind, rows, args.steps, args.warmup)
+    cores = blas_threads() or cpu_cores()
+    sample = (f"float64 NumPy oracle, fwd+bwd of {rows} token rows per step of the "
+              f"{args.workload} shape (V, d full)")
+    out = {
+        "metric": METRIC, "value": round(tps, 3), "unit": "tokens/s", "impl": "reference",
+        "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(t * 1e3, 1), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "kind": kind, "tokens_per_step": rows,
+                   "d": cfg["d"], "V": cfg["V"]},
+        "cpu_baseline": {"value": round(tps, 3), "unit": "tokens/s", "cores": cores,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(tps, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,156 @@
+/*
+ * slm.h - C ABI of the streaming LM-head loss for NVIDIA B200 (sm_100a).
+ *
+ * What is computed.  Hidden states H_q [N, d] are projected by the LM head W [V, d] to
+ * logits z_q = H_q W^T [N, V], which are reduced to one loss per token row and to the
+ * gradients dH_q [N, d] and dW [V, d], without ever storing the [N, V] logits or their
+ * gradient ("Training speculative decoders: removing the logits and attention
+ * bottlenecks", sections "The logits bottleneck in long-context draft-head training",
+ * "Streaming Cross Entropy" and "Backward pass").
+ *
+ * Loss kinds ("Loss Functions", table "Available Losses"; p = softmax(H_p W^T) is the
+ * target, q = softmax(H_q W^T) the draft, alpha = sum_v min(p_v, q_v)):
+ *   SLM_CE         hard-label cross entropy  -log q_y       (labels required)
+ *   SLM_KL         forward KL, target to draft  KL(p || q)
+ *   SLM_TV         total variation  1 - alpha
+ *   SLM_NLA        negative log-acceptance  -log(alpha)   (alpha clamped at 1e-30)
+ *   SLM_LK_HYBRID  lambda * KL + (1 - lambda) * TV,  lambda = exp(-3 alpha) per token,
+ *                  detached (no gradient through lambda)
+ * The target p is detached: gradients flow to H_q and to W through z_q only.
+ *
+ * Masking and normalisation ("Streaming Cross Entropy"; "Correctness: alignment before
+ * chunking"): a row whose label equals ignore_index is masked and contributes 0 to the
+ * loss and to every gradient.  The library returns the masked loss SUM and the number of
+ * valid rows; the mean divides by the number of valid rows (never by a chunk count).
+ * With every row masked the mean is defined as 0 and every gradient is 0.
+ *
+ * Conventions shared by every entry point:
+ *   - Pointers to tensors are DEVICE pointers owned by the caller, on the current CUDA
+ *     device.  The library never allocates device memory: scratch lives in the caller's
+ *     `workspace` (size from slm_workspace_bytes, 256-byte aligned base).
+ *   - bf16 tensors are passed as `const void*` and are row-major, contiguous:
+ *     H_q, H_p [N, d]; W [V, d]; dH_q [N, d].  Every tensor base must be 16-byte aligned
+ *     and d must be a multiple of 8 (16-byte rows for the tensor-memory-access engine).
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  All work is enqueued
+ *     asynchronously on it; no entry point synchronises, except slm_device_status.
+ *   - Errors found on the host (null pointer, bad shape or alignment, small workspace,
+ *     wrong kind, unsupported GPU, CUDA launch error) are returned immediately and nothing
+ *     is enqueued.  Errors found on the device (a label outside [0, V) that is not
+ *     ignore_index, a pipeline wait that ran out of time) are recorded in the workspace
+ *     status word: the affected rows are treated as masked, and slm_device_status reports
+ *     the flag.  Kernels never trap.
+ */
+#ifndef SLM_H_
+#define SLM_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SLM_API __attribute__((visibility("default")))
+#else
+#define SLM_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum slm_loss_kind {
+  SLM_CE = 0,
+  SLM_KL = 1,
+  SLM_TV = 2,
+  SLM_NLA = 3,
+  SLM_LK_HYBRID = 4
+} slm_loss_kind;
+
+typedef enum slm_status {
+  SLM_OK = 0,
+  SLM_ERR_NULL = 1,             /* a required pointer is NULL                          */
+  SLM_ERR_SHAPE = 2,            /* N < 0, d <= 0, V <= 0, d % 8 != 0, or too large      */
+  SLM_ERR_ALIGN = 3,            /* a tensor base is not 16-byte aligned                  */
+  SLM_ERR_KIND = 4,             /* unknown loss kind                                     */
+  SLM_ERR_WORKSPACE = 5,        /* workspace NULL, misaligned or smaller than required  */
+  SLM_ERR_LABEL_RANGE = 6,      /* device: a CE label outside [0, V), row masked         */
+  SLM_ERR_TIMEOUT = 7,          /* device: a pipeline wait ran out of time               */
+  SLM_ERR_CUDA = 8,             /* a CUDA runtime call or launch failed                  */
+  SLM_ERR_UNSUPPORTED_ARCH = 9  /* the current device is not compute capability 10.0    */
+} slm_status;
+
+/* Library version as an integer (major * 10000 + minor * 100 + patch). */
+SLM_API int slm_version(void);
+
+/* Human-readable name of a status code (static string; never NULL). */
+SLM_API const char* slm_status_string(int status);
+
+/* Number of floats per token row of the `stats` array that slm_loss_fwd writes and
+ * slm_loss_bwd reads (layout [k][N], field-major):
+ *   SLM_CE: 1  (L_q = logsumexp z_q)
+ *   SLM_KL: 3  (L_q, L_p, KL)
+ *   SLM_TV, SLM_NLA, SLM_LK_HYBRID: 5  (L_q, L_p, KL, alpha, S = sum_{q_v < p_v} q_v)
+ * Returns 0 for an unknown kind. */
+SLM_API size_t slm_stats_floats(int kind);
+
+/* Bytes of workspace that slm_loss_fwd and slm_loss_bwd need for these sizes.
+ * chunk_tokens is the backward's token chunk (0 = automatic: min(N, 2d) rounded up to
+ * 128); the workspace then holds one bf16 [chunk, V] logits-gradient buffer, which is the
+ * streaming chunk buffer of "Backward pass".  Returns 0 on invalid arguments. */
+SLM_API size_t slm_workspace_bytes(int kind, int64_t N, int64_t d, int64_t V, int64_t chunk_tokens);
+
+/* Forward pass ("Streaming Cross Entropy"; "Available Losses").
+ *   Hq      bf16 [N, d]  draft hidden states (the hidden states for SLM_CE).
+ *   Hp      bf16 [N, d]  target hidden states; required for every kind but SLM_CE
+ *                        (ignored for SLM_CE, may be NULL there).
+ *   W       bf16 [V, d]  LM-head weight, shared by target and draft.
+ *   labels  int32 [N]    SLM_CE: the target token of each row, required; a value equal
+ *                        to ignore_index masks the row, any other value outside [0, V)
+ *                        sets SLM_ERR_LABEL_RANGE and masks the row.
+ *                        Other kinds: optional row mask (NULL = every row valid).
+ *   loss_tok   float [N]  per-token loss (0 on masked rows); may be NULL.
+ *   alpha_tok  float [N]  per-token alpha for TV / NLA / LK_HYBRID; may be NULL.
+ *   loss_sum   double [1] masked loss sum; required.
+ *   n_valid    int64 [1]  number of valid rows; required.
+ *   loss_mean  float [1]  loss_sum / n_valid (0 when n_valid = 0); may be NULL.
+ *   stats      float [slm_stats_floats(kind) * N] per-token statistics kept for the
+ *                        backward (layout above); required when N > 0.
+ *   workspace  device scratch of at least slm_workspace_bytes(kind, N, d, V, *) bytes.
+ * SLM_CE / SLM_KL make one pass of the LM-head GEMM over the vocabulary; the alpha-based
+ * kinds make two (alpha needs the final log-sum-exps). */
+SLM_API int slm_loss_fwd(int kind, const void* Hq, const void* Hp, const void* W,
+                 const int32_t* labels, int32_t ignore_index,
+                 int64_t N, int64_t d, int64_t V,
+                 float* loss_tok, float* alpha_tok, double* loss_sum, int64_t* n_valid,
+                 float* loss_mean, float* stats,
+                 void* workspace, size_t ws_bytes, void* stream);
+
+/* Backward pass ("Backward pass": per token chunk, recompute the logits, form the
+ * logits gradient, produce the chunk's hidden-state gradient and accumulate the LM-head
+ * gradient).  The upstream gradient of token n's loss is
+ *     g_n = valid_n * (grad_tok ? grad_tok[n] : 1) * (grad_scale ? *grad_scale : 1)
+ *           / (n_valid ? max(*n_valid, 1) : 1)
+ * so passing grad_tok = NULL, grad_scale = d(out)/d(mean) and the forward's n_valid gives
+ * the gradient of the mean loss.
+ *   grad_tok    float [N] or NULL;  grad_scale float [1] or NULL;  n_valid int64 [1] or NULL
+ *   stats       float [k * N] written by slm_loss_fwd for the same inputs.
+ *   dHq         bf16 [N, d]  overwritten with dLoss/dH_q.
+ *   dW          float [V, d] dLoss/dW; overwritten when accumulate_dW == 0, else added to.
+ *   chunk_tokens  token chunk of the streaming loop (0 = automatic, see above).
+ * There is no gradient for Hp (the target is detached). */
+SLM_API int slm_loss_bwd(int kind, const void* Hq, const void* Hp, const void* W,
+                 const int32_t* labels, int32_t ignore_index,
+                 int64_t N, int64_t d, int64_t V,
+                 const float* grad_tok, const float* grad_scale, const int64_t* n_valid,
+                 const float* stats, void* dHq, float* dW, int accumulate_dW,
+                 int64_t chunk_tokens, void* workspace, size_t ws_bytes, void* stream);
+
+/* Synchronises `stream`, then returns and clears the device status word of `workspace`:
+ * SLM_OK, SLM_ERR_LABEL_RANGE or SLM_ERR_TIMEOUT (the first found), or SLM_ERR_CUDA if
+ * the stream reported an error.  Every slm_loss_fwd / slm_loss_bwd call also clears the
+ * word when it starts, so the status describes the most recent call. */
+SLM_API int slm_device_status(const void* workspace, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SLM_H_ */

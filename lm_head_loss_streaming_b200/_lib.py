@@ -1,0 +1,118 @@
+"""ctypes binding of ``libslm.so`` (the C ABI declared in ``include/slm.h``).
+
+Argument marshalling only: every function here forwards plain integers (device
+addresses, sizes, a stream handle) to the C entry point of the same name and returns its
+status.  Loading fails loudly when the library has not been built: there is no fallback.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libslm.so")
+
+SLM_CE, SLM_KL, SLM_TV, SLM_NLA, SLM_LK_HYBRID = 0, 1, 2, 3, 4
+KIND = {"ce": SLM_CE, "kl_div": SLM_KL, "tv": SLM_TV, "nla": SLM_NLA,
+        "lk_hybrid": SLM_LK_HYBRID}
+
+SLM_OK = 0
+STATUS_NAMES = {
+    0: "SLM_OK", 1: "SLM_ERR_NULL", 2: "SLM_ERR_SHAPE", 3: "SLM_ERR_ALIGN",
+    4: "SLM_ERR_KIND", 5: "SLM_ERR_WORKSPACE", 6: "SLM_ERR_LABEL_RANGE",
+    7: "SLM_ERR_TIMEOUT", 8: "SLM_ERR_CUDA", 9: "SLM_ERR_UNSUPPORTED_ARCH",
+}
+
+# Every symbol the header declares, with (restype, argtypes).
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_I32 = ctypes.c_int32
+_INT = ctypes.c_int
+_SZ = ctypes.c_size_t
+SIGNATURES = {
+    "slm_version": (_INT, []),
+    "slm_status_string": (ctypes.c_char_p, [_INT]),
+    "slm_stats_floats": (_SZ, [_INT]),
+    "slm_workspace_bytes": (_SZ, [_INT, _I64, _I64, _I64, _I64]),
+    "slm_loss_fwd": (_INT, [_INT, _P, _P, _P, _P, _I32, _I64, _I64, _I64,
+                            _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "slm_loss_bwd": (_INT, [_INT, _P, _P, _P, _P, _I32, _I64, _I64, _I64,
+                            _P, _P, _P, _P, _P, _P, _INT, _I64, _P, _SZ, _P]),
+    "slm_device_status": (_INT, [_P, _P]),
+}
+
+
+class SLMError(RuntimeError):
+    def __init__(self, status, where=""):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)}" if where else status_string(status))
+
+
+_lib = None
+
+
+def load():
+    """Load ``libslm.so`` (raises if it is missing: there is no CPU fallback)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is not built; run `python -m lm_head_loss_streaming_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def status_string(status):
+    try:
+        return load().slm_status_string(int(status)).decode()
+    except ImportError:
+        return STATUS_NAMES.get(int(status), f"status {status}")
+
+
+def check(status, where=""):
+    if status != SLM_OK:
+        raise SLMError(status, where)
+    return status
+
+
+def slm_version():
+    return load().slm_version()
+
+
+def slm_status_string(status):
+    return load().slm_status_string(int(status)).decode()
+
+
+def slm_stats_floats(kind):
+    return load().slm_stats_floats(int(kind))
+
+
+def slm_workspace_bytes(kind, N, d, V, chunk_tokens=0):
+    return load().slm_workspace_bytes(int(kind), int(N), int(d), int(V), int(chunk_tokens))
+
+
+def slm_loss_fwd(kind, Hq, Hp, W, labels, ignore_index, N, d, V, loss_tok, alpha_tok,
+                 loss_sum, n_valid, loss_mean, stats, workspace, ws_bytes, stream):
+    return load().slm_loss_fwd(int(kind), Hq, Hp, W, labels, int(ignore_index), int(N),
+                               int(d), int(V), loss_tok, alpha_tok, loss_sum, n_valid,
+                               loss_mean, stats, workspace, int(ws_bytes), stream)
+
+
+def slm_loss_bwd(kind, Hq, Hp, W, labels, ignore_index, N, d, V, grad_tok, grad_scale,
+                 n_valid, stats, dHq, dW, accumulate_dW, chunk_tokens, workspace, ws_bytes,
+                 stream):
+    return load().slm_loss_bwd(int(kind), Hq, Hp, W, labels, int(ignore_index), int(N),
+                               int(d), int(V), grad_tok, grad_scale, n_valid, stats, dHq, dW,
+                               int(accumulate_dW), int(chunk_tokens), workspace,
+                               int(ws_bytes), stream)
+
+
+def slm_device_status(workspace, stream):
+    return load().slm_device_status(workspace, stream)

@@ -1,0 +1,350 @@
+// slm_api.cu - the C ABI of the streaming LM-head loss (declared in include/slm.h).
+//
+// Host-side orchestration only: argument validation, workspace carving, TMA tensor-map
+// encoding and the launch sequence.  All arithmetic runs in the kernels of
+// slm_kernels.cu.  Nothing here allocates device memory or synchronises (except
+// slm_device_status).
+//
+// Launch sequence ("Training speculative decoders: removing the logits and attention
+// bottlenecks", "Streaming Cross Entropy" and "Backward pass"):
+//   forward   memset(status) -> LM-head GEMM with the online softmax-statistics epilogue
+//             (vocabulary-tiled, one pass for CE / KL) -> per-row combine -> [alpha
+//             losses: second GEMM pass for alpha and S -> combine] -> fixed-order loss
+//             reduction (loss_sum, n_valid, mean).
+//   backward  for each token chunk: GEMM recompute of the chunk's logits with the
+//             logits-gradient epilogue (bf16 chunk buffer) -> dH = dZ W -> dW (+)= dZ^T H.
+
+#include <stdio.h>
+#include <string.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "../../include/slm.h"
+#include "slm_internal.h"
+
+namespace slm {
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr long long kTimeoutCycles = 4000000000LL;  // ~2 s at the B200's boost clock
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+bool valid_kind(int k) { return k >= SLM_CE && k <= SLM_LK_HYBRID; }
+bool dual_kind(int k) { return k != SLM_CE; }
+bool alpha_kind(int k) { return k == SLM_TV || k == SLM_NLA || k == SLM_LK_HYBRID; }
+
+// Forward vocabulary schedule: tiles of BN columns, grouped into at most 64 runs per row
+// (so the per-row partials stay O(N)), each run at least 2048 columns long.
+struct FwdSched {
+  int bn, num_n, vc, units_n, fields;
+};
+
+FwdSched fwd_sched(int kind, int64_t V) {
+  FwdSched f;
+  f.bn = dual_kind(kind) ? kBnDual : kBnSingle;
+  f.num_n = static_cast<int>(ceil_div(V, f.bn));
+  const int min_vc = 2048 / f.bn;
+  f.vc = std::max<int>(min_vc, static_cast<int>(ceil_div(f.num_n, 64)));
+  f.vc = std::min(f.vc, f.num_n);
+  f.units_n = static_cast<int>(ceil_div(f.num_n, f.vc));
+  f.fields = dual_kind(kind) ? 5 : 2;
+  return f;
+}
+
+int64_t default_chunk(int64_t N, int64_t d, int64_t chunk_tokens) {
+  if (N <= 0) return 0;
+  int64_t c = chunk_tokens > 0 ? chunk_tokens : align_up(static_cast<size_t>(2 * d), kBM);
+  return std::max<int64_t>(1, std::min<int64_t>(c, N));
+}
+
+struct Layout {
+  size_t status_off, red_off, nblk, big_off, part_off, zy_off, dz_off, ldz, total;
+};
+
+Layout layout(int kind, int64_t N, int64_t d, int64_t V, int64_t chunk_tokens) {
+  Layout L{};
+  L.status_off = 0;
+  L.nblk = static_cast<size_t>(std::max<int64_t>(1, ceil_div(N, kCombineThreads)));
+  L.red_off = kAlign;
+  size_t off = align_up(L.red_off + L.nblk * (sizeof(double) + sizeof(long long)), kAlign);
+  L.big_off = off;
+  const FwdSched f = fwd_sched(kind, V);
+  const size_t part = static_cast<size_t>(f.units_n) * f.fields * static_cast<size_t>(N) * 4;
+  L.part_off = off;
+  L.zy_off = align_up(L.part_off + part, kAlign);
+  const size_t fwd_end = align_up(L.zy_off + static_cast<size_t>(N) * 4, kAlign);
+  L.ldz = align_up(static_cast<size_t>(V), 8);
+  L.dz_off = off;  // the backward's chunk buffer reuses the forward's partials region
+  const size_t bwd_end =
+      align_up(L.dz_off + static_cast<size_t>(default_chunk(N, d, chunk_tokens)) * L.ldz * 2,
+               kAlign);
+  L.total = std::max(fwd_end, bwd_end);
+  return L;
+}
+
+// ---------------------------------------------------------------------------------------
+// Device checks and tensor maps.
+// ---------------------------------------------------------------------------------------
+int check_device() {
+  static int cache[64];
+  static std::once_flag once;
+  std::call_once(once, [] {
+    for (int i = 0; i < 64; ++i) cache[i] = -1;
+  });
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return SLM_ERR_CUDA;
+  if (cache[dev] < 0) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return SLM_ERR_CUDA;
+    cache[dev] = (major == 10 && minor == 0) ? SLM_OK : SLM_ERR_UNSUPPORTED_ARCH;
+  }
+  return cache[dev];
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 tensor map over a row-major [outer, inner] matrix with `ld` elements per row;
+// box {box_inner, box_outer}, 128-byte swizzle, zero fill out of bounds.
+bool make_map(CUtensorMap* m, const void* base, int64_t inner, int64_t outer, int64_t ld,
+              int box_inner, int box_outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(outer)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(box_inner), static_cast<cuuint32_t>(box_outer)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool misaligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) != 0; }
+
+GemmGeom geom(int64_t M, int64_t Nn, int64_t K, int bn, int vc, int group_m) {
+  GemmGeom g;
+  g.num_m = static_cast<int>(ceil_div(M, kBM));
+  g.num_n = static_cast<int>(ceil_div(Nn, bn));
+  g.k_blocks = static_cast<int>(ceil_div(K, kBK));
+  g.vc = std::max(1, std::min(vc, g.num_n));
+  g.group_m = std::max(1, std::min(group_m, g.num_m));
+  g.units_n = static_cast<int>(ceil_div(g.num_n, g.vc));
+  g.num_units = g.num_m * g.units_n;
+  return g;
+}
+
+int grid_for(const GemmGeom& g) {
+  const int sms = sm_count();
+  return std::max(1, std::min(g.num_units, sms > 0 ? sms : 148));
+}
+
+int common_checks(int kind, const void* Hq, const void* Hp, const void* W, const int32_t* labels,
+                  int64_t N, int64_t d, int64_t V, const void* workspace, size_t ws_bytes,
+                  int64_t chunk_tokens) {
+  if (!valid_kind(kind)) return SLM_ERR_KIND;
+  if (N < 0 || d <= 0 || V <= 0 || (d % 8) != 0) return SLM_ERR_SHAPE;
+  if (N >= (int64_t(1) << 31) || V >= (int64_t(1) << 31) || d >= (int64_t(1) << 31))
+    return SLM_ERR_SHAPE;
+  if (!W || !workspace) return SLM_ERR_NULL;
+  if (N > 0) {
+    if (!Hq) return SLM_ERR_NULL;
+    if (dual_kind(kind) && !Hp) return SLM_ERR_NULL;
+    if (kind == SLM_CE && !labels) return SLM_ERR_NULL;
+  }
+  if (misaligned(W, 16) || (Hq && misaligned(Hq, 16)) || (dual_kind(kind) && Hp && misaligned(Hp, 16)))
+    return SLM_ERR_ALIGN;
+  if (misaligned(workspace, kAlign)) return SLM_ERR_WORKSPACE;
+  if (ws_bytes < layout(kind, N, d, V, chunk_tokens).total) return SLM_ERR_WORKSPACE;
+  return SLM_OK;
+}
+
+#define SLM_TRY_CUDA(expr)                  \
+  do {                                      \
+    if ((expr) != cudaSuccess) return SLM_ERR_CUDA; \
+  } while (0)
+
+}  // namespace
+}  // namespace slm
+
+using namespace slm;
+
+extern "C" {
+
+int slm_version(void) { return 100; }
+
+const char* slm_status_string(int s) {
+  switch (s) {
+    case SLM_OK: return "SLM_OK";
+    case SLM_ERR_NULL: return "SLM_ERR_NULL: a required pointer is NULL";
+    case SLM_ERR_SHAPE: return "SLM_ERR_SHAPE: invalid N, d or V (d must be a positive multiple of 8)";
+    case SLM_ERR_ALIGN: return "SLM_ERR_ALIGN: a tensor base is not 16-byte aligned";
+    case SLM_ERR_KIND: return "SLM_ERR_KIND: unknown loss kind";
+    case SLM_ERR_WORKSPACE: return "SLM_ERR_WORKSPACE: workspace NULL, misaligned or too small";
+    case SLM_ERR_LABEL_RANGE: return "SLM_ERR_LABEL_RANGE: a label outside [0, V) (row masked)";
+    case SLM_ERR_TIMEOUT: return "SLM_ERR_TIMEOUT: a device pipeline wait ran out of time";
+    case SLM_ERR_CUDA: return "SLM_ERR_CUDA: a CUDA call or launch failed";
+    case SLM_ERR_UNSUPPORTED_ARCH: return "SLM_ERR_UNSUPPORTED_ARCH: needs compute capability 10.0 (B200)";
+    default: return "SLM: unknown status";
+  }
+}
+
+size_t slm_stats_floats(int kind) {
+  if (!valid_kind(kind)) return 0;
+  if (kind == SLM_CE) return 1;
+  if (kind == SLM_KL) return 3;
+  return 5;
+}
+
+size_t slm_workspace_bytes(int kind, int64_t N, int64_t d, int64_t V, int64_t chunk_tokens) {
+  if (!valid_kind(kind) || N < 0 || d <= 0 || V <= 0 || (d % 8) != 0) return 0;
+  return layout(kind, N, d, V, chunk_tokens).total;
+}
+
+int slm_loss_fwd(int kind, const void* Hq, const void* Hp, const void* W, const int32_t* labels,
+                 int32_t ignore_index, int64_t N, int64_t d, int64_t V, float* loss_tok,
+                 float* alpha_tok, double* loss_sum, int64_t* n_valid, float* loss_mean,
+                 float* stats, void* workspace, size_t ws_bytes, void* stream) {
+  int st = common_checks(kind, Hq, Hp, W, labels, N, d, V, workspace, ws_bytes, 0);
+  if (st != SLM_OK) return st;
+  if (!loss_sum || !n_valid || (N > 0 && !stats)) return SLM_ERR_NULL;
+  if ((st = check_device()) != SLM_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const Layout L = layout(kind, N, d, V, 0);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int* status = reinterpret_cast<int*>(ws + L.status_off);
+  double* blk_sum = reinterpret_cast<double*>(ws + L.red_off);
+  long long* blk_cnt = reinterpret_cast<long long*>(blk_sum + L.nblk);
+  float* part = reinterpret_cast<float*>(ws + L.part_off);
+  float* zy = reinterpret_cast<float*>(ws + L.zy_off);
+  SLM_TRY_CUDA(cudaMemsetAsync(status, 0, sizeof(int), s));
+  const DevCtl ctl{status, kTimeoutCycles};
+
+  if (N > 0) {
+    const FwdSched f = fwd_sched(kind, V);
+    const GemmGeom g = geom(N, V, d, f.bn, f.vc, 16);
+    CUtensorMap tHq, tHp, tW;
+    if (!make_map(&tHq, Hq, d, N, d, kBK, kBM)) return SLM_ERR_CUDA;
+    if (!make_map(&tW, W, d, V, d, kBK, f.bn)) return SLM_ERR_CUDA;
+    FwdParams p{labels, ignore_index, N, V, part, zy, stats};
+    const int grid = grid_for(g);
+    if (!dual_kind(kind)) {
+      SLM_TRY_CUDA(launch_fwd_ce(tHq, tW, g, p, ctl, grid, s));
+    } else {
+      if (!make_map(&tHp, Hp, d, N, d, kBK, kBM)) return SLM_ERR_CUDA;
+      SLM_TRY_CUDA(launch_fwd_dual(tHq, tHp, tW, g, p, ctl, grid, s));
+    }
+    SLM_TRY_CUDA(launch_combine(kind, 1, part, f.units_n, zy, labels, ignore_index, N, V,
+                                loss_tok, alpha_tok, stats, blk_sum, blk_cnt, status, s));
+    if (alpha_kind(kind)) {
+      SLM_TRY_CUDA(launch_alpha(tHq, tHp, tW, g, p, ctl, grid, s));
+      SLM_TRY_CUDA(launch_combine(kind, 2, part, f.units_n, zy, labels, ignore_index, N, V,
+                                  loss_tok, alpha_tok, stats, blk_sum, blk_cnt, status, s));
+    }
+    SLM_TRY_CUDA(launch_finalize(blk_sum, blk_cnt, static_cast<int>(L.nblk), loss_sum, n_valid,
+                                 loss_mean, s));
+  } else {
+    SLM_TRY_CUDA(cudaMemsetAsync(blk_sum, 0, L.nblk * (sizeof(double) + sizeof(long long)), s));
+    SLM_TRY_CUDA(launch_finalize(blk_sum, blk_cnt, static_cast<int>(L.nblk), loss_sum, n_valid,
+                                 loss_mean, s));
+  }
+  return SLM_OK;
+}
+
+int slm_loss_bwd(int kind, const void* Hq, const void* Hp, const void* W, const int32_t* labels,
+                 int32_t ignore_index, int64_t N, int64_t d, int64_t V, const float* grad_tok,
+                 const float* grad_scale, const int64_t* n_valid, const float* stats, void* dHq,
+                 float* dW, int accumulate_dW, int64_t chunk_tokens, void* workspace,
+                 size_t ws_bytes, void* stream) {
+  int st = common_checks(kind, Hq, Hp, W, labels, N, d, V, workspace, ws_bytes, chunk_tokens);
+  if (st != SLM_OK) return st;
+  if (!dW || (N > 0 && (!dHq || !stats))) return SLM_ERR_NULL;
+  if ((N > 0 && misaligned(dHq, 16)) || misaligned(dW, 16)) return SLM_ERR_ALIGN;
+  if ((st = check_device()) != SLM_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const Layout L = layout(kind, N, d, V, chunk_tokens);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int* status = reinterpret_cast<int*>(ws + L.status_off);
+  __nv_bfloat16* dz = reinterpret_cast<__nv_bfloat16*>(ws + L.dz_off);
+  SLM_TRY_CUDA(cudaMemsetAsync(status, 0, sizeof(int), s));
+  const DevCtl ctl{status, kTimeoutCycles};
+
+  if (N == 0) {
+    if (!accumulate_dW) SLM_TRY_CUDA(launch_zero_f32(dW, V * d, s));
+    return SLM_OK;
+  }
+  const int64_t C = default_chunk(N, d, chunk_tokens);
+  const FwdSched f = fwd_sched(kind, V);
+  CUtensorMap tW_k, tW_mn;
+  if (!make_map(&tW_k, W, d, V, d, kBK, f.bn)) return SLM_ERR_CUDA;
+  if (!make_map(&tW_mn, W, d, V, d, 64, 64)) return SLM_ERR_CUDA;
+  const int64_t ldz = static_cast<int64_t>(L.ldz);
+
+  for (int64_t c0 = 0; c0 < N; c0 += C) {
+    const int64_t rows = std::min<int64_t>(C, N - c0);
+    const __nv_bfloat16* hq = static_cast<const __nv_bfloat16*>(Hq) + c0 * d;
+    // 1) Recompute the chunk's logits and write its logits gradient dZ [rows, V] (bf16).
+    CUtensorMap tHq, tHp;
+    if (!make_map(&tHq, hq, d, rows, d, kBK, kBM)) return SLM_ERR_CUDA;
+    const GemmGeom gz = geom(rows, V, d, f.bn, f.vc, 16);
+    DzParams pz{kind, labels, ignore_index, c0, rows, N, V, stats, grad_tok, grad_scale,
+                n_valid, dz, ldz};
+    if (!dual_kind(kind)) {
+      SLM_TRY_CUDA(launch_dz_ce(tHq, tW_k, gz, pz, ctl, grid_for(gz), s));
+    } else {
+      const __nv_bfloat16* hp = static_cast<const __nv_bfloat16*>(Hp) + c0 * d;
+      if (!make_map(&tHp, hp, d, rows, d, kBK, kBM)) return SLM_ERR_CUDA;
+      SLM_TRY_CUDA(launch_dz_dual(tHq, tHp, tW_k, gz, pz, ctl, grid_for(gz), s));
+    }
+    // 2) dH[chunk] = dZ W   (M = rows, N = d, K = V; W read MN-major).
+    CUtensorMap tDz_k, tDz_mn, tH_mn;
+    if (!make_map(&tDz_k, dz, V, rows, ldz, kBK, kBM)) return SLM_ERR_CUDA;
+    const GemmGeom gh = geom(rows, d, V, kBnGrad, 1, 1);
+    DhParams ph{static_cast<__nv_bfloat16*>(dHq), c0, rows, d};
+    SLM_TRY_CUDA(launch_dh(tDz_k, tW_mn, gh, ph, ctl, grid_for(gh), s));
+    // 3) dW (+)= dZ^T H[chunk]   (M = V, N = d, K = rows; both operands MN-major).
+    if (!make_map(&tDz_mn, dz, V, rows, ldz, 64, 64)) return SLM_ERR_CUDA;
+    if (!make_map(&tH_mn, hq, d, rows, d, 64, 64)) return SLM_ERR_CUDA;
+    const GemmGeom gw = geom(V, d, rows, kBnGrad, 1, 1);
+    DwParams pw{dW, V, d, (accumulate_dW || c0 > 0) ? 1 : 0};
+    SLM_TRY_CUDA(launch_dw(tDz_mn, tH_mn, gw, pw, ctl, grid_for(gw), s));
+  }
+  return SLM_OK;
+}
+
+int slm_device_status(const void* workspace, void* stream) {
+  if (!workspace) return SLM_ERR_NULL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return SLM_ERR_CUDA;
+  int flags = 0;
+  int* status = reinterpret_cast<int*>(const_cast<void*>(workspace));
+  if (cudaMemcpy(&flags, status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return SLM_ERR_CUDA;
+  if (flags != 0 && cudaMemset(status, 0, sizeof(int)) != cudaSuccess) return SLM_ERR_CUDA;
+  if (flags & kFlagTimeout) return SLM_ERR_TIMEOUT;
+  if (flags & kFlagLabelRange) return SLM_ERR_LABEL_RANGE;
+  return SLM_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,117 @@
+// slm_internal.h - types shared by the host orchestrator (slm_api.cu) and the kernels
+// (slm_kernels.cu).  Not part of the public ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace slm {
+
+// Tile shape of every GEMM: 128 rows of the M operand per CTA tile (one TMEM lane per
+// row), 64 bf16 of K per pipeline stage (one 128-byte swizzle row).
+constexpr int kBM = 128;
+constexpr int kBK = 64;
+constexpr int kStages = 4;
+constexpr int kThreads = 192;  // warp 0: TMA producer, warp 1: MMA issuer, warps 2-5: epilogue
+
+// N tile of the forward / logits-gradient GEMMs: 256 vocabulary columns with one
+// accumulator (CE), 128 columns with two accumulators (target and draft logits).
+constexpr int kBnSingle = 256;
+constexpr int kBnDual = 128;
+constexpr int kBnGrad = 256;  // dH and dW GEMMs
+
+// Device status word bits.
+constexpr int kFlagLabelRange = 1;
+constexpr int kFlagTimeout = 2;
+
+enum LossKind : int { kCE = 0, kKL = 1, kTV = 2, kNLA = 3, kLK = 4 };
+
+// Persistent tile schedule.  Work units are (M tile, run of `vc` consecutive N tiles);
+// units are ordered in groups of `group_m` M tiles: for each N run, every M tile of the
+// group, so that CTAs running at the same time share the N-operand tiles in L2.
+struct GemmGeom {
+  int num_m;      // M tiles
+  int num_n;      // N tiles
+  int k_blocks;   // K blocks of kBK
+  int vc;         // N tiles per unit
+  int group_m;    // M tiles per raster group
+  int units_n;    // ceil(num_n / vc)
+  int num_units;  // num_m * units_n
+};
+
+struct DevCtl {
+  int* status;               // device status word (in the workspace)
+  long long timeout_cycles;  // bound of every pipeline wait
+};
+
+// Forward statistics (pass 1) and the alpha pass (pass 2).
+struct FwdParams {
+  const int32_t* labels;  // CE labels (required for CE)
+  int32_t ignore_index;
+  int64_t N, V;
+  float* part;         // [units_n][fields][N]
+  float* zy;           // [N] label logit (CE)
+  const float* stats;  // pass 2: L_q, L_p
+};
+
+// Logits-gradient tile (backward recompute + dZ epilogue).
+struct DzParams {
+  int kind;
+  const int32_t* labels;
+  int32_t ignore_index;
+  int64_t row0, rows;  // token chunk [row0, row0 + rows)
+  int64_t N, V;
+  const float* stats;
+  const float* grad_tok;
+  const float* grad_scale;
+  const int64_t* n_valid;
+  __nv_bfloat16* dz;  // [rows][ldz]
+  int64_t ldz;
+};
+
+struct DhParams {
+  __nv_bfloat16* dH;  // [N][d]
+  int64_t row0, rows, d;
+};
+
+struct DwParams {
+  float* dW;  // [V][d]
+  int64_t V, d;
+  int beta;  // 1: add to dW, 0: overwrite
+};
+
+// Kernel launchers (slm_kernels.cu).  Each returns cudaGetLastError() after the launch.
+int sm_count();
+cudaError_t launch_fwd_ce(const CUtensorMap& tH, const CUtensorMap& tW, const GemmGeom& g,
+                          const FwdParams& p, const DevCtl& c, int grid, cudaStream_t s);
+cudaError_t launch_fwd_dual(const CUtensorMap& tHq, const CUtensorMap& tHp,
+                            const CUtensorMap& tW, const GemmGeom& g, const FwdParams& p,
+                            const DevCtl& c, int grid, cudaStream_t s);
+cudaError_t launch_alpha(const CUtensorMap& tHq, const CUtensorMap& tHp, const CUtensorMap& tW,
+                         const GemmGeom& g, const FwdParams& p, const DevCtl& c, int grid,
+                         cudaStream_t s);
+cudaError_t launch_dz_ce(const CUtensorMap& tH, const CUtensorMap& tW, const GemmGeom& g,
+                         const DzParams& p, const DevCtl& c, int grid, cudaStream_t s);
+cudaError_t launch_dz_dual(const CUtensorMap& tHq, const CUtensorMap& tHp, const CUtensorMap& tW,
+                           const GemmGeom& g, const DzParams& p, const DevCtl& c, int grid,
+                           cudaStream_t s);
+cudaError_t launch_dh(const CUtensorMap& tDz, const CUtensorMap& tW, const GemmGeom& g,
+                      const DhParams& p, const DevCtl& c, int grid, cudaStream_t s);
+cudaError_t launch_dw(const CUtensorMap& tDzT, const CUtensorMap& tH, const GemmGeom& g,
+                      const DwParams& p, const DevCtl& c, int grid, cudaStream_t s);
+
+// Row combines and the deterministic loss reduction.
+cudaError_t launch_combine(int kind, int pass, const float* part, int nch, const float* zy,
+                           const int32_t* labels, int32_t ignore_index, int64_t N, int64_t V,
+                           float* loss_tok, float* alpha_tok, float* stats, double* blk_sum,
+                           long long* blk_cnt, int* status, cudaStream_t s);
+cudaError_t launch_finalize(const double* blk_sum, const long long* blk_cnt, int nblk,
+                            double* loss_sum, int64_t* n_valid, float* loss_mean,
+                            cudaStream_t s);
+cudaError_t launch_zero_f32(float* p, int64_t n, cudaStream_t s);
+
+constexpr int kCombineThreads = 256;
+
+}  // namespace slm

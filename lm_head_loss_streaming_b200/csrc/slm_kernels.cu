@@ -1,0 +1,881 @@
+// slm_kernels.cu - sm_100a kernels of the streaming LM-head loss.
+//
+// One warp-specialised persistent GEMM skeleton serves every contraction of the path:
+//   warp 0      TMA producer: 2-D tiled loads of the A / B operand tiles into a 4-stage
+//               shared-memory ring (128-byte swizzle), completion on "full" mbarriers;
+//   warp 1      MMA issuer: one lane issues tcgen05.mma (bf16 x bf16 -> fp32) into one of
+//               two TMEM accumulator buffers; tcgen05.commit frees ring stages and
+//               publishes finished accumulators;
+//   warps 2-5   epilogue: one thread per tile row reads its row from TMEM (tcgen05.ld)
+//               and applies the fused epilogue while the MMA warp fills the other buffer.
+// The epilogues are what make the path streaming ("Training speculative decoders:
+// removing the logits and attention bottlenecks", "Streaming Cross Entropy" and
+// "Backward pass"): logits tiles live only in TMEM and registers.
+//   EpiFwdCE    online row max / sum of exp and the label logit          (CE forward)
+//   EpiFwdDual  the same for target and draft plus the KL accumulator    (KL forward,
+//               first pass of the alpha losses)
+//   EpiAlpha    alpha = sum min(p, q) and S = sum_{q<p} q                 (second pass)
+//   EpiDz       the logits gradient, rounded to bf16 into the chunk buffer (backward)
+//   EpiDh       dH chunk rows (bf16)                                      (dH = dZ W)
+//   EpiDw       fp32 read-add-write of disjoint dW tiles, no atomics      (dW += dZ^T H)
+// Every pipeline wait is bounded: on expiry the kernel records kFlagTimeout, lets its own
+// copies and MMAs finish, frees TMEM and returns.
+
+#include <math.h>
+
+#include "slm_internal.h"
+#include "sm100.cuh"
+
+namespace slm {
+using namespace sm100;
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr uint32_t kTmemCols = 512;
+
+struct PipeCtl {
+  uint64_t full[kStages];
+  uint64_t empty[kStages];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint64_t fin;
+  uint32_t tmem_base;
+  int abort;
+};
+
+// Bounded wait executed by all 32 lanes of a warp; the result is warp-uniform.
+// honor_abort = false is used for the final waits on a CTA's own in-flight work.
+__device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          const DevCtl& ctl, bool honor_abort = true) {
+  const uint32_t a = smem_u32(bar);
+  bool done = mbar_try_wait(a, parity);
+  if (!done) {
+    const long long t0 = clock64();
+    while (true) {
+      done = mbar_try_wait(a, parity);
+      if (done) break;
+      if (honor_abort && *abort) break;
+      if (clock64() - t0 > ctl.timeout_cycles) {
+        *abort = 1;
+        atomicOr(ctl.status, kFlagTimeout);
+        break;
+      }
+    }
+  }
+  return __all_sync(0xffffffffu, done);
+}
+
+__device__ __forceinline__ void unit_coords(const GemmGeom& g, int u, int& mt, int& j) {
+  const int per_group = g.group_m * g.units_n;
+  const int grp = u / per_group;
+  const int r = u - grp * per_group;
+  const int gm = min(g.group_m, g.num_m - grp * g.group_m);
+  j = r / gm;
+  mt = grp * g.group_m + (r - j * gm);
+}
+
+// ----------------------------------------------------------------------------------------
+// The GEMM skeleton.  A: NUM_A operands of 128 x kBK per stage (K-major: box {64, 128};
+// MN-major: two boxes {64, 64}); B: BN x kBK (K-major: box {64, BN}; MN-major: BN/64
+// boxes {64, 64}).  Accumulator a of buffer b sits at TMEM columns (b * NUM_A + a) * BN.
+// ----------------------------------------------------------------------------------------
+template <int BN, int NUM_A, bool A_MN, bool B_MN, class Epi>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
+                const __grid_constant__ CUtensorMap tmB, const GemmGeom g,
+                const typename Epi::Params ep, const DevCtl ctl) {
+  constexpr uint32_t kABytes = kBM * kBK * 2;
+  constexpr uint32_t kBBytes = BN * kBK * 2;
+  constexpr uint32_t kStageBytes = NUM_A * kABytes + kBBytes;
+  constexpr uint32_t kAccCols = NUM_A * BN;
+  static_assert(2 * kAccCols <= kTmemCols, "two accumulator buffers must fit in TMEM");
+  static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "UMMA N");
+  constexpr uint32_t kIdesc = idesc_bf16_f32(kBM, BN, A_MN, B_MN);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  PipeCtl* pc = reinterpret_cast<PipeCtl*>(smem + kStages * kStageBytes);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&pc->full[s], 1);
+      mbar_init(&pc->empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&pc->tfull[b], 1);
+      mbar_init(&pc->tempty[b], 4 * 32);
+    }
+    mbar_init(&pc->fin, 1);
+    pc->abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA0);
+    if (NUM_A == 2) tma_prefetch_desc(&tmA1);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(&pc->tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = pc->tmem_base;
+  volatile int* abort = &pc->abort;
+
+  if (warp == 0) {
+    // ------------------------------ TMA producer ------------------------------
+    uint32_t it = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; ok && u < g.num_units; u += gridDim.x) {
+      int mt, j;
+      unit_coords(g, u, mt, j);
+      const int n_end = min((j + 1) * g.vc, g.num_n);
+      for (int nt = j * g.vc; ok && nt < n_end; ++nt) {
+        for (int kb = 0; kb < g.k_blocks; ++kb, ++it) {
+          const int s = it % kStages;
+          const uint32_t ph = (it / kStages) & 1u;
+          if (!wait_warp(&pc->empty[s], ph ^ 1u, abort, ctl)) {
+            ok = false;
+            break;
+          }
+          if (lane == 0) {
+            uint8_t* st = smem + s * kStageBytes;
+            mbar_arrive_expect_tx(&pc->full[s], kStageBytes);
+            const int k0 = kb * kBK;
+#pragma unroll
+            for (int a = 0; a < NUM_A; ++a) {
+              const CUtensorMap* map = (a == 0) ? &tmA0 : &tmA1;
+              uint8_t* dst = st + a * kABytes;
+              if (A_MN) {
+                tma_load_2d(dst, map, &pc->full[s], mt * kBM, k0);
+                tma_load_2d(dst + 8192, map, &pc->full[s], mt * kBM + 64, k0);
+              } else {
+                tma_load_2d(dst, map, &pc->full[s], k0, mt * kBM);
+              }
+            }
+            uint8_t* bdst = st + NUM_A * kABytes;
+            if (B_MN) {
+#pragma unroll
+              for (int jb = 0; jb < BN / 64; ++jb)
+                tma_load_2d(bdst + jb * 8192, &tmB, &pc->full[s], nt * BN + jb * 64, k0);
+            } else {
+              tma_load_2d(bdst, &tmB, &pc->full[s], k0, nt * BN);
+            }
+          }
+          __syncwarp();
+        }
+      }
+    }
+    if (!ok) {
+      // Let this CTA's own copies in flight land before the CTA exits.
+      const uint32_t first = it > (uint32_t)kStages ? it - kStages : 0u;
+      for (uint32_t i = first; i < it; ++i)
+        wait_warp(&pc->full[i % kStages], (i / kStages) & 1u, abort, ctl, false);
+    }
+  } else if (warp == 1) {
+    // ------------------------------ MMA issuer ------------------------------
+    uint32_t it = 0, t = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; ok && u < g.num_units; u += gridDim.x) {
+      int mt, j;
+      unit_coords(g, u, mt, j);
+      const int n_end = min((j + 1) * g.vc, g.num_n);
+      for (int nt = j * g.vc; ok && nt < n_end; ++nt, ++t) {
+        const int b = t & 1;
+        const uint32_t ub = (t >> 1) & 1u;
+        if (!wait_warp(&pc->tempty[b], ub ^ 1u, abort, ctl)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t dcol = tmem + b * kAccCols;
+        for (int kb = 0; kb < g.k_blocks; ++kb, ++it) {
+          const int s = it % kStages;
+          const uint32_t ph = (it / kStages) & 1u;
+          if (!wait_warp(&pc->full[s], ph, abort, ctl)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (lane == 0) {
+            const uint32_t a_addr = smem_u32(smem + s * kStageBytes);
+            const uint32_t b_addr = a_addr + NUM_A * kABytes;
+#pragma unroll
+            for (int kk = 0; kk < kBK / 16; ++kk) {
+              const uint64_t bd = B_MN ? smem_desc_sw128(b_addr + kk * 2048, 8192, 1024)
+                                       : smem_desc_sw128(b_addr + kk * 32, 16, 1024);
+#pragma unroll
+              for (int a = 0; a < NUM_A; ++a) {
+                const uint32_t aa = a_addr + a * kABytes;
+                const uint64_t ad = A_MN ? smem_desc_sw128(aa + kk * 2048, 8192, 1024)
+                                         : smem_desc_sw128(aa + kk * 32, 16, 1024);
+                umma_bf16(dcol + a * BN, ad, bd, kIdesc, (kb | kk) != 0 ? 1u : 0u);
+              }
+            }
+            umma_commit(&pc->empty[s]);
+          }
+          __syncwarp();
+        }
+        if (!ok) break;
+        if (lane == 0) umma_commit(&pc->tfull[b]);
+        __syncwarp();
+      }
+    }
+    // Every MMA this thread issued must be complete before TMEM is released.
+    if (lane == 0) umma_commit(&pc->fin);
+    __syncwarp();
+    wait_warp(&pc->fin, 0u, abort, ctl, false);
+  } else {
+    // ------------------------------ epilogue ------------------------------
+    const int q = warp & 3;  // a warp may only touch TMEM lanes [32 * (warp % 4), +32)
+    const int row = q * 32 + lane;
+    const uint32_t lane_bits = static_cast<uint32_t>(q * 32) << 16;
+    Epi epi;
+    uint32_t t = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; ok && u < g.num_units; u += gridDim.x) {
+      int mt, j;
+      unit_coords(g, u, mt, j);
+      const int n_end = min((j + 1) * g.vc, g.num_n);
+      epi.unit_begin(ep, mt, j, row);
+      for (int nt = j * g.vc; nt < n_end; ++nt, ++t) {
+        const int b = t & 1;
+        const uint32_t ub = (t >> 1) & 1u;
+        if (!wait_warp(&pc->tfull[b], ub, abort, ctl)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        epi.template tile<BN>(ep, tmem + lane_bits + b * kAccCols, mt, nt, row);
+        tc_fence_before();
+        mbar_arrive(&pc->tempty[b]);
+      }
+      if (!ok) break;
+      epi.unit_end(ep, mt, j, row);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+}
+
+// ----------------------------------------------------------------------------------------
+// Epilogues.
+// ----------------------------------------------------------------------------------------
+__device__ __forceinline__ float max32(const float (&v)[32]) {
+  float m0 = fmaxf(v[0], v[1]), m1 = fmaxf(v[2], v[3]);
+#pragma unroll
+  for (int i = 4; i < 32; i += 4) {
+    m0 = fmaxf(m0, fmaxf(v[i], v[i + 1]));
+    m1 = fmaxf(m1, fmaxf(v[i + 2], v[i + 3]));
+  }
+  return fmaxf(m0, m1);
+}
+
+__device__ __forceinline__ void mask_tail(float (&v)[32], int64_t col0, int64_t V) {
+#pragma unroll
+  for (int i = 0; i < 32; ++i)
+    if (col0 + i >= V) v[i] = -INFINITY;
+}
+
+// CE forward: per row, online max m (log2 units) and s = sum 2^(z log2e - m) over the
+// unit's vocabulary run, plus the label logit z_y when the label falls in the run.
+struct EpiFwdCE {
+  using Params = FwdParams;
+  float m, s, zyv;
+  int32_t lab;
+  bool has_zy, row_ok;
+  int64_t grow;
+
+  __device__ __forceinline__ void unit_begin(const Params& p, int mt, int, int row) {
+    m = -INFINITY;
+    s = 0.f;
+    has_zy = false;
+    zyv = 0.f;
+    grow = static_cast<int64_t>(mt) * kBM + row;
+    row_ok = grow < p.N;
+    lab = row_ok ? p.labels[grow] : -1;
+  }
+
+  template <int BN>
+  __device__ __forceinline__ void tile(const Params& p, uint32_t tb, int, int nt, int) {
+    const int64_t n0 = static_cast<int64_t>(nt) * BN;
+    const int64_t rel = static_cast<int64_t>(lab) - n0;
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 32) {
+      float v[32];
+      tmem_ld32(tb + c, v);
+      tmem_ld_wait();
+      if (n0 + c + 32 > p.V) mask_tail(v, n0 + c, p.V);
+      if (static_cast<uint64_t>(rel - c) < 32u) {
+        const int o = static_cast<int>(rel - c);
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          if (i == o) zyv = v[i];
+        has_zy = true;
+      }
+      const float mx = max32(v) * kLog2e;
+      if (mx > m) {
+        s *= exp2f(m - mx);
+        m = mx;
+      }
+      if (m != -INFINITY) {
+        float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          a0 += exp2f(fmaf(v[i], kLog2e, -m));
+          a1 += exp2f(fmaf(v[i + 1], kLog2e, -m));
+        }
+        s += a0 + a1;
+      }
+    }
+  }
+
+  __device__ __forceinline__ void unit_end(const Params& p, int, int j, int) {
+    if (!row_ok) return;
+    p.part[(static_cast<int64_t>(j) * 2 + 0) * p.N + grow] = m;
+    p.part[(static_cast<int64_t>(j) * 2 + 1) * p.N + grow] = s;
+    if (has_zy) p.zy[grow] = zyv;
+  }
+};
+
+// KL forward (and the first pass of the alpha losses): per row and for both the draft
+// (q) and the target (p): online max and sum of exp; plus
+// A = sum_v 2^(z_p log2e - m_p) (z_p - z_q), rescaled whenever m_p grows.
+struct EpiFwdDual {
+  using Params = FwdParams;
+  float mq, sq, mp, sp, A;
+  bool row_ok;
+  int64_t grow;
+
+  __device__ __forceinline__ void unit_begin(const Params& p, int mt, int, int row) {
+    mq = mp = -INFINITY;
+    sq = sp = A = 0.f;
+    grow = static_cast<int64_t>(mt) * kBM + row;
+    row_ok = grow < p.N;
+  }
+
+  template <bool TAIL>
+  __device__ __forceinline__ void chunk(float (&vq)[32], float (&vp)[32]) {
+    const float xq = max32(vq) * kLog2e;
+    const float xp = max32(vp) * kLog2e;
+    if (xq > mq) {
+      sq *= exp2f(mq - xq);
+      mq = xq;
+    }
+    if (xp > mp) {
+      const float r = exp2f(mp - xp);
+      sp *= r;
+      A *= r;
+      mp = xp;
+    }
+    if (mq == -INFINITY || mp == -INFINITY) return;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const float eq = exp2f(fmaf(vq[i], kLog2e, -mq));
+      const float e = exp2f(fmaf(vp[i], kLog2e, -mp));
+      sq += eq;
+      sp += e;
+      if (TAIL) {
+        if (e > 0.f) A = fmaf(e, vp[i] - vq[i], A);
+      } else {
+        A = fmaf(e, vp[i] - vq[i], A);
+      }
+    }
+  }
+
+  template <int BN>
+  __device__ __forceinline__ void tile(const Params& p, uint32_t tb, int, int nt, int) {
+    const int64_t n0 = static_cast<int64_t>(nt) * BN;
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 32) {
+      float vq[32], vp[32];
+      tmem_ld32(tb + c, vq);
+      tmem_ld32(tb + BN + c, vp);
+      tmem_ld_wait();
+      if (n0 + c + 32 > p.V) {
+        mask_tail(vq, n0 + c, p.V);
+        mask_tail(vp, n0 + c, p.V);
+        chunk<true>(vq, vp);
+      } else {
+        chunk<false>(vq, vp);
+      }
+    }
+  }
+
+  __device__ __forceinline__ void unit_end(const Params& p, int, int j, int) {
+    if (!row_ok) return;
+    float* base = p.part + static_cast<int64_t>(j) * 5 * p.N + grow;
+    base[0 * p.N] = mq;
+    base[1 * p.N] = sq;
+    base[2 * p.N] = mp;
+    base[3 * p.N] = sp;
+    base[4 * p.N] = A;
+  }
+};
+
+// Second pass of the alpha losses: with the final log-sum-exps L_q and L_p known,
+// alpha += min(p_v, q_v) and S += q_v where q_v < p_v.
+struct EpiAlpha {
+  using Params = FwdParams;
+  float lq2, lp2, al, S;
+  bool row_ok;
+  int64_t grow;
+
+  __device__ __forceinline__ void unit_begin(const Params& p, int mt, int, int row) {
+    al = S = 0.f;
+    grow = static_cast<int64_t>(mt) * kBM + row;
+    row_ok = grow < p.N;
+    lq2 = row_ok ? p.stats[grow] * kLog2e : 0.f;
+    lp2 = row_ok ? p.stats[p.N + grow] * kLog2e : 0.f;
+  }
+
+  template <int BN>
+  __device__ __forceinline__ void tile(const Params& p, uint32_t tb, int, int nt, int) {
+    const int64_t n0 = static_cast<int64_t>(nt) * BN;
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 32) {
+      float vq[32], vp[32];
+      tmem_ld32(tb + c, vq);
+      tmem_ld32(tb + BN + c, vp);
+      tmem_ld_wait();
+      if (n0 + c + 32 > p.V) {
+        mask_tail(vq, n0 + c, p.V);
+        mask_tail(vp, n0 + c, p.V);
+      }
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float qv = exp2f(fmaf(vq[i], kLog2e, -lq2));
+        const float pv = exp2f(fmaf(vp[i], kLog2e, -lp2));
+        al += fminf(pv, qv);
+        S += (qv < pv) ? qv : 0.f;
+      }
+    }
+  }
+
+  __device__ __forceinline__ void unit_end(const Params& p, int, int j, int) {
+    if (!row_ok) return;
+    p.part[(static_cast<int64_t>(j) * 2 + 0) * p.N + grow] = al;
+    p.part[(static_cast<int64_t>(j) * 2 + 1) * p.N + grow] = S;
+  }
+};
+
+// Upstream gradient of one row: valid * grad_tok * grad_scale / max(n_valid, 1).
+__device__ __forceinline__ float row_grad(const DzParams& p, int64_t n, bool valid) {
+  if (!valid) return 0.f;
+  float g = p.grad_tok ? p.grad_tok[n] : 1.f;
+  if (p.grad_scale) g *= *p.grad_scale;
+  if (p.n_valid) {
+    const long long nv = static_cast<long long>(*p.n_valid);
+    g /= static_cast<float>(nv > 0 ? nv : 1);
+  }
+  return g;
+}
+
+__device__ __forceinline__ void store_bf16_row32(__nv_bfloat16* dst, const float (&v)[32],
+                                                 int64_t col0, int64_t limit) {
+  if (col0 + 32 <= limit) {
+    uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      uint32_t w[4];
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        __nv_bfloat162 b2 = __floats2bfloat162_rn(v[8 * k + 2 * h], v[8 * k + 2 * h + 1]);
+        w[h] = *reinterpret_cast<uint32_t*>(&b2);
+      }
+      d4[k] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      if (col0 + i < limit) dst[i] = __float2bfloat16_rn(v[i]);
+  }
+}
+
+// Backward logits-gradient tile: recomputed logits -> dZ (bf16) of the token chunk.
+//   CE:      dz_j = g (q_j - [j = y])
+//   others:  dz_j = ck (q_j - p_j) + cm q_j (m_j - S),  m_j = [q_j < p_j]
+//            KL: ck = g, cm = 0;  TV: ck = 0, cm = -g;  NLA: ck = 0, cm = -g / alpha;
+//            LK: ck = g lambda, cm = -g (1 - lambda), lambda = exp(-3 alpha) (detached).
+template <bool DUAL>
+struct EpiDz {
+  using Params = DzParams;
+  float lq2, lp2, g, ck, cm, S;
+  int32_t lab;
+  bool row_ok;
+  int64_t lrow;
+
+  __device__ __forceinline__ void unit_begin(const Params& p, int mt, int, int row) {
+    lrow = static_cast<int64_t>(mt) * kBM + row;
+    row_ok = lrow < p.rows;
+    const int64_t n = p.row0 + lrow;
+    lq2 = lp2 = g = ck = cm = S = 0.f;
+    lab = -1;
+    if (!row_ok) return;
+    bool valid = true;
+    if (p.labels) {
+      lab = p.labels[n];
+      valid = lab != p.ignore_index;
+      if (!DUAL && (lab < 0 || lab >= p.V)) valid = false;
+    }
+    g = row_grad(p, n, valid);
+    lq2 = p.stats[n] * kLog2e;
+    if (DUAL) {
+      lp2 = p.stats[p.N + n] * kLog2e;
+      if (p.kind == kKL) {
+        ck = g;
+      } else {
+        const float al = p.stats[3 * p.N + n];
+        S = p.stats[4 * p.N + n];
+        if (p.kind == kTV) {
+          cm = -g;
+        } else if (p.kind == kNLA) {
+          cm = -g / fmaxf(al, 1e-30f);
+        } else {
+          const float lam = expf(-3.f * al);
+          ck = g * lam;
+          cm = -g * (1.f - lam);
+        }
+      }
+    }
+  }
+
+  template <int BN>
+  __device__ __forceinline__ void tile(const Params& p, uint32_t tb, int, int nt, int) {
+    const int64_t n0 = static_cast<int64_t>(nt) * BN;
+    __nv_bfloat16* out = p.dz + lrow * p.ldz + n0;
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 32) {
+      float vq[32];
+      tmem_ld32(tb + c, vq);
+      if (DUAL) {
+        float vp[32];
+        tmem_ld32(tb + BN + c, vp);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float qv = exp2f(fmaf(vq[i], kLog2e, -lq2));
+          const float pv = exp2f(fmaf(vp[i], kLog2e, -lp2));
+          const float mS = ((qv < pv) ? 1.f : 0.f) - S;
+          vq[i] = fmaf(ck, qv - pv, cm * qv * mS);
+        }
+      } else {
+        tmem_ld_wait();
+        const int64_t rel = static_cast<int64_t>(lab) - (n0 + c);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float qv = exp2f(fmaf(vq[i], kLog2e, -lq2));
+          vq[i] = g * (qv - (rel == i ? 1.f : 0.f));
+        }
+      }
+      if (row_ok) store_bf16_row32(out + c, vq, n0 + c, p.V);
+    }
+  }
+
+  __device__ __forceinline__ void unit_end(const Params&, int, int, int) {}
+};
+
+// dH rows of the chunk: fp32 accumulator -> bf16.
+struct EpiDh {
+  using Params = DhParams;
+  __device__ __forceinline__ void unit_begin(const Params&, int, int, int) {}
+  __device__ __forceinline__ void unit_end(const Params&, int, int, int) {}
+  template <int BN>
+  __device__ __forceinline__ void tile(const Params& p, uint32_t tb, int mt, int nt, int row) {
+    const int64_t lrow = static_cast<int64_t>(mt) * kBM + row;
+    const bool ok = lrow < p.rows;
+    const int64_t n0 = static_cast<int64_t>(nt) * BN;
+    __nv_bfloat16* out = p.dH + (p.row0 + lrow) * p.d + n0;
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 32) {
+      float v[32];
+      tmem_ld32(tb + c, v);
+      tmem_ld_wait();
+      if (ok && n0 + c < p.d) store_bf16_row32(out + c, v, n0 + c, p.d);
+    }
+  }
+};
+
+// dW tile: fp32 read-add-write (or plain write) of rows this CTA owns exclusively.
+struct EpiDw {
+  using Params = DwParams;
+  __device__ __forceinline__ void unit_begin(const Params&, int, int, int) {}
+  __device__ __forceinline__ void unit_end(const Params&, int, int, int) {}
+  template <int BN>
+  __device__ __forceinline__ void tile(const Params& p, uint32_t tb, int mt, int nt, int row) {
+    const int64_t v = static_cast<int64_t>(mt) * kBM + row;
+    const bool ok = v < p.V;
+    const int64_t n0 = static_cast<int64_t>(nt) * BN;
+    float* out = p.dW + v * p.d + n0;
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 32) {
+      float x[32];
+      tmem_ld32(tb + c, x);
+      tmem_ld_wait();
+      if (!ok || n0 + c >= p.d) continue;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        if (n0 + c + 4 * k + 4 <= p.d) {
+          float4* dst = reinterpret_cast<float4*>(out + c + 4 * k);
+          float4 r = make_float4(x[4 * k], x[4 * k + 1], x[4 * k + 2], x[4 * k + 3]);
+          if (p.beta) {
+            const float4 o = *dst;
+            r.x += o.x;
+            r.y += o.y;
+            r.z += o.z;
+            r.w += o.w;
+          }
+          *dst = r;
+        }
+      }
+    }
+  }
+};
+
+// ----------------------------------------------------------------------------------------
+// Launchers.
+// ----------------------------------------------------------------------------------------
+int sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (dev < 0 || dev >= 64) return 0;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+template <int BN, int NUM_A, bool A_MN, bool B_MN, class Epi>
+static cudaError_t launch_gemm(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b,
+                               const GemmGeom& g, const typename Epi::Params& p, const DevCtl& c,
+                               int grid, cudaStream_t s) {
+  constexpr size_t kStageBytes = NUM_A * kBM * kBK * 2 + BN * kBK * 2;
+  constexpr size_t kSmem = 1024 + kStages * kStageBytes + sizeof(PipeCtl);
+  auto kern = gemm_kernel<BN, NUM_A, A_MN, B_MN, Epi>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(kSmem));
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kThreads, kSmem, s>>>(a0, a1, b, g, p, c);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fwd_ce(const CUtensorMap& tH, const CUtensorMap& tW, const GemmGeom& g,
+                          const FwdParams& p, const DevCtl& c, int grid, cudaStream_t s) {
+  return launch_gemm<kBnSingle, 1, false, false, EpiFwdCE>(tH, tH, tW, g, p, c, grid, s);
+}
+cudaError_t launch_fwd_dual(const CUtensorMap& tHq, const CUtensorMap& tHp, const CUtensorMap& tW,
+                            const GemmGeom& g, const FwdParams& p, const DevCtl& c, int grid,
+                            cudaStream_t s) {
+  return launch_gemm<kBnDual, 2, false, false, EpiFwdDual>(tHq, tHp, tW, g, p, c, grid, s);
+}
+cudaError_t launch_alpha(const CUtensorMap& tHq, const CUtensorMap& tHp, const CUtensorMap& tW,
+                         const GemmGeom& g, const FwdParams& p, const DevCtl& c, int grid,
+                         cudaStream_t s) {
+  return launch_gemm<kBnDual, 2, false, false, EpiAlpha>(tHq, tHp, tW, g, p, c, grid, s);
+}
+cudaError_t launch_dz_ce(const CUtensorMap& tH, const CUtensorMap& tW, const GemmGeom& g,
+                         const DzParams& p, const DevCtl& c, int grid, cudaStream_t s) {
+  return launch_gemm<kBnSingle, 1, false, false, EpiDz<false>>(tH, tH, tW, g, p, c, grid, s);
+}
+cudaError_t launch_dz_dual(const CUtensorMap& tHq, const CUtensorMap& tHp, const CUtensorMap& tW,
+                           const GemmGeom& g, const DzParams& p, const DevCtl& c, int grid,
+                           cudaStream_t s) {
+  return launch_gemm<kBnDual, 2, false, false, EpiDz<true>>(tHq, tHp, tW, g, p, c, grid, s);
+}
+cudaError_t launch_dh(const CUtensorMap& tDz, const CUtensorMap& tW, const GemmGeom& g,
+                      const DhParams& p, const DevCtl& c, int grid, cudaStream_t s) {
+  return launch_gemm<kBnGrad, 1, false, true, EpiDh>(tDz, tDz, tW, g, p, c, grid, s);
+}
+cudaError_t launch_dw(const CUtensorMap& tDzT, const CUtensorMap& tH, const GemmGeom& g,
+                      const DwParams& p, const DevCtl& c, int grid, cudaStream_t s) {
+  return launch_gemm<kBnGrad, 1, true, true, EpiDw>(tDzT, tDzT, tH, g, p, c, grid, s);
+}
+
+// ----------------------------------------------------------------------------------------
+// Row combines: merge the per-unit partials of each row into the final statistics and the
+// per-token loss, then reduce the block's loss sum and valid count in a fixed order.
+// ----------------------------------------------------------------------------------------
+__device__ __forceinline__ void block_reduce_store(double v, long long c, double* blk_sum,
+                                                   long long* blk_cnt) {
+  __shared__ double ss[kCombineThreads / 32];
+  __shared__ long long sc[kCombineThreads / 32];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    v += __shfl_down_sync(0xffffffffu, v, o);
+    c += __shfl_down_sync(0xffffffffu, c, o);
+  }
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  if (l == 0) {
+    ss[w] = v;
+    sc[w] = c;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double t = 0.0;
+    long long k = 0;
+    for (int i = 0; i < kCombineThreads / 32; ++i) {
+      t += ss[i];
+      k += sc[i];
+    }
+    blk_sum[blockIdx.x] = t;
+    blk_cnt[blockIdx.x] = k;
+  }
+}
+
+__global__ void __launch_bounds__(kCombineThreads)
+    combine_kernel(int kind, int pass, const float* __restrict__ part, int nch,
+                   const float* __restrict__ zy, const int32_t* __restrict__ labels,
+                   int32_t ignore_index, int64_t N, int64_t V, float* loss_tok,
+                   float* alpha_tok, float* stats, double* blk_sum, long long* blk_cnt,
+                   int* status) {
+  const int64_t n = static_cast<int64_t>(blockIdx.x) * kCombineThreads + threadIdx.x;
+  double lsum = 0.0;
+  long long cnt = 0;
+  if (n < N) {
+    bool valid = true;
+    int32_t y = 0;
+    if (labels) {
+      y = labels[n];
+      valid = y != ignore_index;
+      if (kind == kCE && valid && (y < 0 || y >= V)) {
+        atomicOr(status, kFlagLabelRange);
+        valid = false;
+      }
+    }
+    float loss = 0.f;
+    if (kind == kCE) {
+      float M = -INFINITY;
+      for (int j = 0; j < nch; ++j) M = fmaxf(M, part[(2 * (int64_t)j) * N + n]);
+      float S = 0.f;
+      for (int j = 0; j < nch; ++j)
+        S += part[(2 * (int64_t)j + 1) * N + n] * exp2f(part[(2 * (int64_t)j) * N + n] - M);
+      const float L = (M + log2f(S)) * kLn2;
+      stats[n] = L;
+      loss = valid ? (L - zy[n]) : 0.f;
+    } else if (pass == 1) {
+      float Mq = -INFINITY, Mp = -INFINITY;
+      for (int j = 0; j < nch; ++j) {
+        const float* b = part + (int64_t)j * 5 * N + n;
+        Mq = fmaxf(Mq, b[0]);
+        Mp = fmaxf(Mp, b[2 * N]);
+      }
+      float Sq = 0.f, Sp = 0.f, A = 0.f;
+      for (int j = 0; j < nch; ++j) {
+        const float* b = part + (int64_t)j * 5 * N + n;
+        Sq += b[N] * exp2f(b[0] - Mq);
+        const float r = exp2f(b[2 * N] - Mp);
+        Sp += b[3 * N] * r;
+        A += b[4 * N] * r;
+      }
+      const float Lq = (Mq + log2f(Sq)) * kLn2;
+      const float Lp = (Mp + log2f(Sp)) * kLn2;
+      const float kl = A / Sp - Lp + Lq;
+      stats[n] = Lq;
+      stats[N + n] = Lp;
+      stats[2 * N + n] = kl;
+      loss = valid ? kl : 0.f;
+    } else {
+      float al = 0.f, S = 0.f;
+      for (int j = 0; j < nch; ++j) {
+        al += part[(2 * (int64_t)j) * N + n];
+        S += part[(2 * (int64_t)j + 1) * N + n];
+      }
+      stats[3 * N + n] = al;
+      stats[4 * N + n] = S;
+      if (alpha_tok) alpha_tok[n] = al;
+      const float kl = stats[2 * N + n];
+      float l;
+      if (kind == kTV) {
+        l = 1.f - al;
+      } else if (kind == kNLA) {
+        l = -logf(fmaxf(al, 1e-30f));
+      } else {
+        const float lam = expf(-3.f * al);
+        l = lam * kl + (1.f - lam) * (1.f - al);
+      }
+      loss = valid ? l : 0.f;
+    }
+    if (loss_tok) loss_tok[n] = loss;
+    lsum = static_cast<double>(loss);
+    cnt = valid ? 1 : 0;
+  }
+  block_reduce_store(lsum, cnt, blk_sum, blk_cnt);
+}
+
+__global__ void __launch_bounds__(1024)
+    finalize_kernel(const double* blk_sum, const long long* blk_cnt, int nblk, double* loss_sum,
+                    int64_t* n_valid, float* loss_mean) {
+  __shared__ double ss[32];
+  __shared__ long long sc[32];
+  double v = 0.0;
+  long long c = 0;
+  for (int i = threadIdx.x; i < nblk; i += blockDim.x) {
+    v += blk_sum[i];
+    c += blk_cnt[i];
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    v += __shfl_down_sync(0xffffffffu, v, o);
+    c += __shfl_down_sync(0xffffffffu, c, o);
+  }
+  if ((threadIdx.x & 31) == 0) {
+    ss[threadIdx.x >> 5] = v;
+    sc[threadIdx.x >> 5] = c;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double t = 0.0;
+    long long k = 0;
+    for (int i = 0; i < (int)(blockDim.x >> 5); ++i) {
+      t += ss[i];
+      k += sc[i];
+    }
+    *loss_sum = t;
+    *n_valid = static_cast<int64_t>(k);
+    if (loss_mean) *loss_mean = k > 0 ? static_cast<float>(t / static_cast<double>(k)) : 0.f;
+  }
+}
+
+__global__ void zero_f32_kernel(float* p, int64_t n) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    p[i] = 0.f;
+}
+
+cudaError_t launch_combine(int kind, int pass, const float* part, int nch, const float* zy,
+                           const int32_t* labels, int32_t ignore_index, int64_t N, int64_t V,
+                           float* loss_tok, float* alpha_tok, float* stats, double* blk_sum,
+                           long long* blk_cnt, int* status, cudaStream_t s) {
+  const int blocks = static_cast<int>((N + kCombineThreads - 1) / kCombineThreads);
+  combine_kernel<<<blocks, kCombineThreads, 0, s>>>(kind, pass, part, nch, zy, labels,
+                                                    ignore_index, N, V, loss_tok, alpha_tok,
+                                                    stats, blk_sum, blk_cnt, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_finalize(const double* blk_sum, const long long* blk_cnt, int nblk,
+                            double* loss_sum, int64_t* n_valid, float* loss_mean,
+                            cudaStream_t s) {
+  finalize_kernel<<<1, 1024, 0, s>>>(blk_sum, blk_cnt, nblk, loss_sum, n_valid, loss_mean);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_zero_f32(float* p, int64_t n, cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  const int sms = sm_count() > 0 ? sm_count() : 148;
+  zero_f32_kernel<<<sms * 4, 256, 0, s>>>(p, n);
+  return cudaGetLastError();
+}
+
+}  // namespace slm

@@ -1,0 +1,160 @@
+"""PyTorch-facing API of the streaming LM-head loss.
+
+PyTorch supplies device memory and the current stream; the loss, its statistics and its
+gradients are computed by the kernels of ``libslm.so`` through the C ABI.  The interface
+is the one of a regular loss function with a custom backward rule ("Training speculative
+decoders: removing the logits and attention bottlenecks", "Backward pass").
+"""
+
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import torch
+
+from . import _lib
+from .synthetic import IGNORE_INDEX
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _stream():
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _kind_id(kind):
+    if isinstance(kind, int):
+        return kind
+    try:
+        return _lib.KIND[kind]
+    except KeyError:
+        raise ValueError(f"unknown loss kind {kind!r}; expected one of {list(_lib.KIND)}")
+
+
+def _check_inputs(kind, hidden, weight, labels, target_hidden):
+    for name, t in (("hidden", hidden), ("weight", weight), ("target_hidden", target_hidden)):
+        if t is None:
+            continue
+        if not t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor")
+    if labels is not None and (labels.dtype != torch.int32 or not labels.is_contiguous()):
+        raise ValueError("labels must be a contiguous int32 tensor")
+    if kind != _lib.SLM_CE and target_hidden is None:
+        raise ValueError("distribution losses need target_hidden (H_p)")
+    if kind == _lib.SLM_CE and labels is None:
+        raise ValueError("ce needs labels")
+
+
+@dataclass
+class FwdResult:
+    kind: int
+    loss_mean: torch.Tensor   # float32 [1]
+    loss_sum: torch.Tensor    # float64 [1]
+    n_valid: torch.Tensor     # int64 [1]
+    loss_tok: torch.Tensor    # float32 [N]
+    alpha_tok: torch.Tensor | None
+    stats: torch.Tensor       # float32 [k, N]
+    workspace: torch.Tensor   # uint8
+
+
+def workspace_bytes(kind, N, d, V, chunk_tokens=0):
+    return _lib.slm_workspace_bytes(_kind_id(kind), N, d, V, chunk_tokens)
+
+
+def lm_head_loss_fwd(kind, hidden, weight, labels=None, target_hidden=None,
+                     ignore_index=IGNORE_INDEX, workspace=None, chunk_tokens=0,
+                     out=None) -> FwdResult:
+    """Forward through ``slm_loss_fwd``; returns the per-token loss, the sums and the
+    statistics the backward needs.  ``out`` may hold preallocated result buffers."""
+    k = _kind_id(kind)
+    _check_inputs(k, hidden, weight, labels, target_hidden)
+    N, d = hidden.shape
+    V = weight.shape[0]
+    dev = hidden.device
+    ws_need = _lib.slm_workspace_bytes(k, N, d, V, chunk_tokens)
+    if workspace is None or workspace.numel() < ws_need:
+        workspace = torch.empty(max(ws_need, 256), dtype=torch.uint8, device=dev)
+    if out is None:
+        nk = _lib.slm_stats_floats(k)
+        out = FwdResult(
+            k,
+            torch.empty(1, dtype=torch.float32, device=dev),
+            torch.empty(1, dtype=torch.float64, device=dev),
+            torch.empty(1, dtype=torch.int64, device=dev),
+            torch.empty(N, dtype=torch.float32, device=dev),
+            torch.empty(N, dtype=torch.float32, device=dev) if k >= _lib.SLM_TV else None,
+            torch.empty(nk, N, dtype=torch.float32, device=dev),
+            workspace)
+    else:
+        out.workspace = workspace
+    st = _lib.slm_loss_fwd(k, _ptr(hidden), _ptr(target_hidden), _ptr(weight), _ptr(labels),
+                           ignore_index, N, d, V, _ptr(out.loss_tok), _ptr(out.alpha_tok),
+                           _ptr(out.loss_sum), _ptr(out.n_valid), _ptr(out.loss_mean),
+                           _ptr(out.stats), _ptr(workspace), workspace.numel(), _stream())
+    _lib.check(st, "slm_loss_fwd")
+    return out
+
+
+def lm_head_loss_bwd(fwd: FwdResult, hidden, weight, labels=None, target_hidden=None,
+                     ignore_index=IGNORE_INDEX, grad_tok=None, grad_scale=None,
+                     normalize=True, dH=None, dW=None, accumulate_dW=False, chunk_tokens=0):
+    """Backward through ``slm_loss_bwd``.  With ``normalize`` the upstream gradient is
+    divided by the forward's valid-row count (gradient of the mean loss).
+    Returns (dH bf16 [N, d], dW fp32 [V, d])."""
+    k = fwd.kind
+    N, d = hidden.shape
+    V = weight.shape[0]
+    dev = hidden.device
+    if dH is None:
+        dH = torch.empty(N, d, dtype=torch.bfloat16, device=dev)
+    if dW is None:
+        dW = torch.empty(V, d, dtype=torch.float32, device=dev)
+    ws_need = _lib.slm_workspace_bytes(k, N, d, V, chunk_tokens)
+    ws = fwd.workspace
+    if ws.numel() < ws_need:
+        ws = torch.empty(ws_need, dtype=torch.uint8, device=dev)
+    st = _lib.slm_loss_bwd(k, _ptr(hidden), _ptr(target_hidden), _ptr(weight), _ptr(labels),
+                           ignore_index, N, d, V, _ptr(grad_tok), _ptr(grad_scale),
+                           _ptr(fwd.n_valid) if normalize else None, _ptr(fwd.stats),
+                           _ptr(dH), _ptr(dW), 1 if accumulate_dW else 0, chunk_tokens,
+                           _ptr(ws), ws.numel(), _stream())
+    _lib.check(st, "slm_loss_bwd")
+    return dH, dW
+
+
+def device_status(fwd: FwdResult):
+    """Synchronise and return the device status of the last call on this workspace."""
+    return _lib.slm_device_status(_ptr(fwd.workspace), _stream())
+
+
+class StreamingLMHeadLoss(torch.autograd.Function):
+    """Mean streaming LM-head loss with a custom backward: gradients for the draft hidden
+    states and the LM-head weight; the target hidden states are detached."""
+
+    @staticmethod
+    def forward(ctx, hidden, weight, labels, target_hidden, kind, ignore_index, chunk_tokens):
+        fwd = lm_head_loss_fwd(kind, hidden, weight, labels, target_hidden, ignore_index,
+                               chunk_tokens=chunk_tokens)
+        ctx.save_for_backward(hidden, weight, labels, target_hidden)
+        ctx.fwd = fwd
+        ctx.ignore_index = ignore_index
+        ctx.chunk_tokens = chunk_tokens
+        return fwd.loss_mean.reshape(())
+
+    @staticmethod
+    def backward(ctx, grad_out):
+        hidden, weight, labels, target_hidden = ctx.saved_tensors
+        g = grad_out.reshape(1).to(torch.float32).contiguous()
+        dH, dW = lm_head_loss_bwd(ctx.fwd, hidden, weight, labels, target_hidden,
+                                  ctx.ignore_index, grad_scale=g,
+                                  chunk_tokens=ctx.chunk_tokens)
+        return dH, dW.to(weight.dtype), None, None, None, None, None
+
+
+def streaming_lm_head_loss(hidden, weight, labels=None, target_hidden=None, kind="ce",
+                           ignore_index=IGNORE_INDEX, chunk_tokens=0):
+    """Mean loss over valid rows; differentiable w.r.t. ``hidden`` and ``weight``."""
+    return StreamingLMHeadLoss.apply(hidden, weight, labels, target_hidden, _kind_id(kind),
+                                     ignore_index, chunk_tokens)

@@ -1,0 +1,99 @@
+"""Shared helpers of the GPU parity tests: run the CUDA path through the C ABI and the
+float64 oracle on the same seeded inputs, and compare within the stated tolerances.
+
+Tolerances (bf16 inputs, fp32 accumulation; the oracle is float64):
+  * loss:      |L_gpu - L_ref| <= 2e-3 |L_ref| on the mean loss, and per token
+               max_n |l_gpu - l_ref| <= 2e-3 * max(max_n |l_ref|, 1e-2)
+  * gradients: max |dX_gpu - dX_ref| / max |dX_ref| <= 1e-2 for X in {H_q, W}
+"""
+
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+
+LOSS_RTOL = 2e-3
+GRAD_RTOL = 1e-2
+
+
+def _np64(t):
+    return t.detach().to("cpu").double().numpy()
+
+
+def gpu_fwd_bwd(inp, kind=None, chunk_tokens=0, grad_tok=None, normalize=True,
+                accumulate_dW=None):
+    """Forward and backward through the C ABI on cuda:0.  Returns numpy results plus the
+    device status after each call."""
+    from lm_head_loss_streaming_b200 import _lib
+    from lm_head_loss_streaming_b200.loss import (device_status, lm_head_loss_bwd,
+                                                  lm_head_loss_fwd)
+
+    kind = kind or inp.kind
+    dev = torch.device("cuda", 0)
+    Hq = inp.Hq.to(dev)
+    W = inp.W.to(dev)
+    Hp = inp.Hp.to(dev) if (kind != "ce" and inp.Hp is not None) else None
+    labels = inp.labels.to(dev) if inp.labels is not None else None
+    fwd = lm_head_loss_fwd(kind, Hq, W, labels, Hp, inp.ignore_index,
+                           chunk_tokens=chunk_tokens)
+    st_fwd = device_status(fwd)
+    gt = None
+    if grad_tok is not None:
+        gt = torch.as_tensor(grad_tok, dtype=torch.float32).to(dev).contiguous()
+    dW = None
+    if accumulate_dW is not None:
+        dW = torch.as_tensor(accumulate_dW, dtype=torch.float32).to(dev).contiguous()
+    dH, dW = lm_head_loss_bwd(fwd, Hq, W, labels, Hp, inp.ignore_index, grad_tok=gt,
+                              normalize=normalize, chunk_tokens=chunk_tokens, dW=dW,
+                              accumulate_dW=accumulate_dW is not None)
+    st_bwd = device_status(fwd)
+    torch.cuda.synchronize()
+    out = dict(
+        loss_tok=_np64(fwd.loss_tok), loss_mean=float(fwd.loss_mean.item()),
+        loss_sum=float(fwd.loss_sum.item()), n_valid=int(fwd.n_valid.item()),
+        stats=_np64(fwd.stats), alpha=None if fwd.alpha_tok is None else _np64(fwd.alpha_tok),
+        dH=_np64(dH), dW=_np64(dW), st_fwd=st_fwd, st_bwd=st_bwd,
+    )
+    assert _lib.SLM_OK == 0
+    return out
+
+
+def oracle_fwd_bwd(inp, kind=None, rows=None, grad_tok=None, chunk_size=512):
+    """The oracle on the same inputs (optionally on a subset of rows)."""
+    kind = kind or inp.kind
+    sl = slice(None) if rows is None else rows
+    Hq = inp.Hq[sl]
+    Hp = None if kind == "ce" else inp.Hp[sl]
+    lab = None if inp.labels is None else inp.labels[sl]
+    f = oracle.forward(kind, Hq, inp.W, lab, Hp, inp.ignore_index, chunk_size)
+    dH, dW = oracle.backward(kind, Hq, inp.W, lab, Hp, grad_tok, inp.ignore_index,
+                             chunk_size)
+    f["dH"] = dH
+    f["dW"] = dW
+    return f
+
+
+def assert_loss_close(gpu_tok, ref_tok, gpu_mean=None, ref_mean=None, what=""):
+    gpu_tok = np.asarray(gpu_tok)
+    ref_tok = np.asarray(ref_tok)
+    assert np.isfinite(gpu_tok).all(), f"{what}: non-finite per-token loss"
+    scale = max(float(np.abs(ref_tok).max()) if ref_tok.size else 0.0, 1e-2)
+    err = float(np.abs(gpu_tok - ref_tok).max()) if ref_tok.size else 0.0
+    assert err <= LOSS_RTOL * scale, f"{what}: per-token loss err {err:.3e} > {LOSS_RTOL}*{scale:.3e}"
+    if ref_mean is not None:
+        tol = LOSS_RTOL * max(abs(ref_mean), 1e-2)
+        assert abs(gpu_mean - ref_mean) <= tol, f"{what}: mean {gpu_mean} vs {ref_mean}"
+
+
+def assert_grad_close(g, r, what=""):
+    g = np.asarray(g)
+    r = np.asarray(r)
+    assert np.isfinite(g).all(), f"{what}: non-finite gradient"
+    den = float(np.abs(r).max()) if r.size else 0.0
+    err = float(np.abs(g - r).max()) if r.size else 0.0
+    if den == 0.0:
+        assert err <= 1e-6, f"{what}: expected zero gradient, max {err:.3e}"
+        return
+    assert err / den <= GRAD_RTOL, f"{what}: grad rel err {err / den:.3e} > {GRAD_RTOL}"

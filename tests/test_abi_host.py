@@ -1,0 +1,116 @@
+"""The C ABI library on a machine without a GPU: it loads, exports every symbol the header
+declares, and rejects invalid arguments on the host before touching CUDA."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from lm_head_loss_streaming_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "slm.h")
+
+
+def _declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(slm_[a-z_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(_lib.LIB_PATH):
+        from lm_head_loss_streaming_b200.build import build
+        build()
+    return _lib.load()
+
+
+def test_exports_every_declared_symbol(lib):
+    names = _declared_functions()
+    assert set(names) == set(_lib.SIGNATURES), names
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(_lib, "_lib", None)
+    monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "libslm.so"))
+    with pytest.raises(ImportError):
+        _lib.load()
+
+
+def test_status_strings_and_sizes(lib):
+    assert _lib.slm_version() >= 100
+    for code, name in _lib.STATUS_NAMES.items():
+        assert _lib.slm_status_string(code).startswith(name)
+    assert _lib.slm_stats_floats(_lib.SLM_CE) == 1
+    assert _lib.slm_stats_floats(_lib.SLM_KL) == 3
+    for k in (_lib.SLM_TV, _lib.SLM_NLA, _lib.SLM_LK_HYBRID):
+        assert _lib.slm_stats_floats(k) == 5
+    assert _lib.slm_stats_floats(7) == 0
+    assert _lib.slm_workspace_bytes(_lib.SLM_CE, 16, 12, 100) == 0  # d % 8 != 0
+    assert _lib.slm_workspace_bytes(9, 16, 16, 100) == 0
+
+
+def test_workspace_holds_chunk_buffer(lib):
+    # The backward's chunk buffer: chunk x V x bf16 (V padded to 8), chunk = min(N, 2d).
+    N, d, V = 16384, 4096, 128256
+    ws = _lib.slm_workspace_bytes(_lib.SLM_KL, N, d, V)
+    assert ws >= 8192 * V * 2
+    # O(N d + V d): far below the fp32 logits of the whole batch.
+    assert ws < N * V * 4 / 3
+    ws_small = _lib.slm_workspace_bytes(_lib.SLM_KL, N, d, V, 1024)
+    assert 1024 * V * 2 <= ws_small < ws
+    assert _lib.slm_workspace_bytes(_lib.SLM_CE, 0, 8, 10) > 0
+
+
+A = 1 << 20  # a 256-byte aligned fake address; never dereferenced on these paths
+
+
+def _fwd(**kw):
+    args = dict(kind=0, Hq=A, Hp=None, W=A, labels=A, ignore_index=-100, N=4, d=16, V=32,
+                loss_tok=A, alpha_tok=None, loss_sum=A, n_valid=A, loss_mean=None, stats=A,
+                workspace=A, ws_bytes=1 << 30, stream=None)
+    args.update(kw)
+    return _lib.slm_loss_fwd(*args.values())
+
+
+def _bwd(**kw):
+    args = dict(kind=0, Hq=A, Hp=None, W=A, labels=A, ignore_index=-100, N=4, d=16, V=32,
+                grad_tok=None, grad_scale=None, n_valid=None, stats=A, dHq=A, dW=A,
+                accumulate_dW=0, chunk_tokens=0, workspace=A, ws_bytes=1 << 30, stream=None)
+    args.update(kw)
+    return _lib.slm_loss_bwd(*args.values())
+
+
+@pytest.mark.parametrize("fn", [_fwd, _bwd])
+def test_host_errors(lib, fn):
+    assert fn(kind=5) == 4                   # SLM_ERR_KIND
+    assert fn(kind=-1) == 4
+    assert fn(d=12) == 2                     # SLM_ERR_SHAPE: d % 8
+    assert fn(d=0) == 2
+    assert fn(V=0) == 2
+    assert fn(N=-1) == 2
+    assert fn(W=None) == 1                   # SLM_ERR_NULL
+    assert fn(Hq=None) == 1
+    assert fn(labels=None) == 1              # CE needs labels
+    assert fn(kind=1) == 1                   # KL needs Hp
+    assert fn(workspace=None) == 1
+    assert fn(W=A + 8) == 3                  # SLM_ERR_ALIGN
+    assert fn(Hq=A + 2) == 3
+    assert fn(workspace=A + 16) == 5         # SLM_ERR_WORKSPACE: alignment
+    assert fn(ws_bytes=16) == 5              # SLM_ERR_WORKSPACE: size
+
+
+def test_fwd_output_pointer_errors(lib):
+    assert _fwd(loss_sum=None) == 1
+    assert _fwd(n_valid=None) == 1
+    assert _fwd(stats=None) == 1
+
+
+def test_bwd_output_pointer_errors(lib):
+    assert _bwd(dW=None) == 1
+    assert _bwd(dHq=None) == 1
+    assert _bwd(dW=A + 4) == 3
