@@ -91,7 +91,8 @@ SLM_API const char* slm_status_string(int status);
  * Returns 0 for an unknown kind. */
 SLM_API size_t slm_stats_floats(int kind);
 
-/* Bytes of workspace that slm_loss_fwd and slm_loss_bwd need for these sizes.
+/* Bytes of workspace that slm_loss_fwd and slm_loss_bwd need for these sizes (the
+ * forward alone needs no more than the value for any chunk_tokens).
  * chunk_tokens is the backward's token chunk (0 = automatic: min(N, 2d) rounded up to
  * 128); the workspace then holds one bf16 [chunk, V] logits-gradient buffer, which is the
  * streaming chunk buffer of "Backward pass".  Returns 0 on invalid arguments. */

@@ -61,7 +61,10 @@ int64_t default_chunk(int64_t N, int64_t d, int64_t chunk_tokens) {
 }
 
 struct Layout {
-  size_t status_off, red_off, nblk, big_off, part_off, zy_off, dz_off, ldz, total;
+  size_t status_off, red_off, nblk, big_off, part_off, zy_off, dz_off, ldz;
+  size_t fwd_total;  // bytes the forward uses
+  size_t bwd_total;  // bytes the backward uses with this chunk size
+  size_t total;      // max of the two
 };
 
 Layout layout(int kind, int64_t N, int64_t d, int64_t V, int64_t chunk_tokens) {
@@ -81,6 +84,8 @@ Layout layout(int kind, int64_t N, int64_t d, int64_t V, int64_t chunk_tokens) {
   const size_t bwd_end =
       align_up(L.dz_off + static_cast<size_t>(default_chunk(N, d, chunk_tokens)) * L.ldz * 2,
                kAlign);
+  L.fwd_total = fwd_end;
+  L.bwd_total = bwd_end;
   L.total = std::max(fwd_end, bwd_end);
   return L;
 }
@@ -160,9 +165,10 @@ int grid_for(const GemmGeom& g) {
   return std::max(1, std::min(g.num_units, sms > 0 ? sms : 148));
 }
 
+// `backward` selects which pass's workspace needs are checked.
 int common_checks(int kind, const void* Hq, const void* Hp, const void* W, const int32_t* labels,
                   int64_t N, int64_t d, int64_t V, const void* workspace, size_t ws_bytes,
-                  int64_t chunk_tokens) {
+                  int64_t chunk_tokens, bool backward) {
   if (!valid_kind(kind)) return SLM_ERR_KIND;
   if (N < 0 || d <= 0 || V <= 0 || (d % 8) != 0) return SLM_ERR_SHAPE;
   if (N >= (int64_t(1) << 31) || V >= (int64_t(1) << 31) || d >= (int64_t(1) << 31))
@@ -176,7 +182,8 @@ int common_checks(int kind, const void* Hq, const void* Hp, const void* W, const
   if (misaligned(W, 16) || (Hq && misaligned(Hq, 16)) || (dual_kind(kind) && Hp && misaligned(Hp, 16)))
     return SLM_ERR_ALIGN;
   if (misaligned(workspace, kAlign)) return SLM_ERR_WORKSPACE;
-  if (ws_bytes < layout(kind, N, d, V, chunk_tokens).total) return SLM_ERR_WORKSPACE;
+  const Layout L = layout(kind, N, d, V, chunk_tokens);
+  if (ws_bytes < (backward ? L.bwd_total : L.fwd_total)) return SLM_ERR_WORKSPACE;
   return SLM_OK;
 }
 
@@ -226,7 +233,7 @@ int slm_loss_fwd(int kind, const void* Hq, const void* Hp, const void* W, const 
                  int32_t ignore_index, int64_t N, int64_t d, int64_t V, float* loss_tok,
                  float* alpha_tok, double* loss_sum, int64_t* n_valid, float* loss_mean,
                  float* stats, void* workspace, size_t ws_bytes, void* stream) {
-  int st = common_checks(kind, Hq, Hp, W, labels, N, d, V, workspace, ws_bytes, 0);
+  int st = common_checks(kind, Hq, Hp, W, labels, N, d, V, workspace, ws_bytes, 0, false);
   if (st != SLM_OK) return st;
   if (!loss_sum || !n_valid || (N > 0 && !stats)) return SLM_ERR_NULL;
   if ((st = check_device()) != SLM_OK) return st;
@@ -277,7 +284,8 @@ int slm_loss_bwd(int kind, const void* Hq, const void* Hp, const void* W, const 
                  const float* grad_scale, const int64_t* n_valid, const float* stats, void* dHq,
                  float* dW, int accumulate_dW, int64_t chunk_tokens, void* workspace,
                  size_t ws_bytes, void* stream) {
-  int st = common_checks(kind, Hq, Hp, W, labels, N, d, V, workspace, ws_bytes, chunk_tokens);
+  int st = common_checks(kind, Hq, Hp, W, labels, N, d, V, workspace, ws_bytes, chunk_tokens,
+                         true);
   if (st != SLM_OK) return st;
   if (!dW || (N > 0 && (!dHq || !stats))) return SLM_ERR_NULL;
   if ((N > 0 && misaligned(dHq, 16)) || misaligned(dW, 16)) return SLM_ERR_ALIGN;

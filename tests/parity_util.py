@@ -87,12 +87,59 @@ def assert_loss_close(gpu_tok, ref_tok, gpu_mean=None, ref_mean=None, what=""):
         assert abs(gpu_mean - ref_mean) <= tol, f"{what}: mean {gpu_mean} vs {ref_mean}"
 
 
-def assert_grad_close(g, r, what=""):
+# Relative band |q_v - p_v| <= TIE_BAND * max(q_v, p_v) inside which the GPU's fp32
+# decision m_v = [q_v < p_v] may legitimately differ from the oracle's float64 one: the
+# GPU's q and p each carry a relative error of a few 1e-6 (fp32 logits accumulated over d
+# products, ex2.approx, fp32 sums).
+TIE_BAND = 1e-5
+
+
+def tie_slack(inp, kind, rows=None, grad_tok=None):
+    """Elementwise bound on how far dH (rows) and dW may move if every near-tie of the
+    indicator m_v = [q_v < p_v] is decided the other way.  Zero for kinds without it.
+
+    Flipping m_j of row n changes dz_nj by c_n q_nj and, through S_n, every dz_nk by
+    c_n q_nk q_nj, where c_n = g_n (tv), g_n / alpha_n (nla), g_n (1 - lambda_n) (lk_hybrid).
+    """
+    if kind not in ("tv", "nla", "lk_hybrid"):
+        return 0.0, 0.0
+    sl = slice(None) if rows is None else rows
+    Hq = inp.Hq[sl].double().numpy()
+    Hp = inp.Hp[sl].double().numpy()
+    W = inp.W.double().numpy()
+    q = np.exp(oracle.log_softmax(oracle.logits(Hq, W)))
+    p = np.exp(oracle.log_softmax(oracle.logits(Hp, W)))
+    n = Hq.shape[0]
+    valid = np.ones(n, dtype=bool)
+    if inp.labels is not None:
+        valid = inp.labels[sl].numpy() != inp.ignore_index
+    if grad_tok is None:
+        g = np.full(n, 1.0 / max(int(valid.sum()), 1))
+    else:
+        g = np.asarray(grad_tok, dtype=np.float64)
+    g = np.where(valid, np.abs(g), 0.0)
+    alpha = np.minimum(p, q).sum(axis=1)
+    if kind == "tv":
+        c = g
+    elif kind == "nla":
+        c = g / alpha
+    else:
+        c = g * (1.0 - np.exp(-3.0 * alpha))
+    near = np.abs(q - p) <= TIE_BAND * np.maximum(q, p)
+    qn = np.where(near, q, 0.0)
+    qsum = qn.sum(axis=1)
+    aW, aH = np.abs(W), np.abs(Hq)
+    slack_h = c[:, None] * (qn @ aW + qsum[:, None] * (q @ aW))
+    slack_w = (c[:, None] * qn).T @ aH + ((c * qsum)[:, None] * q).T @ aH
+    return slack_h, slack_w
+
+
+def assert_grad_close(g, r, what="", slack=0.0):
     g = np.asarray(g)
     r = np.asarray(r)
     assert np.isfinite(g).all(), f"{what}: non-finite gradient"
     den = float(np.abs(r).max()) if r.size else 0.0
-    err = float(np.abs(g - r).max()) if r.size else 0.0
+    err = float(np.maximum(np.abs(g - r) - slack, 0.0).max()) if r.size else 0.0
     if den == 0.0:
         assert err <= 1e-6, f"{what}: expected zero gradient, max {err:.3e}"
         return

@@ -1,0 +1,110 @@
+"""Parity at the workloads' full sizes, in the launch configuration the benchmark times.
+
+The GPU runs the whole batch.  The float64 oracle recomputes a seeded sample of rows one
+by one (a row's loss depends on no other row).  For the gradients, the upstream gradient
+is 1 on the sampled rows and 0 elsewhere, so dH on the sampled rows and the whole dW
+(a sum of per-row terms) are exactly what the oracle computes from those rows alone.
+With the full mean-loss gradient, two identities that hold at any size are checked:
+<dH, H_q> = <dW, W> (both equal sum_n g_n sum_v dz_nv z_nv) and sum_v dW[v, :] = 0.
+"""
+
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from lm_head_loss_streaming_b200 import synthetic
+from parity_util import assert_grad_close, assert_loss_close, oracle_fwd_bwd, tie_slack
+
+pytestmark = pytest.mark.gpu
+
+CASES = [("llama1b_ce", "ce"), ("llama8b_kl", "kl_div"), ("alpha_losses", "tv"),
+         ("alpha_losses", "nla"), ("alpha_losses", "lk_hybrid"), ("llama405b_ce", "ce")]
+R = 48
+
+
+def _host_ram_gb():
+    try:
+        return os.sysconf("SC_PAGE_SIZE") * os.sysconf("SC_PHYS_PAGES") / 1e9
+    except (ValueError, OSError):
+        return 0.0
+
+
+_cache = {}
+
+
+def _inputs(name):
+    if name not in _cache:
+        _cache.clear()
+        _cache[name] = synthetic.workload(name, seed=0, device="cpu")
+    return _cache[name]
+
+
+def _sample_rows(inp, r):
+    rng = np.random.default_rng(123)
+    rows = set(rng.choice(inp.N, size=r - 4, replace=False).tolist())
+    rows.update([0, inp.N - 1])
+    if inp.labels is not None:
+        masked = np.nonzero(inp.labels.numpy() == inp.ignore_index)[0]
+        rows.update(masked[:2].tolist())
+    return np.array(sorted(rows))
+
+
+@pytest.mark.parametrize("name,kind", CASES)
+def test_full_size_sampled_rows(name, kind):
+    from lm_head_loss_streaming_b200.loss import (device_status, lm_head_loss_bwd,
+                                                  lm_head_loss_fwd)
+    if name == "llama405b_ce" and _host_ram_gb() < 160:
+        pytest.skip("the float64 oracle of the 405B-shaped head needs ~60 GB of host RAM")
+    inp = _inputs(name)
+    dev = torch.device("cuda", 0)
+    Hq, W = inp.Hq.to(dev), inp.W.to(dev)
+    Hp = inp.Hp.to(dev) if (kind != "ce") else None
+    lab = inp.labels.to(dev) if inp.labels is not None else None
+    fwd = lm_head_loss_fwd(kind, Hq, W, lab, Hp, inp.ignore_index)
+    assert device_status(fwd) == 0
+    rows = _sample_rows(inp, R)
+    g = np.zeros(inp.N, dtype=np.float32)
+    g[rows] = 1.0
+    dH, dW = lm_head_loss_bwd(fwd, Hq, W, lab, Hp, inp.ignore_index,
+                              grad_tok=torch.from_numpy(g).to(dev), normalize=False)
+    assert device_status(fwd) == 0
+    loss_tok = fwd.loss_tok.double().cpu().numpy()
+    # Sum over the batch equals the reported loss_sum (fixed-order fp64 reduction).
+    assert abs(loss_tok.sum() - fwd.loss_sum.item()) <= 1e-5 * max(1.0, abs(loss_tok.sum()))
+    nv = int(fwd.n_valid.item())
+    if inp.labels is not None:
+        assert nv == int((inp.labels != inp.ignore_index).sum())
+    else:
+        assert nv == inp.N
+
+    ref = oracle_fwd_bwd(inp, kind, rows=torch.from_numpy(rows),
+                         grad_tok=np.ones(len(rows)))
+    assert_loss_close(loss_tok[rows], ref["loss_tok"], what=f"{name} {kind} loss")
+    sh, sw = tie_slack(inp, kind, rows=torch.from_numpy(rows), grad_tok=np.ones(len(rows)))
+    dH_np = dH[torch.from_numpy(rows).to(dev)].double().cpu().numpy()
+    assert_grad_close(dH_np, ref["dH"], f"{name} {kind} dH rows", sh)
+    others = torch.ones(inp.N, dtype=torch.bool, device=dev)
+    others[torch.from_numpy(rows).to(dev)] = False
+    assert float(dH[others].abs().max()) == 0.0
+    assert_grad_close(dW.double().cpu().numpy(), ref["dW"], f"{name} {kind} dW", sw)
+
+
+@pytest.mark.parametrize("name,kind", CASES[:3] + CASES[5:])
+def test_full_size_gradient_identities(name, kind):
+    from lm_head_loss_streaming_b200.loss import lm_head_loss_bwd, lm_head_loss_fwd
+    inp = _inputs(name)
+    dev = torch.device("cuda", 0)
+    Hq, W = inp.Hq.to(dev), inp.W.to(dev)
+    Hp = inp.Hp.to(dev) if (kind != "ce") else None
+    lab = inp.labels.to(dev) if inp.labels is not None else None
+    fwd = lm_head_loss_fwd(kind, Hq, W, lab, Hp, inp.ignore_index)
+    dH, dW = lm_head_loss_bwd(fwd, Hq, W, lab, Hp, inp.ignore_index)
+    a = float((dH.double() * Hq.double()).sum())
+    b = float((dW.double() * W.double()).sum())
+    assert abs(a - b) <= 1e-2 * max(abs(a), abs(b)), (a, b)
+    colsum = dW.double().sum(0).abs()
+    colabs = dW.double().abs().sum(0)
+    assert float((colsum / colabs.clamp_min(1e-30)).max()) <= 1e-2
+    assert torch.isfinite(fwd.loss_tok).all()
