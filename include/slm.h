@@ -150,6 +150,32 @@ SLM_API int slm_loss_bwd(int kind, const void* Hq, const void* Hp, const void* W
  * word when it starts, so the status describes the most recent call. */
 SLM_API int slm_device_status(const void* workspace, void* stream);
 
+/* Size of the device scratch array behind slm_loss_fwd_noalloc: 32 MiB per GPU that loads
+ * the library's device code, held until the process exits. */
+#define SLM_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/* Forward pass for callers that cannot allocate device memory.  The pages have no
+ * counterpart to this entry point; it exists for hosts that have no allocator of their own
+ * to hand out a workspace (a plain C program linking this library), runtimes whose enqueue
+ * path must not call cudaMalloc because it can synchronise the device, and processes with a
+ * fixed memory budget.
+ * Same arguments, outputs and results as slm_loss_fwd, without the workspace: the scratch
+ * lives in a fixed __device__ array of SLM_NOALLOC_SCRATCH_BYTES.  Sizes whose forward
+ * scratch exceeds it return SLM_ERR_WORKSPACE before anything is enqueued (at V = 128256
+ * that is N > ~66,000 rows for SLM_CE and N > ~26,500 rows for the other kinds).
+ *   device_flags  int [1] device memory or NULL: receives the device status bits of this
+ *                 call (0 = none; 1 = a CE label outside [0, V); 2 = a wait ran out of time).
+ * The first call on each device looks up the array's device address (and may load the
+ * library's device code), so make it before any stream capture.  Every call shares the one
+ * array: calls that overlap on the GPU race and must be serialised by the caller.  Nothing
+ * is allocated.  The backward still takes a caller workspace (slm_loss_bwd). */
+SLM_API int slm_loss_fwd_noalloc(int kind, const void* Hq, const void* Hp, const void* W,
+                                 const int32_t* labels, int32_t ignore_index,
+                                 int64_t N, int64_t d, int64_t V,
+                                 float* loss_tok, float* alpha_tok, double* loss_sum,
+                                 int64_t* n_valid, float* loss_mean, float* stats,
+                                 int* device_flags, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

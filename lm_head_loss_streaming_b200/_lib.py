@@ -40,6 +40,8 @@ SIGNATURES = {
     "slm_loss_bwd": (_INT, [_INT, _P, _P, _P, _P, _I32, _I64, _I64, _I64,
                             _P, _P, _P, _P, _P, _P, _INT, _I64, _P, _SZ, _P]),
     "slm_device_status": (_INT, [_P, _P]),
+    "slm_loss_fwd_noalloc": (_INT, [_INT, _P, _P, _P, _P, _I32, _I64, _I64, _I64,
+                                    _P, _P, _P, _P, _P, _P, _P, _P]),
 }
 
 
@@ -116,3 +118,13 @@ def slm_loss_bwd(kind, Hq, Hp, W, labels, ignore_index, N, d, V, grad_tok, grad_
 
 def slm_device_status(workspace, stream):
     return load().slm_device_status(workspace, stream)
+
+
+def slm_loss_fwd_noalloc(kind, Hq, Hp, W, labels, ignore_index, N, d, V, loss_tok, alpha_tok,
+                         loss_sum, n_valid, loss_mean, stats, device_flags, stream):
+    """Forward with the library's own fixed device scratch (no workspace argument), for
+    callers that cannot allocate device memory."""
+    return load().slm_loss_fwd_noalloc(int(kind), Hq, Hp, W, labels, int(ignore_index),
+                                       int(N), int(d), int(V), loss_tok, alpha_tok,
+                                       loss_sum, n_valid, loss_mean, stats, device_flags,
+                                       stream)

@@ -22,7 +22,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libslm.so")
 BUILD_DIR = os.path.join(ROOT, "_build")
 
-SOURCES = ["slm_api.cu", "slm_kernels.cu"]
+SOURCES = ["slm_api.cu", "slm_kernels.cu", "slm_noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "--use_fast_math", "-Xcompiler", "-fPIC",
          "-Xcompiler", "-fvisibility=hidden", "-I", INCLUDE, "-I", CSRC]

@@ -1,0 +1,102 @@
+"""The allocation-free forward entry point, slm_loss_fwd_noalloc, called through the C ABI.
+
+It is meant for callers that cannot allocate device memory: hosts with no allocator of
+their own to hand out a workspace, runtimes whose enqueue path must not call cudaMalloc,
+and processes held to a fixed memory budget.  Its scratch is a fixed device array inside
+the library, shared by every call, so these tests check two calls in a row (and a third
+that repeats the first) against the regular workspace-based slm_loss_fwd, within the
+parity tests' loss tolerance, and check that sizes beyond the array are refused.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from lm_head_loss_streaming_b200 import _lib, synthetic
+from lm_head_loss_streaming_b200.loss import lm_head_loss_fwd
+
+pytestmark = pytest.mark.gpu
+
+LOSS_RTOL = 2e-3
+
+
+def _on_gpu(inp):
+    dev = torch.device("cuda", 0)
+    return (inp.Hq.to(dev), inp.W.to(dev),
+            inp.Hp.to(dev) if inp.Hp is not None else None,
+            inp.labels.to(dev) if inp.labels is not None else None)
+
+
+def _noalloc_fwd(inp):
+    Hq, W, Hp, lab = _on_gpu(inp)
+    k = _lib.KIND[inp.kind]
+    dev = Hq.device
+    N, d, V = inp.N, inp.d, inp.V
+    loss_tok = torch.full((N,), float("nan"), device=dev)
+    alpha = torch.full((N,), float("nan"), device=dev) if k >= _lib.SLM_TV else None
+    loss_sum = torch.zeros(1, dtype=torch.float64, device=dev)
+    n_valid = torch.zeros(1, dtype=torch.int64, device=dev)
+    loss_mean = torch.zeros(1, device=dev)
+    stats = torch.full((_lib.slm_stats_floats(k), N), float("nan"), device=dev)
+    flags = torch.full((1,), -1, dtype=torch.int32, device=dev)
+    ptr = lambda t: None if t is None else t.data_ptr()  # noqa: E731
+    st = _lib.slm_loss_fwd_noalloc(k, ptr(Hq), ptr(Hp), ptr(W), ptr(lab), inp.ignore_index,
+                                   N, d, V, ptr(loss_tok), ptr(alpha), ptr(loss_sum),
+                                   ptr(n_valid), ptr(loss_mean), ptr(stats), ptr(flags),
+                                   torch.cuda.current_stream().cuda_stream)
+    assert st == _lib.SLM_OK, _lib.status_string(st)
+    torch.cuda.synchronize()
+    return dict(loss_tok=loss_tok.double().cpu().numpy(), loss_sum=loss_sum.item(),
+                n_valid=n_valid.item(), loss_mean=loss_mean.item(),
+                stats=stats.double().cpu().numpy(), flags=int(flags.item()))
+
+
+def _workspace_fwd(inp):
+    Hq, W, Hp, lab = _on_gpu(inp)
+    r = lm_head_loss_fwd(inp.kind, Hq, W, lab, Hp, inp.ignore_index)
+    torch.cuda.synchronize()
+    return dict(loss_tok=r.loss_tok.double().cpu().numpy(), loss_sum=r.loss_sum.item(),
+                n_valid=r.n_valid.item(), loss_mean=r.loss_mean.item(),
+                stats=r.stats.double().cpu().numpy())
+
+
+def _assert_same(got, ref):
+    assert got["flags"] == 0
+    assert got["n_valid"] == ref["n_valid"]
+    scale = max(np.abs(ref["loss_tok"]).max(), 1e-2)
+    assert np.abs(got["loss_tok"] - ref["loss_tok"]).max() <= LOSS_RTOL * scale
+    assert abs(got["loss_mean"] - ref["loss_mean"]) <= LOSS_RTOL * max(abs(ref["loss_mean"]), 1e-2)
+    assert abs(got["loss_sum"] - ref["loss_sum"]) <= LOSS_RTOL * max(abs(ref["loss_sum"]), 1e-2)
+    assert np.allclose(got["stats"], ref["stats"], rtol=1e-5, atol=1e-4)
+
+
+def test_noalloc_forward_matches_workspace_forward_two_calls_in_a_row():
+    first = synthetic.make("ce", 700, 256, 5000, w_std=0.05, ignore_frac=0.1, seed=21)
+    second = synthetic.make("kl_div", 513, 128, 3001, w_std=0.05, seed=22)
+    ref1 = _workspace_fwd(first)
+    ref2 = _workspace_fwd(second)
+    got1 = _noalloc_fwd(first)
+    _assert_same(got1, ref1)
+    got2 = _noalloc_fwd(second)
+    _assert_same(got2, ref2)
+    # The shared scratch keeps the previous call's contents; a repeat of the first call
+    # must not see them.
+    again = _noalloc_fwd(first)
+    _assert_same(again, ref1)
+    assert np.array_equal(again["loss_tok"], got1["loss_tok"])
+
+
+def test_noalloc_alpha_kind():
+    inp = synthetic.make("lk_hybrid", 300, 128, 2000, w_std=0.05, seed=23)
+    _assert_same(_noalloc_fwd(inp), _workspace_fwd(inp))
+
+
+def test_noalloc_refuses_sizes_beyond_its_scratch():
+    # KL at V = 128256 needs ~1.26 KB of forward scratch per row: 100000 rows do not fit.
+    fake = 1 << 20  # aligned, never dereferenced: the call returns before enqueuing work
+    st = _lib.slm_loss_fwd_noalloc(_lib.SLM_KL, fake, fake, fake, None, -100, 100000, 8,
+                                   128256, None, None, fake, fake, None, fake, None,
+                                   torch.cuda.current_stream().cuda_stream)
+    assert st == 5  # SLM_ERR_WORKSPACE
+    assert _lib.slm_loss_fwd_noalloc(9, None, None, None, None, -100, 1, 8, 8, None, None,
+                                     None, None, None, None, None, None) == 4  # SLM_ERR_KIND
