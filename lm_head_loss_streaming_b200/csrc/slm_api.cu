@@ -27,6 +27,8 @@ namespace slm {
 namespace {
 
 constexpr size_t kAlign = 256;
+constexpr int kPairM = 2 * kBM;   // M rows of one 2-SM tile
+constexpr int kGroupPairs = 8;    // pair M tiles per raster group (2048 token rows)
 constexpr long long kTimeoutCycles = 4000000000LL;  // ~2 s at the B200's boost clock
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -148,9 +150,10 @@ bool make_map(CUtensorMap* m, const void* base, int64_t inner, int64_t outer, in
 
 bool misaligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) != 0; }
 
-GemmGeom geom(int64_t M, int64_t Nn, int64_t K, int bn, int vc, int group_m) {
+// Tile schedule of a GEMM with M tiles of `bm` rows (256: a 2-SM CTA pair).
+GemmGeom geom(int64_t M, int64_t Nn, int64_t K, int bn, int vc, int group_m, int bm) {
   GemmGeom g;
-  g.num_m = static_cast<int>(ceil_div(M, kBM));
+  g.num_m = static_cast<int>(ceil_div(M, bm));
   g.num_n = static_cast<int>(ceil_div(Nn, bn));
   g.k_blocks = static_cast<int>(ceil_div(K, kBK));
   g.vc = std::max(1, std::min(vc, g.num_n));
@@ -250,10 +253,10 @@ int slm_loss_fwd(int kind, const void* Hq, const void* Hp, const void* W, const 
 
   if (N > 0) {
     const FwdSched f = fwd_sched(kind, V);
-    const GemmGeom g = geom(N, V, d, f.bn, f.vc, 16);
+    const GemmGeom g = geom(N, V, d, f.bn, f.vc, kGroupPairs, kPairM);
     CUtensorMap tHq, tHp, tW;
     if (!make_map(&tHq, Hq, d, N, d, kBK, kBM)) return SLM_ERR_CUDA;
-    if (!make_map(&tW, W, d, V, d, kBK, f.bn)) return SLM_ERR_CUDA;
+    if (!make_map(&tW, W, d, V, d, kBK, f.bn / 2)) return SLM_ERR_CUDA;
     FwdParams p{labels, ignore_index, N, V, part, zy, stats};
     const int grid = grid_for(g);
     if (!dual_kind(kind)) {
@@ -305,7 +308,7 @@ int slm_loss_bwd(int kind, const void* Hq, const void* Hp, const void* W, const 
   const int64_t C = default_chunk(N, d, chunk_tokens);
   const FwdSched f = fwd_sched(kind, V);
   CUtensorMap tW_k, tW_mn;
-  if (!make_map(&tW_k, W, d, V, d, kBK, f.bn)) return SLM_ERR_CUDA;
+  if (!make_map(&tW_k, W, d, V, d, kBK, f.bn / 2)) return SLM_ERR_CUDA;
   if (!make_map(&tW_mn, W, d, V, d, 64, 64)) return SLM_ERR_CUDA;
   const int64_t ldz = static_cast<int64_t>(L.ldz);
 
@@ -315,7 +318,7 @@ int slm_loss_bwd(int kind, const void* Hq, const void* Hp, const void* W, const 
     // 1) Recompute the chunk's logits and write its logits gradient dZ [rows, V] (bf16).
     CUtensorMap tHq, tHp;
     if (!make_map(&tHq, hq, d, rows, d, kBK, kBM)) return SLM_ERR_CUDA;
-    const GemmGeom gz = geom(rows, V, d, f.bn, f.vc, 16);
+    const GemmGeom gz = geom(rows, V, d, f.bn, f.vc, kGroupPairs, kPairM);
     DzParams pz{kind, labels, ignore_index, c0, rows, N, V, stats, grad_tok, grad_scale,
                 n_valid, dz, ldz};
     if (!dual_kind(kind)) {
@@ -328,13 +331,13 @@ int slm_loss_bwd(int kind, const void* Hq, const void* Hp, const void* W, const 
     // 2) dH[chunk] = dZ W   (M = rows, N = d, K = V; W read MN-major).
     CUtensorMap tDz_k, tDz_mn, tH_mn;
     if (!make_map(&tDz_k, dz, V, rows, ldz, kBK, kBM)) return SLM_ERR_CUDA;
-    const GemmGeom gh = geom(rows, d, V, kBnGrad, 1, 1);
+    const GemmGeom gh = geom(rows, d, V, kBnGrad, 1, 1, kPairM);
     DhParams ph{static_cast<__nv_bfloat16*>(dHq), c0, rows, d};
     SLM_TRY_CUDA(launch_dh(tDz_k, tW_mn, gh, ph, ctl, grid_for(gh), s));
     // 3) dW (+)= dZ^T H[chunk]   (M = V, N = d, K = rows; both operands MN-major).
     if (!make_map(&tDz_mn, dz, V, rows, ldz, 64, 64)) return SLM_ERR_CUDA;
     if (!make_map(&tH_mn, hq, d, rows, d, 64, 64)) return SLM_ERR_CUDA;
-    const GemmGeom gw = geom(V, d, rows, kBnGrad, 1, 1);
+    const GemmGeom gw = geom(V, d, rows, kBnGrad, 1, 1, kPairM);
     DwParams pw{dW, V, d, (accumulate_dW || c0 > 0) ? 1 : 0};
     SLM_TRY_CUDA(launch_dw(tDz_mn, tH_mn, gw, pw, ctl, grid_for(gw), s));
   }

@@ -23,6 +23,8 @@
 
 #include <math.h>
 
+#include <algorithm>
+
 #include "slm_internal.h"
 #include "sm100.cuh"
 
@@ -242,7 +244,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int mt, j;
       unit_coords(g, u, mt, j);
       const int n_end = min((j + 1) * g.vc, g.num_n);
-      epi.unit_begin(ep, mt, j, row);
+      epi.unit_begin(ep, mt * kBM, j, row);
       for (int nt = j * g.vc; nt < n_end; ++nt, ++t) {
         const int b = t & 1;
         const uint32_t ub = (t >> 1) & 1u;
@@ -251,12 +253,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
-        epi.template tile<BN>(ep, tmem + lane_bits + b * kAccCols, mt, nt, row);
+        epi.template tile<BN>(ep, tmem + lane_bits + b * kAccCols, mt * kBM, nt, row);
         tc_fence_before();
         mbar_arrive(&pc->tempty[b]);
       }
       if (!ok) break;
-      epi.unit_end(ep, mt, j, row);
+      epi.unit_end(ep, mt * kBM, j, row);
     }
   }
 
@@ -264,6 +266,246 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+}
+
+// ----------------------------------------------------------------------------------------
+// The 2-SM skeleton: a cluster of two CTAs shares each MMA (cta_group::2, M = 256).
+// CTA r of the pair loads rows [128 r, 128 r + 128) of its 256-row M tile and columns
+// [r BN/2, (r + 1) BN/2) of the N tile into its own shared memory; both CTAs' copies count
+// on the leader's "full" barrier; the leader's single MMA thread multiplies the pair's
+// operands into both CTAs' TMEM and releases stages and accumulators in both CTAs with
+// multicast commits; each CTA's epilogue reads its own 128 accumulator rows and reports
+// back to the leader.  Per CTA, a stage of shared memory holds half the B operand of the
+// 1-CTA form, which halves the shared-memory operand traffic per flop.
+// ----------------------------------------------------------------------------------------
+template <int STAGES>
+struct PairCtl {
+  uint64_t full[STAGES];
+  uint64_t empty[STAGES];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint64_t fin;
+  uint32_t tmem_base;
+  int abort;
+};
+
+template <int BN, int NUM_A, bool A_MN, bool B_MN, int STAGES>
+struct PairShape {
+  static constexpr int kBNH = BN / 2;  // B rows (K-major) or columns (MN-major) per CTA
+  static constexpr uint32_t kABytes = kBM * kBK * 2;
+  static constexpr uint32_t kBBytes = kBNH * kBK * 2;
+  static constexpr uint32_t kStageBytes = NUM_A * kABytes + kBBytes;
+  static constexpr size_t kSmem = 1024 + STAGES * static_cast<size_t>(kStageBytes) +
+                                  sizeof(PairCtl<STAGES>);
+};
+
+template <int BN, int NUM_A, bool A_MN, bool B_MN, int STAGES, class Epi>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0,
+                     const __grid_constant__ CUtensorMap tmA1,
+                     const __grid_constant__ CUtensorMap tmB, const GemmGeom g,
+                     const typename Epi::Params ep, const DevCtl ctl) {
+  using Sh = PairShape<BN, NUM_A, A_MN, B_MN, STAGES>;
+  constexpr int kBNH = Sh::kBNH;
+  constexpr uint32_t kABytes = Sh::kABytes;
+  constexpr uint32_t kStageBytes = Sh::kStageBytes;
+  constexpr uint32_t kAccCols = NUM_A * BN;
+  static_assert(2 * kAccCols <= kTmemCols, "two accumulator buffers must fit in TMEM");
+  static_assert(BN % 32 == 0 && BN >= 64 && BN <= 256, "UMMA N for M = 256");
+  static_assert(kBNH % 64 == 0, "each CTA's B half is whole 64-element boxes");
+  constexpr uint32_t kIdesc = idesc_bf16_f32(2 * kBM, BN, A_MN, B_MN);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  PairCtl<STAGES>* pc = reinterpret_cast<PairCtl<STAGES>*>(smem + STAGES * kStageBytes);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1;
+  const int npairs = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&pc->full[s], 1);
+      mbar_init(&pc->empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&pc->tfull[b], 1);
+      mbar_init(&pc->tempty[b], 2 * 4);  // one arrive per epilogue warp of both CTAs
+    }
+    mbar_init(&pc->fin, 1);
+    pc->abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA0);
+    if (NUM_A == 2) tma_prefetch_desc(&tmA1);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(&pc->tmem_base, kTmemCols);
+    tmem_relinquish_pair();
+  }
+  // Both CTAs' barriers exist before either CTA touches the other's.
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem = pc->tmem_base;
+  volatile int* abort = &pc->abort;
+
+  if (warp == 0) {
+    // ------------------------------ TMA producer (both CTAs) ------------------------------
+    uint32_t it = 0;
+    bool ok = true;
+    for (int u = pair; ok && u < g.num_units; u += npairs) {
+      int mt, j;
+      unit_coords(g, u, mt, j);
+      const int mrow = mt * 2 * kBM + static_cast<int>(rank) * kBM;
+      const int n_end = min((j + 1) * g.vc, g.num_n);
+      for (int nt = j * g.vc; ok && nt < n_end; ++nt) {
+        const int ncol = nt * BN + static_cast<int>(rank) * kBNH;
+        for (int kb = 0; kb < g.k_blocks; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1u;
+          if (!wait_warp(&pc->empty[s], ph ^ 1u, abort, ctl)) {
+            ok = false;
+            break;
+          }
+          if (lane == 0) {
+            uint8_t* st = smem + s * kStageBytes;
+            if (leader) mbar_arrive_expect_tx(&pc->full[s], 2 * kStageBytes);
+            const int k0 = kb * kBK;
+#pragma unroll
+            for (int a = 0; a < NUM_A; ++a) {
+              const CUtensorMap* map = (a == 0) ? &tmA0 : &tmA1;
+              uint8_t* dst = st + a * kABytes;
+              if (A_MN) {
+                tma_load_2d_pair(dst, map, &pc->full[s], mrow, k0);
+                tma_load_2d_pair(dst + 8192, map, &pc->full[s], mrow + 64, k0);
+              } else {
+                tma_load_2d_pair(dst, map, &pc->full[s], k0, mrow);
+              }
+            }
+            uint8_t* bdst = st + NUM_A * kABytes;
+            if (B_MN) {
+#pragma unroll
+              for (int jb = 0; jb < kBNH / 64; ++jb)
+                tma_load_2d_pair(bdst + jb * 8192, &tmB, &pc->full[s], ncol + jb * 64, k0);
+            } else {
+              tma_load_2d_pair(bdst, &tmB, &pc->full[s], k0, ncol);
+            }
+          }
+          __syncwarp();
+        }
+      }
+    }
+    if (!ok) {
+      if (leader) {
+        // The full barriers count both CTAs' copies: waiting on them lets the pair's
+        // copies in flight land before either CTA leaves the final cluster barrier.
+        const uint32_t first = it > (uint32_t)STAGES ? it - STAGES : 0u;
+        for (uint32_t i = first; i < it; ++i)
+          wait_warp(&pc->full[i % STAGES], (i / STAGES) & 1u, abort, ctl, false);
+      } else {
+        for (int i = 0; i < 100; ++i) __nanosleep(1000);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------ MMA issuer (leader only) ------------------------------
+    if (leader) {
+      uint32_t it = 0, t = 0;
+      bool ok = true;
+      for (int u = pair; ok && u < g.num_units; u += npairs) {
+        int mt, j;
+        unit_coords(g, u, mt, j);
+        const int n_end = min((j + 1) * g.vc, g.num_n);
+        for (int nt = j * g.vc; ok && nt < n_end; ++nt, ++t) {
+          const int b = t & 1;
+          const uint32_t ub = (t >> 1) & 1u;
+          if (!wait_warp(&pc->tempty[b], ub ^ 1u, abort, ctl)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t dcol = tmem + b * kAccCols;
+          for (int kb = 0; kb < g.k_blocks; ++kb, ++it) {
+            const int s = it % STAGES;
+            const uint32_t ph = (it / STAGES) & 1u;
+            if (!wait_warp(&pc->full[s], ph, abort, ctl)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            if (lane == 0) {
+              const uint32_t a_addr = smem_u32(smem + s * kStageBytes);
+              const uint32_t b_addr = a_addr + NUM_A * kABytes;
+#pragma unroll
+              for (int kk = 0; kk < kBK / 16; ++kk) {
+                const uint64_t bd = B_MN ? smem_desc_sw128(b_addr + kk * 2048, 8192, 1024)
+                                         : smem_desc_sw128(b_addr + kk * 32, 16, 1024);
+#pragma unroll
+                for (int a = 0; a < NUM_A; ++a) {
+                  const uint32_t aa = a_addr + a * kABytes;
+                  const uint64_t ad = A_MN ? smem_desc_sw128(aa + kk * 2048, 8192, 1024)
+                                           : smem_desc_sw128(aa + kk * 32, 16, 1024);
+                  umma_bf16_pair(dcol + a * BN, ad, bd, kIdesc, (kb | kk) != 0 ? 1u : 0u);
+                }
+              }
+              umma_commit_pair_mc(&pc->empty[s], 0x3);
+            }
+            __syncwarp();
+          }
+          if (!ok) break;
+          if (lane == 0) umma_commit_pair_mc(&pc->tfull[b], 0x3);
+          __syncwarp();
+        }
+      }
+      // Every MMA must be complete (in both CTAs' TMEM) before TMEM is released.
+      if (lane == 0) umma_commit_pair_mc(&pc->fin, 0x1);
+      __syncwarp();
+      wait_warp(&pc->fin, 0u, abort, ctl, false);
+    }
+  } else {
+    // ------------------------------ epilogue (both CTAs) ------------------------------
+    const int q = warp & 3;  // a warp may only touch TMEM lanes [32 * (warp % 4), +32)
+    const int row = q * 32 + lane;
+    const uint32_t lane_bits = static_cast<uint32_t>(q * 32) << 16;
+    const uint32_t tempty_leader0 = mapa_shared(smem_u32(&pc->tempty[0]), 0);
+    const uint32_t tempty_leader1 = mapa_shared(smem_u32(&pc->tempty[1]), 0);
+    Epi epi;
+    uint32_t t = 0;
+    bool ok = true;
+    for (int u = pair; ok && u < g.num_units; u += npairs) {
+      int mt, j;
+      unit_coords(g, u, mt, j);
+      const int row0 = mt * 2 * kBM + static_cast<int>(rank) * kBM;
+      const int n_end = min((j + 1) * g.vc, g.num_n);
+      epi.unit_begin(ep, row0, j, row);
+      for (int nt = j * g.vc; nt < n_end; ++nt, ++t) {
+        const int b = t & 1;
+        const uint32_t ub = (t >> 1) & 1u;
+        if (!wait_warp(&pc->tfull[b], ub, abort, ctl)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        epi.template tile<BN>(ep, tmem + lane_bits + b * kAccCols, row0, nt, row);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(b ? tempty_leader1 : tempty_leader0);
+      }
+      if (!ok) break;
+      epi.unit_end(ep, row0, j, row);
+    }
+  }
+
+  // Neither CTA leaves while the other may still signal its barriers or use its TMEM.
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc_pair(tmem, kTmemCols);
 }
 
 // ----------------------------------------------------------------------------------------
@@ -294,12 +536,12 @@ struct EpiFwdCE {
   bool has_zy, row_ok;
   int64_t grow;
 
-  __device__ __forceinline__ void unit_begin(const Params& p, int mt, int, int row) {
+  __device__ __forceinline__ void unit_begin(const Params& p, int row0, int, int row) {
     m = -INFINITY;
     s = 0.f;
     has_zy = false;
     zyv = 0.f;
-    grow = static_cast<int64_t>(mt) * kBM + row;
+    grow = static_cast<int64_t>(row0) + row;
     row_ok = grow < p.N;
     lab = row_ok ? p.labels[grow] : -1;
   }
@@ -355,10 +597,10 @@ struct EpiFwdDual {
   bool row_ok;
   int64_t grow;
 
-  __device__ __forceinline__ void unit_begin(const Params& p, int mt, int, int row) {
+  __device__ __forceinline__ void unit_begin(const Params& p, int row0, int, int row) {
     mq = mp = -INFINITY;
     sq = sp = A = 0.f;
-    grow = static_cast<int64_t>(mt) * kBM + row;
+    grow = static_cast<int64_t>(row0) + row;
     row_ok = grow < p.N;
   }
 
@@ -429,9 +671,9 @@ struct EpiAlpha {
   bool row_ok;
   int64_t grow;
 
-  __device__ __forceinline__ void unit_begin(const Params& p, int mt, int, int row) {
+  __device__ __forceinline__ void unit_begin(const Params& p, int row0, int, int row) {
     al = S = 0.f;
-    grow = static_cast<int64_t>(mt) * kBM + row;
+    grow = static_cast<int64_t>(row0) + row;
     row_ok = grow < p.N;
     lq2 = row_ok ? p.stats[grow] * kLog2e : 0.f;
     lp2 = row_ok ? p.stats[p.N + grow] * kLog2e : 0.f;
@@ -513,8 +755,8 @@ struct EpiDz {
   bool row_ok;
   int64_t lrow;
 
-  __device__ __forceinline__ void unit_begin(const Params& p, int mt, int, int row) {
-    lrow = static_cast<int64_t>(mt) * kBM + row;
+  __device__ __forceinline__ void unit_begin(const Params& p, int row0, int, int row) {
+    lrow = static_cast<int64_t>(row0) + row;
     row_ok = lrow < p.rows;
     const int64_t n = p.row0 + lrow;
     lq2 = lp2 = g = ck = cm = S = 0.f;
@@ -589,8 +831,8 @@ struct EpiDh {
   __device__ __forceinline__ void unit_begin(const Params&, int, int, int) {}
   __device__ __forceinline__ void unit_end(const Params&, int, int, int) {}
   template <int BN>
-  __device__ __forceinline__ void tile(const Params& p, uint32_t tb, int mt, int nt, int row) {
-    const int64_t lrow = static_cast<int64_t>(mt) * kBM + row;
+  __device__ __forceinline__ void tile(const Params& p, uint32_t tb, int row0, int nt, int row) {
+    const int64_t lrow = static_cast<int64_t>(row0) + row;
     const bool ok = lrow < p.rows;
     const int64_t n0 = static_cast<int64_t>(nt) * BN;
     __nv_bfloat16* out = p.dH + (p.row0 + lrow) * p.d + n0;
@@ -610,8 +852,8 @@ struct EpiDw {
   __device__ __forceinline__ void unit_begin(const Params&, int, int, int) {}
   __device__ __forceinline__ void unit_end(const Params&, int, int, int) {}
   template <int BN>
-  __device__ __forceinline__ void tile(const Params& p, uint32_t tb, int mt, int nt, int row) {
-    const int64_t v = static_cast<int64_t>(mt) * kBM + row;
+  __device__ __forceinline__ void tile(const Params& p, uint32_t tb, int row0, int nt, int row) {
+    const int64_t v = static_cast<int64_t>(row0) + row;
     const bool ok = v < p.V;
     const int64_t n0 = static_cast<int64_t>(nt) * BN;
     float* out = p.dW + v * p.d + n0;
@@ -670,36 +912,85 @@ static cudaError_t launch_gemm(const CUtensorMap& a0, const CUtensorMap& a1, con
   return cudaGetLastError();
 }
 
+// Persistent 2-SM launch: clusters of two CTAs, at most as many clusters as can be
+// resident at once (so the static unit schedule never waits for a second wave).
+template <int BN, int NUM_A, bool A_MN, bool B_MN, int STAGES, class Epi>
+static cudaError_t launch_gemm_pair(const CUtensorMap& a0, const CUtensorMap& a1,
+                                    const CUtensorMap& b, const GemmGeom& g,
+                                    const typename Epi::Params& p, const DevCtl& c,
+                                    cudaStream_t s) {
+  using Sh = PairShape<BN, NUM_A, A_MN, B_MN, STAGES>;
+  constexpr size_t kSmem = Sh::kSmem;
+  static_assert(kSmem <= 232448, "shared memory per CTA");
+  auto kern = gemm_pair_kernel<BN, NUM_A, A_MN, B_MN, STAGES, Epi>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(kSmem));
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = kSmem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  static int max_clusters[64] = {0};
+  int dev = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (max_clusters[dev] == 0) {
+    int n = 0;
+    cfg.gridDim = dim3(2 * 512, 1, 1);
+    if ((e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg)) != cudaSuccess) return e;
+    max_clusters[dev] = n > 0 ? n : 1;
+  }
+  const int pairs = std::max(1, std::min(g.num_units, max_clusters[dev]));
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  e = cudaLaunchKernelEx(&cfg, kern, a0, a1, b, g, p, c);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
 cudaError_t launch_fwd_ce(const CUtensorMap& tH, const CUtensorMap& tW, const GemmGeom& g,
                           const FwdParams& p, const DevCtl& c, int grid, cudaStream_t s) {
-  return launch_gemm<kBnSingle, 1, false, false, EpiFwdCE>(tH, tH, tW, g, p, c, grid, s);
+  (void)grid;
+  return launch_gemm_pair<kBnSingle, 1, false, false, 6, EpiFwdCE>(tH, tH, tW, g, p, c, s);
 }
 cudaError_t launch_fwd_dual(const CUtensorMap& tHq, const CUtensorMap& tHp, const CUtensorMap& tW,
                             const GemmGeom& g, const FwdParams& p, const DevCtl& c, int grid,
                             cudaStream_t s) {
-  return launch_gemm<kBnDual, 2, false, false, EpiFwdDual>(tHq, tHp, tW, g, p, c, grid, s);
+  (void)grid;
+  return launch_gemm_pair<kBnDual, 2, false, false, 5, EpiFwdDual>(tHq, tHp, tW, g, p, c, s);
 }
 cudaError_t launch_alpha(const CUtensorMap& tHq, const CUtensorMap& tHp, const CUtensorMap& tW,
                          const GemmGeom& g, const FwdParams& p, const DevCtl& c, int grid,
                          cudaStream_t s) {
-  return launch_gemm<kBnDual, 2, false, false, EpiAlpha>(tHq, tHp, tW, g, p, c, grid, s);
+  (void)grid;
+  return launch_gemm_pair<kBnDual, 2, false, false, 5, EpiAlpha>(tHq, tHp, tW, g, p, c, s);
 }
 cudaError_t launch_dz_ce(const CUtensorMap& tH, const CUtensorMap& tW, const GemmGeom& g,
                          const DzParams& p, const DevCtl& c, int grid, cudaStream_t s) {
-  return launch_gemm<kBnSingle, 1, false, false, EpiDz<false>>(tH, tH, tW, g, p, c, grid, s);
+  (void)grid;
+  return launch_gemm_pair<kBnSingle, 1, false, false, 6, EpiDz<false>>(tH, tH, tW, g, p, c, s);
 }
 cudaError_t launch_dz_dual(const CUtensorMap& tHq, const CUtensorMap& tHp, const CUtensorMap& tW,
                            const GemmGeom& g, const DzParams& p, const DevCtl& c, int grid,
                            cudaStream_t s) {
-  return launch_gemm<kBnDual, 2, false, false, EpiDz<true>>(tHq, tHp, tW, g, p, c, grid, s);
+  (void)grid;
+  return launch_gemm_pair<kBnDual, 2, false, false, 5, EpiDz<true>>(tHq, tHp, tW, g, p, c, s);
 }
 cudaError_t launch_dh(const CUtensorMap& tDz, const CUtensorMap& tW, const GemmGeom& g,
                       const DhParams& p, const DevCtl& c, int grid, cudaStream_t s) {
-  return launch_gemm<kBnGrad, 1, false, true, EpiDh>(tDz, tDz, tW, g, p, c, grid, s);
+  (void)grid;
+  return launch_gemm_pair<kBnGrad, 1, false, true, 6, EpiDh>(tDz, tDz, tW, g, p, c, s);
 }
 cudaError_t launch_dw(const CUtensorMap& tDzT, const CUtensorMap& tH, const GemmGeom& g,
                       const DwParams& p, const DevCtl& c, int grid, cudaStream_t s) {
-  return launch_gemm<kBnGrad, 1, true, true, EpiDw>(tDzT, tDzT, tH, g, p, c, grid, s);
+  (void)grid;
+  return launch_gemm_pair<kBnGrad, 1, true, true, 6, EpiDw>(tDzT, tDzT, tH, g, p, c, s);
 }
 
 // ----------------------------------------------------------------------------------------
