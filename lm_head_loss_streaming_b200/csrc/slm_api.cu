@@ -38,20 +38,22 @@ bool valid_kind(int k) { return k >= SLM_CE && k <= SLM_LK_HYBRID; }
 bool dual_kind(int k) { return k != SLM_CE; }
 bool alpha_kind(int k) { return k == SLM_TV || k == SLM_NLA || k == SLM_LK_HYBRID; }
 
-// Forward vocabulary schedule: tiles of BN columns, grouped into at most 64 runs per row
-// (so the per-row partials stay O(N)), each run at least 2048 columns long.
+// Forward vocabulary schedule: tiles of `bn` columns, grouped into at most 32 runs per row
+// (so the per-row partials stay O(N)), each run at least 2048 columns long.  Each run
+// leaves kFwdPartsPerRun partial slots per row (one per epilogue warpgroup).
 struct FwdSched {
-  int bn, num_n, vc, units_n, fields;
+  int bn, num_n, vc, units_n, slots, fields;
 };
 
 FwdSched fwd_sched(int kind, int64_t V) {
   FwdSched f;
-  f.bn = dual_kind(kind) ? kBnDual : kBnSingle;
+  f.bn = dual_kind(kind) ? kTileDual : kTileCE;
   f.num_n = static_cast<int>(ceil_div(V, f.bn));
   const int min_vc = 2048 / f.bn;
-  f.vc = std::max<int>(min_vc, static_cast<int>(ceil_div(f.num_n, 64)));
+  f.vc = std::max<int>(min_vc, static_cast<int>(ceil_div(f.num_n, 32)));
   f.vc = std::min(f.vc, f.num_n);
   f.units_n = static_cast<int>(ceil_div(f.num_n, f.vc));
+  f.slots = f.units_n * kFwdPartsPerRun;
   f.fields = dual_kind(kind) ? 5 : 2;
   return f;
 }
@@ -77,7 +79,7 @@ Layout layout(int kind, int64_t N, int64_t d, int64_t V, int64_t chunk_tokens) {
   size_t off = align_up(L.red_off + L.nblk * (sizeof(double) + sizeof(long long)), kAlign);
   L.big_off = off;
   const FwdSched f = fwd_sched(kind, V);
-  const size_t part = static_cast<size_t>(f.units_n) * f.fields * static_cast<size_t>(N) * 4;
+  const size_t part = static_cast<size_t>(f.slots) * f.fields * static_cast<size_t>(N) * 4;
   L.part_off = off;
   L.zy_off = align_up(L.part_off + part, kAlign);
   const size_t fwd_end = align_up(L.zy_off + static_cast<size_t>(N) * 4, kAlign);
@@ -161,11 +163,6 @@ GemmGeom geom(int64_t M, int64_t Nn, int64_t K, int bn, int vc, int group_m, int
   g.units_n = static_cast<int>(ceil_div(g.num_n, g.vc));
   g.num_units = g.num_m * g.units_n;
   return g;
-}
-
-int grid_for(const GemmGeom& g) {
-  const int sms = sm_count();
-  return std::max(1, std::min(g.num_units, sms > 0 ? sms : 148));
 }
 
 // `backward` selects which pass's workspace needs are checked.
@@ -256,20 +253,19 @@ int slm_loss_fwd(int kind, const void* Hq, const void* Hp, const void* W, const 
     const GemmGeom g = geom(N, V, d, f.bn, f.vc, kGroupPairs, kPairM);
     CUtensorMap tHq, tHp, tW;
     if (!make_map(&tHq, Hq, d, N, d, kBK, kBM)) return SLM_ERR_CUDA;
-    if (!make_map(&tW, W, d, V, d, kBK, f.bn / 2)) return SLM_ERR_CUDA;
+    if (!make_map(&tW, W, d, V, d, kBK, 128)) return SLM_ERR_CUDA;
     FwdParams p{labels, ignore_index, N, V, part, zy, stats};
-    const int grid = grid_for(g);
     if (!dual_kind(kind)) {
-      SLM_TRY_CUDA(launch_fwd_ce(tHq, tW, g, p, ctl, grid, s));
+      SLM_TRY_CUDA(launch_fwd_ce(tHq, tW, g, p, ctl, s));
     } else {
       if (!make_map(&tHp, Hp, d, N, d, kBK, kBM)) return SLM_ERR_CUDA;
-      SLM_TRY_CUDA(launch_fwd_dual(tHq, tHp, tW, g, p, ctl, grid, s));
+      SLM_TRY_CUDA(launch_fwd_dual(tHq, tHp, tW, g, p, ctl, s));
     }
-    SLM_TRY_CUDA(launch_combine(kind, 1, part, f.units_n, zy, labels, ignore_index, N, V,
+    SLM_TRY_CUDA(launch_combine(kind, 1, part, f.slots, zy, labels, ignore_index, N, V,
                                 loss_tok, alpha_tok, stats, blk_sum, blk_cnt, status, s));
     if (alpha_kind(kind)) {
-      SLM_TRY_CUDA(launch_alpha(tHq, tHp, tW, g, p, ctl, grid, s));
-      SLM_TRY_CUDA(launch_combine(kind, 2, part, f.units_n, zy, labels, ignore_index, N, V,
+      SLM_TRY_CUDA(launch_alpha(tHq, tHp, tW, g, p, ctl, s));
+      SLM_TRY_CUDA(launch_combine(kind, 2, part, f.slots, zy, labels, ignore_index, N, V,
                                   loss_tok, alpha_tok, stats, blk_sum, blk_cnt, status, s));
     }
     SLM_TRY_CUDA(launch_finalize(blk_sum, blk_cnt, static_cast<int>(L.nblk), loss_sum, n_valid,
@@ -308,7 +304,7 @@ int slm_loss_bwd(int kind, const void* Hq, const void* Hp, const void* W, const 
   const int64_t C = default_chunk(N, d, chunk_tokens);
   const FwdSched f = fwd_sched(kind, V);
   CUtensorMap tW_k, tW_mn;
-  if (!make_map(&tW_k, W, d, V, d, kBK, f.bn / 2)) return SLM_ERR_CUDA;
+  if (!make_map(&tW_k, W, d, V, d, kBK, 128)) return SLM_ERR_CUDA;
   if (!make_map(&tW_mn, W, d, V, d, 64, 64)) return SLM_ERR_CUDA;
   const int64_t ldz = static_cast<int64_t>(L.ldz);
 
@@ -322,24 +318,24 @@ int slm_loss_bwd(int kind, const void* Hq, const void* Hp, const void* W, const 
     DzParams pz{kind, labels, ignore_index, c0, rows, N, V, stats, grad_tok, grad_scale,
                 n_valid, dz, ldz};
     if (!dual_kind(kind)) {
-      SLM_TRY_CUDA(launch_dz_ce(tHq, tW_k, gz, pz, ctl, grid_for(gz), s));
+      SLM_TRY_CUDA(launch_dz_ce(tHq, tW_k, gz, pz, ctl, s));
     } else {
       const __nv_bfloat16* hp = static_cast<const __nv_bfloat16*>(Hp) + c0 * d;
       if (!make_map(&tHp, hp, d, rows, d, kBK, kBM)) return SLM_ERR_CUDA;
-      SLM_TRY_CUDA(launch_dz_dual(tHq, tHp, tW_k, gz, pz, ctl, grid_for(gz), s));
+      SLM_TRY_CUDA(launch_dz_dual(tHq, tHp, tW_k, gz, pz, ctl, s));
     }
     // 2) dH[chunk] = dZ W   (M = rows, N = d, K = V; W read MN-major).
     CUtensorMap tDz_k, tDz_mn, tH_mn;
     if (!make_map(&tDz_k, dz, V, rows, ldz, kBK, kBM)) return SLM_ERR_CUDA;
-    const GemmGeom gh = geom(rows, d, V, kBnGrad, 1, 1, kPairM);
+    const GemmGeom gh = geom(rows, d, V, kTileDh, 1, 1, kPairM);
     DhParams ph{static_cast<__nv_bfloat16*>(dHq), c0, rows, d};
-    SLM_TRY_CUDA(launch_dh(tDz_k, tW_mn, gh, ph, ctl, grid_for(gh), s));
+    SLM_TRY_CUDA(launch_dh(tDz_k, tW_mn, gh, ph, ctl, s));
     // 3) dW (+)= dZ^T H[chunk]   (M = V, N = d, K = rows; both operands MN-major).
     if (!make_map(&tDz_mn, dz, V, rows, ldz, 64, 64)) return SLM_ERR_CUDA;
     if (!make_map(&tH_mn, hq, d, rows, d, 64, 64)) return SLM_ERR_CUDA;
-    const GemmGeom gw = geom(V, d, rows, kBnGrad, 1, 1, kPairM);
+    const GemmGeom gw = geom(V, d, rows, kTileDw, 1, 1, kPairM);
     DwParams pw{dW, V, d, (accumulate_dW || c0 > 0) ? 1 : 0};
-    SLM_TRY_CUDA(launch_dw(tDz_mn, tH_mn, gw, pw, ctl, grid_for(gw), s));
+    SLM_TRY_CUDA(launch_dw(tDz_mn, tH_mn, gw, pw, ctl, s));
   }
   return SLM_OK;
 }

@@ -9,18 +9,18 @@
 
 namespace slm {
 
-// Tile shape of every GEMM: 128 rows of the M operand per CTA tile (one TMEM lane per
-// row), 64 bf16 of K per pipeline stage (one 128-byte swizzle row).
-constexpr int kBM = 128;
-constexpr int kBK = 64;
-constexpr int kStages = 4;
-constexpr int kThreads = 192;  // warp 0: TMA producer, warp 1: MMA issuer, warps 2-5: epilogue
-
-// N tile of the forward / logits-gradient GEMMs: 256 vocabulary columns with one
-// accumulator (CE), 128 columns with two accumulators (target and draft logits).
-constexpr int kBnSingle = 256;
-constexpr int kBnDual = 128;
-constexpr int kBnGrad = 256;  // dH and dW GEMMs
+// Tile shape of every GEMM: a 2-SM CTA pair computes 256 rows of the M operand (128 per
+// CTA, one TMEM lane per row) with 64 bf16 of K per pipeline stage (one 128-byte swizzle
+// row).  N tile widths (columns of one accumulator):
+constexpr int kBM = 128;          // M rows per CTA
+constexpr int kBK = 64;           // K per stage
+constexpr int kTileCE = 512;      // CE forward / logits-gradient: one accumulator, 2 x 256-wide MMAs
+constexpr int kTileDual = 256;    // target + draft: two accumulators of 256 columns
+constexpr int kTileDh = 512;      // dH = dZ W
+constexpr int kTileDw = 256;      // dW += dZ^T H (double-buffered)
+// The forward epilogue runs as two warpgroups, each over half of the tile's columns, and
+// each writes its own per-row partial statistics: partial slots per vocabulary run.
+constexpr int kFwdPartsPerRun = 2;
 
 // Device status word bits.
 constexpr int kFlagLabelRange = 1;
@@ -51,7 +51,7 @@ struct FwdParams {
   const int32_t* labels;  // CE labels (required for CE)
   int32_t ignore_index;
   int64_t N, V;
-  float* part;         // [units_n][fields][N]
+  float* part;         // [units_n * kFwdPartsPerRun][fields][N]
   float* zy;           // [N] label logit (CE)
   const float* stats;  // pass 2: L_q, L_p
 };
@@ -82,25 +82,25 @@ struct DwParams {
   int beta;  // 1: add to dW, 0: overwrite
 };
 
-// Kernel launchers (slm_kernels.cu).  Each returns cudaGetLastError() after the launch.
+// Kernel launchers (slm_kernels.cu).  Each returns the launch's error status.
 int sm_count();
 cudaError_t launch_fwd_ce(const CUtensorMap& tH, const CUtensorMap& tW, const GemmGeom& g,
-                          const FwdParams& p, const DevCtl& c, int grid, cudaStream_t s);
+                          const FwdParams& p, const DevCtl& c, cudaStream_t s);
 cudaError_t launch_fwd_dual(const CUtensorMap& tHq, const CUtensorMap& tHp,
                             const CUtensorMap& tW, const GemmGeom& g, const FwdParams& p,
-                            const DevCtl& c, int grid, cudaStream_t s);
+                            const DevCtl& c, cudaStream_t s);
 cudaError_t launch_alpha(const CUtensorMap& tHq, const CUtensorMap& tHp, const CUtensorMap& tW,
-                         const GemmGeom& g, const FwdParams& p, const DevCtl& c, int grid,
+                         const GemmGeom& g, const FwdParams& p, const DevCtl& c,
                          cudaStream_t s);
 cudaError_t launch_dz_ce(const CUtensorMap& tH, const CUtensorMap& tW, const GemmGeom& g,
-                         const DzParams& p, const DevCtl& c, int grid, cudaStream_t s);
+                         const DzParams& p, const DevCtl& c, cudaStream_t s);
 cudaError_t launch_dz_dual(const CUtensorMap& tHq, const CUtensorMap& tHp, const CUtensorMap& tW,
-                           const GemmGeom& g, const DzParams& p, const DevCtl& c, int grid,
+                           const GemmGeom& g, const DzParams& p, const DevCtl& c,
                            cudaStream_t s);
 cudaError_t launch_dh(const CUtensorMap& tDz, const CUtensorMap& tW, const GemmGeom& g,
-                      const DhParams& p, const DevCtl& c, int grid, cudaStream_t s);
+                      const DhParams& p, const DevCtl& c, cudaStream_t s);
 cudaError_t launch_dw(const CUtensorMap& tDzT, const CUtensorMap& tH, const GemmGeom& g,
-                      const DwParams& p, const DevCtl& c, int grid, cudaStream_t s);
+                      const DwParams& p, const DevCtl& c, cudaStream_t s);
 
 // Row combines and the deterministic loss reduction.
 cudaError_t launch_combine(int kind, int pass, const float* part, int nch, const float* zy,

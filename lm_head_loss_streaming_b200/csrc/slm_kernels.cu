@@ -1,13 +1,19 @@
 // slm_kernels.cu - sm_100a kernels of the streaming LM-head loss.
 //
-// One warp-specialised persistent GEMM skeleton serves every contraction of the path:
-//   warp 0      TMA producer: 2-D tiled loads of the A / B operand tiles into a 4-stage
-//               shared-memory ring (128-byte swizzle), completion on "full" mbarriers;
-//   warp 1      MMA issuer: one lane issues tcgen05.mma (bf16 x bf16 -> fp32) into one of
-//               two TMEM accumulator buffers; tcgen05.commit frees ring stages and
-//               publishes finished accumulators;
-//   warps 2-5   epilogue: one thread per tile row reads its row from TMEM (tcgen05.ld)
-//               and applies the fused epilogue while the MMA warp fills the other buffer.
+// One warp-specialised persistent GEMM skeleton serves every contraction of the path.  A
+// cluster of two CTAs (one per SM) shares each tensor-core MMA (tcgen05.mma.cta_group::2,
+// M = 256): CTA r of the pair holds rows [128 r, 128 r + 128) of the A operand tile and
+// half of every B slice in its own shared memory, and receives its 128 accumulator rows
+// in its own tensor memory (TMEM).
+//   warp 0      TMA producer (both CTAs): 2-D tiled loads with 128-byte swizzle into a
+//               ring of shared-memory stages; both CTAs' copies complete on the leader
+//               CTA's "full" barrier;
+//   warp 1      MMA issuer (leader CTA only): one lane issues the pair's MMAs (bf16 x bf16
+//               -> fp32) and releases ring stages and accumulators in both CTAs with
+//               multicast tcgen05.commit;
+//   warps 2..   epilogue (both CTAs): one or two warpgroups, one thread per tile row, each
+//               warpgroup over its share of the tile's columns, reading TMEM with
+//               tcgen05.ld and applying the fused epilogue.
 // The epilogues are what make the path streaming ("Training speculative decoders:
 // removing the logits and attention bottlenecks", "Streaming Cross Entropy" and
 // "Backward pass"): logits tiles live only in TMEM and registers.
@@ -34,16 +40,6 @@ using namespace sm100;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr uint32_t kTmemCols = 512;
-
-struct PipeCtl {
-  uint64_t full[kStages];
-  uint64_t empty[kStages];
-  uint64_t tfull[2];
-  uint64_t tempty[2];
-  uint64_t fin;
-  uint32_t tmem_base;
-  int abort;
-};
 
 // Bounded wait executed by all 32 lanes of a warp; the result is warp-uniform.
 // honor_abort = false is used for the final waits on a CTA's own in-flight work.
@@ -77,206 +73,13 @@ __device__ __forceinline__ void unit_coords(const GemmGeom& g, int u, int& mt, i
 }
 
 // ----------------------------------------------------------------------------------------
-// The GEMM skeleton.  A: NUM_A operands of 128 x kBK per stage (K-major: box {64, 128};
-// MN-major: two boxes {64, 64}); B: BN x kBK (K-major: box {64, BN}; MN-major: BN/64
-// boxes {64, 64}).  Accumulator a of buffer b sits at TMEM columns (b * NUM_A + a) * BN.
-// ----------------------------------------------------------------------------------------
-template <int BN, int NUM_A, bool A_MN, bool B_MN, class Epi>
-__global__ void __launch_bounds__(kThreads, 1)
-    gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
-                const __grid_constant__ CUtensorMap tmB, const GemmGeom g,
-                const typename Epi::Params ep, const DevCtl ctl) {
-  constexpr uint32_t kABytes = kBM * kBK * 2;
-  constexpr uint32_t kBBytes = BN * kBK * 2;
-  constexpr uint32_t kStageBytes = NUM_A * kABytes + kBBytes;
-  constexpr uint32_t kAccCols = NUM_A * BN;
-  static_assert(2 * kAccCols <= kTmemCols, "two accumulator buffers must fit in TMEM");
-  static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "UMMA N");
-  constexpr uint32_t kIdesc = idesc_bf16_f32(kBM, BN, A_MN, B_MN);
-
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  PipeCtl* pc = reinterpret_cast<PipeCtl*>(smem + kStages * kStageBytes);
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&pc->full[s], 1);
-      mbar_init(&pc->empty[s], 1);
-    }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&pc->tfull[b], 1);
-      mbar_init(&pc->tempty[b], 4 * 32);
-    }
-    mbar_init(&pc->fin, 1);
-    pc->abort = 0;
-    fence_barrier_init();
-  }
-  if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tmA0);
-    if (NUM_A == 2) tma_prefetch_desc(&tmA1);
-    tma_prefetch_desc(&tmB);
-  }
-  if (warp == 1) {
-    tmem_alloc(&pc->tmem_base, kTmemCols);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = pc->tmem_base;
-  volatile int* abort = &pc->abort;
-
-  if (warp == 0) {
-    // ------------------------------ TMA producer ------------------------------
-    uint32_t it = 0;
-    bool ok = true;
-    for (int u = blockIdx.x; ok && u < g.num_units; u += gridDim.x) {
-      int mt, j;
-      unit_coords(g, u, mt, j);
-      const int n_end = min((j + 1) * g.vc, g.num_n);
-      for (int nt = j * g.vc; ok && nt < n_end; ++nt) {
-        for (int kb = 0; kb < g.k_blocks; ++kb, ++it) {
-          const int s = it % kStages;
-          const uint32_t ph = (it / kStages) & 1u;
-          if (!wait_warp(&pc->empty[s], ph ^ 1u, abort, ctl)) {
-            ok = false;
-            break;
-          }
-          if (lane == 0) {
-            uint8_t* st = smem + s * kStageBytes;
-            mbar_arrive_expect_tx(&pc->full[s], kStageBytes);
-            const int k0 = kb * kBK;
-#pragma unroll
-            for (int a = 0; a < NUM_A; ++a) {
-              const CUtensorMap* map = (a == 0) ? &tmA0 : &tmA1;
-              uint8_t* dst = st + a * kABytes;
-              if (A_MN) {
-                tma_load_2d(dst, map, &pc->full[s], mt * kBM, k0);
-                tma_load_2d(dst + 8192, map, &pc->full[s], mt * kBM + 64, k0);
-              } else {
-                tma_load_2d(dst, map, &pc->full[s], k0, mt * kBM);
-              }
-            }
-            uint8_t* bdst = st + NUM_A * kABytes;
-            if (B_MN) {
-#pragma unroll
-              for (int jb = 0; jb < BN / 64; ++jb)
-                tma_load_2d(bdst + jb * 8192, &tmB, &pc->full[s], nt * BN + jb * 64, k0);
-            } else {
-              tma_load_2d(bdst, &tmB, &pc->full[s], k0, nt * BN);
-            }
-          }
-          __syncwarp();
-        }
-      }
-    }
-    if (!ok) {
-      // Let this CTA's own copies in flight land before the CTA exits.
-      const uint32_t first = it > (uint32_t)kStages ? it - kStages : 0u;
-      for (uint32_t i = first; i < it; ++i)
-        wait_warp(&pc->full[i % kStages], (i / kStages) & 1u, abort, ctl, false);
-    }
-  } else if (warp == 1) {
-    // ------------------------------ MMA issuer ------------------------------
-    uint32_t it = 0, t = 0;
-    bool ok = true;
-    for (int u = blockIdx.x; ok && u < g.num_units; u += gridDim.x) {
-      int mt, j;
-      unit_coords(g, u, mt, j);
-      const int n_end = min((j + 1) * g.vc, g.num_n);
-      for (int nt = j * g.vc; ok && nt < n_end; ++nt, ++t) {
-        const int b = t & 1;
-        const uint32_t ub = (t >> 1) & 1u;
-        if (!wait_warp(&pc->tempty[b], ub ^ 1u, abort, ctl)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t dcol = tmem + b * kAccCols;
-        for (int kb = 0; kb < g.k_blocks; ++kb, ++it) {
-          const int s = it % kStages;
-          const uint32_t ph = (it / kStages) & 1u;
-          if (!wait_warp(&pc->full[s], ph, abort, ctl)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          if (lane == 0) {
-            const uint32_t a_addr = smem_u32(smem + s * kStageBytes);
-            const uint32_t b_addr = a_addr + NUM_A * kABytes;
-#pragma unroll
-            for (int kk = 0; kk < kBK / 16; ++kk) {
-              const uint64_t bd = B_MN ? smem_desc_sw128(b_addr + kk * 2048, 8192, 1024)
-                                       : smem_desc_sw128(b_addr + kk * 32, 16, 1024);
-#pragma unroll
-              for (int a = 0; a < NUM_A; ++a) {
-                const uint32_t aa = a_addr + a * kABytes;
-                const uint64_t ad = A_MN ? smem_desc_sw128(aa + kk * 2048, 8192, 1024)
-                                         : smem_desc_sw128(aa + kk * 32, 16, 1024);
-                umma_bf16(dcol + a * BN, ad, bd, kIdesc, (kb | kk) != 0 ? 1u : 0u);
-              }
-            }
-            umma_commit(&pc->empty[s]);
-          }
-          __syncwarp();
-        }
-        if (!ok) break;
-        if (lane == 0) umma_commit(&pc->tfull[b]);
-        __syncwarp();
-      }
-    }
-    // Every MMA this thread issued must be complete before TMEM is released.
-    if (lane == 0) umma_commit(&pc->fin);
-    __syncwarp();
-    wait_warp(&pc->fin, 0u, abort, ctl, false);
-  } else {
-    // ------------------------------ epilogue ------------------------------
-    const int q = warp & 3;  // a warp may only touch TMEM lanes [32 * (warp % 4), +32)
-    const int row = q * 32 + lane;
-    const uint32_t lane_bits = static_cast<uint32_t>(q * 32) << 16;
-    Epi epi;
-    uint32_t t = 0;
-    bool ok = true;
-    for (int u = blockIdx.x; ok && u < g.num_units; u += gridDim.x) {
-      int mt, j;
-      unit_coords(g, u, mt, j);
-      const int n_end = min((j + 1) * g.vc, g.num_n);
-      epi.unit_begin(ep, mt * kBM, j, row);
-      for (int nt = j * g.vc; nt < n_end; ++nt, ++t) {
-        const int b = t & 1;
-        const uint32_t ub = (t >> 1) & 1u;
-        if (!wait_warp(&pc->tfull[b], ub, abort, ctl)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        epi.template tile<BN>(ep, tmem + lane_bits + b * kAccCols, mt * kBM, nt, row);
-        tc_fence_before();
-        mbar_arrive(&pc->tempty[b]);
-      }
-      if (!ok) break;
-      epi.unit_end(ep, mt * kBM, j, row);
-    }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, kTmemCols);
-}
-
-// ----------------------------------------------------------------------------------------
-// The 2-SM skeleton: a cluster of two CTAs shares each MMA (cta_group::2, M = 256).
-// CTA r of the pair loads rows [128 r, 128 r + 128) of its 256-row M tile and columns
-// [r BN/2, (r + 1) BN/2) of the N tile into its own shared memory; both CTAs' copies count
-// on the leader's "full" barrier; the leader's single MMA thread multiplies the pair's
-// operands into both CTAs' TMEM and releases stages and accumulators in both CTAs with
-// multicast commits; each CTA's epilogue reads its own 128 accumulator rows and reports
-// back to the leader.  Per CTA, a stage of shared memory holds half the B operand of the
-// 1-CTA form, which halves the shared-memory operand traffic per flop.
+// Pair GEMM configuration.
+//   BNI    N of one MMA instruction (<= 256); each CTA holds BNI / 2 of it ("B slice")
+//   NSUB   MMA instructions along N per accumulator: tile N = NSUB * BNI
+//   NUM_A  A operands sharing the B tile, one accumulator each (1, or 2 for target+draft)
+//   NBUF   TMEM accumulator buffers (2: the epilogue of one tile overlaps the next tile's
+//          MMAs; 1: wider tiles, fewer bytes from L2 per flop)
+//   NWG    epilogue warpgroups, each over 1/NWG of the tile's columns
 // ----------------------------------------------------------------------------------------
 template <int STAGES>
 struct PairCtl {
@@ -289,31 +92,39 @@ struct PairCtl {
   int abort;
 };
 
-template <int BN, int NUM_A, bool A_MN, bool B_MN, int STAGES>
-struct PairShape {
-  static constexpr int kBNH = BN / 2;  // B rows (K-major) or columns (MN-major) per CTA
+template <int BNI, int NSUB, int NUM_A, int NBUF, int NWG, bool A_MN, bool B_MN, int STAGES>
+struct PairCfg {
+  static constexpr int kTileN = NSUB * BNI;
+  static constexpr int kSliceN = BNI / 2;
   static constexpr uint32_t kABytes = kBM * kBK * 2;
-  static constexpr uint32_t kBBytes = kBNH * kBK * 2;
-  static constexpr uint32_t kStageBytes = NUM_A * kABytes + kBBytes;
-  static constexpr size_t kSmem = 1024 + STAGES * static_cast<size_t>(kStageBytes) +
-                                  sizeof(PairCtl<STAGES>);
+  static constexpr uint32_t kSliceBytes = kSliceN * kBK * 2;
+  static constexpr uint32_t kStageBytes = NUM_A * kABytes + NSUB * kSliceBytes;
+  static constexpr uint32_t kAccCols = NUM_A * kTileN;  // TMEM columns per buffer
+  static constexpr int kThreads = 64 + 128 * NWG;
+  static constexpr int kEpiCols = kTileN / NWG;  // columns per epilogue warpgroup
+  static constexpr size_t kSmem =
+      1024 + STAGES * static_cast<size_t>(kStageBytes) + sizeof(PairCtl<STAGES>);
+  static_assert(NBUF * kAccCols <= kTmemCols, "accumulator buffers must fit in TMEM");
+  static_assert(BNI % 128 == 0 && BNI <= 256, "UMMA N (M = 256) and whole 64-wide B boxes");
+  static_assert(kEpiCols % 32 == 0, "epilogue column share");
+  static_assert(kSmem <= 232448, "shared memory per CTA");
 };
 
-template <int BN, int NUM_A, bool A_MN, bool B_MN, int STAGES, class Epi>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int BNI, int NSUB, int NUM_A, int NBUF, int NWG, bool A_MN, bool B_MN, int STAGES,
+          class Epi>
+__global__ void __launch_bounds__(64 + 128 * NWG, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0,
                      const __grid_constant__ CUtensorMap tmA1,
                      const __grid_constant__ CUtensorMap tmB, const GemmGeom g,
                      const typename Epi::Params ep, const DevCtl ctl) {
-  using Sh = PairShape<BN, NUM_A, A_MN, B_MN, STAGES>;
-  constexpr int kBNH = Sh::kBNH;
-  constexpr uint32_t kABytes = Sh::kABytes;
-  constexpr uint32_t kStageBytes = Sh::kStageBytes;
-  constexpr uint32_t kAccCols = NUM_A * BN;
-  static_assert(2 * kAccCols <= kTmemCols, "two accumulator buffers must fit in TMEM");
-  static_assert(BN % 32 == 0 && BN >= 64 && BN <= 256, "UMMA N for M = 256");
-  static_assert(kBNH % 64 == 0, "each CTA's B half is whole 64-element boxes");
-  constexpr uint32_t kIdesc = idesc_bf16_f32(2 * kBM, BN, A_MN, B_MN);
+  using C = PairCfg<BNI, NSUB, NUM_A, NBUF, NWG, A_MN, B_MN, STAGES>;
+  constexpr int kTileN = C::kTileN;
+  constexpr int kSliceN = C::kSliceN;
+  constexpr uint32_t kABytes = C::kABytes;
+  constexpr uint32_t kSliceBytes = C::kSliceBytes;
+  constexpr uint32_t kStageBytes = C::kStageBytes;
+  constexpr uint32_t kAccCols = C::kAccCols;
+  constexpr uint32_t kIdesc = idesc_bf16_f32(2 * kBM, BNI, A_MN, B_MN);
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -333,7 +144,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&pc->tfull[b], 1);
-      mbar_init(&pc->tempty[b], 2 * 4);  // one arrive per epilogue warp of both CTAs
+      mbar_init(&pc->tempty[b], 2 * 4 * NWG);  // one arrive per epilogue warp, both CTAs
     }
     mbar_init(&pc->fin, 1);
     pc->abort = 0;
@@ -365,7 +176,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int mrow = mt * 2 * kBM + static_cast<int>(rank) * kBM;
       const int n_end = min((j + 1) * g.vc, g.num_n);
       for (int nt = j * g.vc; ok && nt < n_end; ++nt) {
-        const int ncol = nt * BN + static_cast<int>(rank) * kBNH;
         for (int kb = 0; kb < g.k_blocks; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
@@ -388,13 +198,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tma_load_2d_pair(dst, map, &pc->full[s], k0, mrow);
               }
             }
-            uint8_t* bdst = st + NUM_A * kABytes;
-            if (B_MN) {
 #pragma unroll
-              for (int jb = 0; jb < kBNH / 64; ++jb)
-                tma_load_2d_pair(bdst + jb * 8192, &tmB, &pc->full[s], ncol + jb * 64, k0);
-            } else {
-              tma_load_2d_pair(bdst, &tmB, &pc->full[s], k0, ncol);
+            for (int sub = 0; sub < NSUB; ++sub) {
+              uint8_t* bdst = st + NUM_A * kABytes + sub * kSliceBytes;
+              const int ncol = nt * kTileN + sub * BNI + static_cast<int>(rank) * kSliceN;
+              if (B_MN) {
+#pragma unroll
+                for (int jb = 0; jb < kSliceN / 64; ++jb)
+                  tma_load_2d_pair(bdst + jb * 8192, &tmB, &pc->full[s], ncol + jb * 64, k0);
+              } else {
+                tma_load_2d_pair(bdst, &tmB, &pc->full[s], k0, ncol);
+              }
             }
           }
           __syncwarp();
@@ -422,8 +236,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         unit_coords(g, u, mt, j);
         const int n_end = min((j + 1) * g.vc, g.num_n);
         for (int nt = j * g.vc; ok && nt < n_end; ++nt, ++t) {
-          const int b = t & 1;
-          const uint32_t ub = (t >> 1) & 1u;
+          const int b = (NBUF == 2) ? static_cast<int>(t & 1u) : 0;
+          const uint32_t ub = (NBUF == 2) ? ((t >> 1) & 1u) : (t & 1u);
           if (!wait_warp(&pc->tempty[b], ub ^ 1u, abort, ctl)) {
             ok = false;
             break;
@@ -443,14 +257,19 @@ __global__ void __launch_bounds__(kThreads, 1)
               const uint32_t b_addr = a_addr + NUM_A * kABytes;
 #pragma unroll
               for (int kk = 0; kk < kBK / 16; ++kk) {
-                const uint64_t bd = B_MN ? smem_desc_sw128(b_addr + kk * 2048, 8192, 1024)
-                                         : smem_desc_sw128(b_addr + kk * 32, 16, 1024);
 #pragma unroll
-                for (int a = 0; a < NUM_A; ++a) {
-                  const uint32_t aa = a_addr + a * kABytes;
-                  const uint64_t ad = A_MN ? smem_desc_sw128(aa + kk * 2048, 8192, 1024)
-                                           : smem_desc_sw128(aa + kk * 32, 16, 1024);
-                  umma_bf16_pair(dcol + a * BN, ad, bd, kIdesc, (kb | kk) != 0 ? 1u : 0u);
+                for (int sub = 0; sub < NSUB; ++sub) {
+                  const uint32_t bs = b_addr + sub * kSliceBytes;
+                  const uint64_t bd = B_MN ? smem_desc_sw128(bs + kk * 2048, 8192, 1024)
+                                           : smem_desc_sw128(bs + kk * 32, 16, 1024);
+#pragma unroll
+                  for (int a = 0; a < NUM_A; ++a) {
+                    const uint32_t aa = a_addr + a * kABytes;
+                    const uint64_t ad = A_MN ? smem_desc_sw128(aa + kk * 2048, 8192, 1024)
+                                             : smem_desc_sw128(aa + kk * 32, 16, 1024);
+                    umma_bf16_pair(dcol + (a * NSUB + sub) * BNI, ad, bd, kIdesc,
+                                   (kb | kk) != 0 ? 1u : 0u);
+                  }
                 }
               }
               umma_commit_pair_mc(&pc->empty[s], 0x3);
@@ -470,8 +289,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------ epilogue (both CTAs) ------------------------------
     const int q = warp & 3;  // a warp may only touch TMEM lanes [32 * (warp % 4), +32)
+    const int wg = (warp - 2) >> 2;
     const int row = q * 32 + lane;
     const uint32_t lane_bits = static_cast<uint32_t>(q * 32) << 16;
+    const int c0 = wg * C::kEpiCols;
+    const int c1 = c0 + C::kEpiCols;
     const uint32_t tempty_leader0 = mapa_shared(smem_u32(&pc->tempty[0]), 0);
     const uint32_t tempty_leader1 = mapa_shared(smem_u32(&pc->tempty[1]), 0);
     Epi epi;
@@ -482,22 +304,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       unit_coords(g, u, mt, j);
       const int row0 = mt * 2 * kBM + static_cast<int>(rank) * kBM;
       const int n_end = min((j + 1) * g.vc, g.num_n);
-      epi.unit_begin(ep, row0, j, row);
+      epi.unit_begin(ep, row0, row);
       for (int nt = j * g.vc; nt < n_end; ++nt, ++t) {
-        const int b = t & 1;
-        const uint32_t ub = (t >> 1) & 1u;
+        const int b = (NBUF == 2) ? static_cast<int>(t & 1u) : 0;
+        const uint32_t ub = (NBUF == 2) ? ((t >> 1) & 1u) : (t & 1u);
         if (!wait_warp(&pc->tfull[b], ub, abort, ctl)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        epi.template tile<BN>(ep, tmem + lane_bits + b * kAccCols, row0, nt, row);
+        epi.template tile<kTileN>(ep, tmem + lane_bits + b * kAccCols, row0,
+                                  static_cast<int64_t>(nt) * kTileN, c0, c1, row);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(b ? tempty_leader1 : tempty_leader0);
       }
       if (!ok) break;
-      epi.unit_end(ep, row0, j, row);
+      epi.unit_end(ep, row0, j * NWG + wg, row);
     }
   }
 
@@ -509,7 +332,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ----------------------------------------------------------------------------------------
-// Epilogues.
+// Epilogues.  tile<TN>(p, tb, row0, n0, c0, c1, row): this thread owns row `row0 + row`
+// of the M operand; accumulator a's column c (of the TN-wide tile that starts at global
+// column n0) is at TMEM address tb + a * TN + c; the thread's warpgroup covers columns
+// [c0, c1).  unit_end receives the partial slot of (vocabulary run, warpgroup).
 // ----------------------------------------------------------------------------------------
 __device__ __forceinline__ float max32(const float (&v)[32]) {
   float m0 = fmaxf(v[0], v[1]), m1 = fmaxf(v[2], v[3]);
@@ -528,7 +354,8 @@ __device__ __forceinline__ void mask_tail(float (&v)[32], int64_t col0, int64_t 
 }
 
 // CE forward: per row, online max m (log2 units) and s = sum 2^(z log2e - m) over the
-// unit's vocabulary run, plus the label logit z_y when the label falls in the run.
+// warpgroup's columns of the unit's vocabulary run, plus the label logit z_y when the
+// label falls there.
 struct EpiFwdCE {
   using Params = FwdParams;
   float m, s, zyv;
@@ -536,7 +363,7 @@ struct EpiFwdCE {
   bool has_zy, row_ok;
   int64_t grow;
 
-  __device__ __forceinline__ void unit_begin(const Params& p, int row0, int, int row) {
+  __device__ __forceinline__ void unit_begin(const Params& p, int row0, int row) {
     m = -INFINITY;
     s = 0.f;
     has_zy = false;
@@ -546,12 +373,12 @@ struct EpiFwdCE {
     lab = row_ok ? p.labels[grow] : -1;
   }
 
-  template <int BN>
-  __device__ __forceinline__ void tile(const Params& p, uint32_t tb, int, int nt, int) {
-    const int64_t n0 = static_cast<int64_t>(nt) * BN;
+  template <int TN>
+  __device__ __forceinline__ void tile(const Params& p, uint32_t tb, int, int64_t n0, int c0,
+                                       int c1, int) {
     const int64_t rel = static_cast<int64_t>(lab) - n0;
 #pragma unroll 1
-    for (int c = 0; c < BN; c += 32) {
+    for (int c = c0; c < c1; c += 32) {
       float v[32];
       tmem_ld32(tb + c, v);
       tmem_ld_wait();
@@ -580,16 +407,16 @@ struct EpiFwdCE {
     }
   }
 
-  __device__ __forceinline__ void unit_end(const Params& p, int, int j, int) {
+  __device__ __forceinline__ void unit_end(const Params& p, int, int slot, int) {
     if (!row_ok) return;
-    p.part[(static_cast<int64_t>(j) * 2 + 0) * p.N + grow] = m;
-    p.part[(static_cast<int64_t>(j) * 2 + 1) * p.N + grow] = s;
+    p.part[(static_cast<int64_t>(slot) * 2 + 0) * p.N + grow] = m;
+    p.part[(static_cast<int64_t>(slot) * 2 + 1) * p.N + grow] = s;
     if (has_zy) p.zy[grow] = zyv;
   }
 };
 
 // KL forward (and the first pass of the alpha losses): per row and for both the draft
-// (q) and the target (p): online max and sum of exp; plus
+// (q, accumulator 0) and the target (p, accumulator 1): online max and sum of exp; plus
 // A = sum_v 2^(z_p log2e - m_p) (z_p - z_q), rescaled whenever m_p grows.
 struct EpiFwdDual {
   using Params = FwdParams;
@@ -597,7 +424,7 @@ struct EpiFwdDual {
   bool row_ok;
   int64_t grow;
 
-  __device__ __forceinline__ void unit_begin(const Params& p, int row0, int, int row) {
+  __device__ __forceinline__ void unit_begin(const Params& p, int row0, int row) {
     mq = mp = -INFINITY;
     sq = sp = A = 0.f;
     grow = static_cast<int64_t>(row0) + row;
@@ -633,14 +460,14 @@ struct EpiFwdDual {
     }
   }
 
-  template <int BN>
-  __device__ __forceinline__ void tile(const Params& p, uint32_t tb, int, int nt, int) {
-    const int64_t n0 = static_cast<int64_t>(nt) * BN;
+  template <int TN>
+  __device__ __forceinline__ void tile(const Params& p, uint32_t tb, int, int64_t n0, int c0,
+                                       int c1, int) {
 #pragma unroll 1
-    for (int c = 0; c < BN; c += 32) {
+    for (int c = c0; c < c1; c += 32) {
       float vq[32], vp[32];
       tmem_ld32(tb + c, vq);
-      tmem_ld32(tb + BN + c, vp);
+      tmem_ld32(tb + TN + c, vp);
       tmem_ld_wait();
       if (n0 + c + 32 > p.V) {
         mask_tail(vq, n0 + c, p.V);
@@ -652,9 +479,9 @@ struct EpiFwdDual {
     }
   }
 
-  __device__ __forceinline__ void unit_end(const Params& p, int, int j, int) {
+  __device__ __forceinline__ void unit_end(const Params& p, int, int slot, int) {
     if (!row_ok) return;
-    float* base = p.part + static_cast<int64_t>(j) * 5 * p.N + grow;
+    float* base = p.part + static_cast<int64_t>(slot) * 5 * p.N + grow;
     base[0 * p.N] = mq;
     base[1 * p.N] = sq;
     base[2 * p.N] = mp;
@@ -671,7 +498,7 @@ struct EpiAlpha {
   bool row_ok;
   int64_t grow;
 
-  __device__ __forceinline__ void unit_begin(const Params& p, int row0, int, int row) {
+  __device__ __forceinline__ void unit_begin(const Params& p, int row0, int row) {
     al = S = 0.f;
     grow = static_cast<int64_t>(row0) + row;
     row_ok = grow < p.N;
@@ -679,14 +506,14 @@ struct EpiAlpha {
     lp2 = row_ok ? p.stats[p.N + grow] * kLog2e : 0.f;
   }
 
-  template <int BN>
-  __device__ __forceinline__ void tile(const Params& p, uint32_t tb, int, int nt, int) {
-    const int64_t n0 = static_cast<int64_t>(nt) * BN;
+  template <int TN>
+  __device__ __forceinline__ void tile(const Params& p, uint32_t tb, int, int64_t n0, int c0,
+                                       int c1, int) {
 #pragma unroll 1
-    for (int c = 0; c < BN; c += 32) {
+    for (int c = c0; c < c1; c += 32) {
       float vq[32], vp[32];
       tmem_ld32(tb + c, vq);
-      tmem_ld32(tb + BN + c, vp);
+      tmem_ld32(tb + TN + c, vp);
       tmem_ld_wait();
       if (n0 + c + 32 > p.V) {
         mask_tail(vq, n0 + c, p.V);
@@ -702,10 +529,10 @@ struct EpiAlpha {
     }
   }
 
-  __device__ __forceinline__ void unit_end(const Params& p, int, int j, int) {
+  __device__ __forceinline__ void unit_end(const Params& p, int, int slot, int) {
     if (!row_ok) return;
-    p.part[(static_cast<int64_t>(j) * 2 + 0) * p.N + grow] = al;
-    p.part[(static_cast<int64_t>(j) * 2 + 1) * p.N + grow] = S;
+    p.part[(static_cast<int64_t>(slot) * 2 + 0) * p.N + grow] = al;
+    p.part[(static_cast<int64_t>(slot) * 2 + 1) * p.N + grow] = S;
   }
 };
 
@@ -755,7 +582,7 @@ struct EpiDz {
   bool row_ok;
   int64_t lrow;
 
-  __device__ __forceinline__ void unit_begin(const Params& p, int row0, int, int row) {
+  __device__ __forceinline__ void unit_begin(const Params& p, int row0, int row) {
     lrow = static_cast<int64_t>(row0) + row;
     row_ok = lrow < p.rows;
     const int64_t n = p.row0 + lrow;
@@ -790,17 +617,17 @@ struct EpiDz {
     }
   }
 
-  template <int BN>
-  __device__ __forceinline__ void tile(const Params& p, uint32_t tb, int, int nt, int) {
-    const int64_t n0 = static_cast<int64_t>(nt) * BN;
+  template <int TN>
+  __device__ __forceinline__ void tile(const Params& p, uint32_t tb, int, int64_t n0, int c0,
+                                       int c1, int) {
     __nv_bfloat16* out = p.dz + lrow * p.ldz + n0;
 #pragma unroll 1
-    for (int c = 0; c < BN; c += 32) {
+    for (int c = c0; c < c1; c += 32) {
       float vq[32];
       tmem_ld32(tb + c, vq);
       if (DUAL) {
         float vp[32];
-        tmem_ld32(tb + BN + c, vp);
+        tmem_ld32(tb + TN + c, vp);
         tmem_ld_wait();
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
@@ -818,7 +645,7 @@ struct EpiDz {
           vq[i] = g * (qv - (rel == i ? 1.f : 0.f));
         }
       }
-      if (row_ok) store_bf16_row32(out + c, vq, n0 + c, p.V);
+      if (row_ok && n0 + c < p.V) store_bf16_row32(out + c, vq, n0 + c, p.V);
     }
   }
 
@@ -828,16 +655,16 @@ struct EpiDz {
 // dH rows of the chunk: fp32 accumulator -> bf16.
 struct EpiDh {
   using Params = DhParams;
-  __device__ __forceinline__ void unit_begin(const Params&, int, int, int) {}
+  __device__ __forceinline__ void unit_begin(const Params&, int, int) {}
   __device__ __forceinline__ void unit_end(const Params&, int, int, int) {}
-  template <int BN>
-  __device__ __forceinline__ void tile(const Params& p, uint32_t tb, int row0, int nt, int row) {
+  template <int TN>
+  __device__ __forceinline__ void tile(const Params& p, uint32_t tb, int row0, int64_t n0,
+                                       int c0, int c1, int row) {
     const int64_t lrow = static_cast<int64_t>(row0) + row;
     const bool ok = lrow < p.rows;
-    const int64_t n0 = static_cast<int64_t>(nt) * BN;
     __nv_bfloat16* out = p.dH + (p.row0 + lrow) * p.d + n0;
 #pragma unroll 1
-    for (int c = 0; c < BN; c += 32) {
+    for (int c = c0; c < c1; c += 32) {
       float v[32];
       tmem_ld32(tb + c, v);
       tmem_ld_wait();
@@ -849,16 +676,16 @@ struct EpiDh {
 // dW tile: fp32 read-add-write (or plain write) of rows this CTA owns exclusively.
 struct EpiDw {
   using Params = DwParams;
-  __device__ __forceinline__ void unit_begin(const Params&, int, int, int) {}
+  __device__ __forceinline__ void unit_begin(const Params&, int, int) {}
   __device__ __forceinline__ void unit_end(const Params&, int, int, int) {}
-  template <int BN>
-  __device__ __forceinline__ void tile(const Params& p, uint32_t tb, int row0, int nt, int row) {
+  template <int TN>
+  __device__ __forceinline__ void tile(const Params& p, uint32_t tb, int row0, int64_t n0,
+                                       int c0, int c1, int row) {
     const int64_t v = static_cast<int64_t>(row0) + row;
     const bool ok = v < p.V;
-    const int64_t n0 = static_cast<int64_t>(nt) * BN;
     float* out = p.dW + v * p.d + n0;
 #pragma unroll 1
-    for (int c = 0; c < BN; c += 32) {
+    for (int c = c0; c < c1; c += 32) {
       float x[32];
       tmem_ld32(tb + c, x);
       tmem_ld_wait();
@@ -883,7 +710,8 @@ struct EpiDw {
 };
 
 // ----------------------------------------------------------------------------------------
-// Launchers.
+// Launchers: persistent 2-SM launches with clusters of two CTAs, at most as many clusters
+// as can be resident at once (so the static unit schedule never waits for a second wave).
 // ----------------------------------------------------------------------------------------
 int sm_count() {
   static int cached[64] = {0};
@@ -898,33 +726,15 @@ int sm_count() {
   return cached[dev];
 }
 
-template <int BN, int NUM_A, bool A_MN, bool B_MN, class Epi>
-static cudaError_t launch_gemm(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b,
-                               const GemmGeom& g, const typename Epi::Params& p, const DevCtl& c,
-                               int grid, cudaStream_t s) {
-  constexpr size_t kStageBytes = NUM_A * kBM * kBK * 2 + BN * kBK * 2;
-  constexpr size_t kSmem = 1024 + kStages * kStageBytes + sizeof(PipeCtl);
-  auto kern = gemm_kernel<BN, NUM_A, A_MN, B_MN, Epi>;
+template <int BNI, int NSUB, int NUM_A, int NBUF, int NWG, bool A_MN, bool B_MN, int STAGES,
+          class Epi>
+static cudaError_t launch_pair(const CUtensorMap& a0, const CUtensorMap& a1,
+                               const CUtensorMap& b, const GemmGeom& g,
+                               const typename Epi::Params& p, const DevCtl& c, cudaStream_t s) {
+  using Cfg = PairCfg<BNI, NSUB, NUM_A, NBUF, NWG, A_MN, B_MN, STAGES>;
+  auto kern = gemm_pair_kernel<BNI, NSUB, NUM_A, NBUF, NWG, A_MN, B_MN, STAGES, Epi>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(kSmem));
-  if (e != cudaSuccess) return e;
-  kern<<<grid, kThreads, kSmem, s>>>(a0, a1, b, g, p, c);
-  return cudaGetLastError();
-}
-
-// Persistent 2-SM launch: clusters of two CTAs, at most as many clusters as can be
-// resident at once (so the static unit schedule never waits for a second wave).
-template <int BN, int NUM_A, bool A_MN, bool B_MN, int STAGES, class Epi>
-static cudaError_t launch_gemm_pair(const CUtensorMap& a0, const CUtensorMap& a1,
-                                    const CUtensorMap& b, const GemmGeom& g,
-                                    const typename Epi::Params& p, const DevCtl& c,
-                                    cudaStream_t s) {
-  using Sh = PairShape<BN, NUM_A, A_MN, B_MN, STAGES>;
-  constexpr size_t kSmem = Sh::kSmem;
-  static_assert(kSmem <= 232448, "shared memory per CTA");
-  auto kern = gemm_pair_kernel<BN, NUM_A, A_MN, B_MN, STAGES, Epi>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(kSmem));
+                                       static_cast<int>(Cfg::kSmem));
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
@@ -932,8 +742,8 @@ static cudaError_t launch_gemm_pair(const CUtensorMap& a0, const CUtensorMap& a1
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = kSmem;
+  cfg.blockDim = dim3(Cfg::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = Cfg::kSmem;
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
@@ -949,48 +759,45 @@ static cudaError_t launch_gemm_pair(const CUtensorMap& a0, const CUtensorMap& a1
   }
   const int pairs = std::max(1, std::min(g.num_units, max_clusters[dev]));
   cfg.gridDim = dim3(2 * pairs, 1, 1);
-  e = cudaLaunchKernelEx(&cfg, kern, a0, a1, b, g, p, c);
-  if (e != cudaSuccess) return e;
-  return cudaGetLastError();
+  return cudaLaunchKernelEx(&cfg, kern, a0, a1, b, g, p, c);
 }
 
+// Forward statistics and logits gradient: A = hidden states (K-major), B = W (K-major).
+//   CE:   one accumulator, tile 256 x 512 (two 256-wide MMAs), single TMEM buffer
+//   dual: target + draft accumulators, tile 256 x 256 each, single TMEM buffer
+// dH: A = dZ (K-major), B = W (MN-major), tile 256 x 512, single buffer.
+// dW: A = dZ^T (MN-major), B = H (MN-major), tile 256 x 256, double-buffered (its fp32
+//     read-add-write epilogue overlaps the next tile's MMAs).
 cudaError_t launch_fwd_ce(const CUtensorMap& tH, const CUtensorMap& tW, const GemmGeom& g,
-                          const FwdParams& p, const DevCtl& c, int grid, cudaStream_t s) {
-  (void)grid;
-  return launch_gemm_pair<kBnSingle, 1, false, false, 6, EpiFwdCE>(tH, tH, tW, g, p, c, s);
+                          const FwdParams& p, const DevCtl& c, cudaStream_t s) {
+  return launch_pair<256, 2, 1, 1, 2, false, false, 4, EpiFwdCE>(tH, tH, tW, g, p, c, s);
 }
 cudaError_t launch_fwd_dual(const CUtensorMap& tHq, const CUtensorMap& tHp, const CUtensorMap& tW,
-                            const GemmGeom& g, const FwdParams& p, const DevCtl& c, int grid,
+                            const GemmGeom& g, const FwdParams& p, const DevCtl& c,
                             cudaStream_t s) {
-  (void)grid;
-  return launch_gemm_pair<kBnDual, 2, false, false, 5, EpiFwdDual>(tHq, tHp, tW, g, p, c, s);
+  return launch_pair<256, 1, 2, 1, 2, false, false, 4, EpiFwdDual>(tHq, tHp, tW, g, p, c, s);
 }
 cudaError_t launch_alpha(const CUtensorMap& tHq, const CUtensorMap& tHp, const CUtensorMap& tW,
-                         const GemmGeom& g, const FwdParams& p, const DevCtl& c, int grid,
+                         const GemmGeom& g, const FwdParams& p, const DevCtl& c,
                          cudaStream_t s) {
-  (void)grid;
-  return launch_gemm_pair<kBnDual, 2, false, false, 5, EpiAlpha>(tHq, tHp, tW, g, p, c, s);
+  return launch_pair<256, 1, 2, 1, 2, false, false, 4, EpiAlpha>(tHq, tHp, tW, g, p, c, s);
 }
 cudaError_t launch_dz_ce(const CUtensorMap& tH, const CUtensorMap& tW, const GemmGeom& g,
-                         const DzParams& p, const DevCtl& c, int grid, cudaStream_t s) {
-  (void)grid;
-  return launch_gemm_pair<kBnSingle, 1, false, false, 6, EpiDz<false>>(tH, tH, tW, g, p, c, s);
+                         const DzParams& p, const DevCtl& c, cudaStream_t s) {
+  return launch_pair<256, 2, 1, 1, 2, false, false, 4, EpiDz<false>>(tH, tH, tW, g, p, c, s);
 }
 cudaError_t launch_dz_dual(const CUtensorMap& tHq, const CUtensorMap& tHp, const CUtensorMap& tW,
-                           const GemmGeom& g, const DzParams& p, const DevCtl& c, int grid,
+                           const GemmGeom& g, const DzParams& p, const DevCtl& c,
                            cudaStream_t s) {
-  (void)grid;
-  return launch_gemm_pair<kBnDual, 2, false, false, 5, EpiDz<true>>(tHq, tHp, tW, g, p, c, s);
+  return launch_pair<256, 1, 2, 1, 2, false, false, 4, EpiDz<true>>(tHq, tHp, tW, g, p, c, s);
 }
 cudaError_t launch_dh(const CUtensorMap& tDz, const CUtensorMap& tW, const GemmGeom& g,
-                      const DhParams& p, const DevCtl& c, int grid, cudaStream_t s) {
-  (void)grid;
-  return launch_gemm_pair<kBnGrad, 1, false, true, 6, EpiDh>(tDz, tDz, tW, g, p, c, s);
+                      const DhParams& p, const DevCtl& c, cudaStream_t s) {
+  return launch_pair<256, 2, 1, 1, 2, false, true, 4, EpiDh>(tDz, tDz, tW, g, p, c, s);
 }
 cudaError_t launch_dw(const CUtensorMap& tDzT, const CUtensorMap& tH, const GemmGeom& g,
-                      const DwParams& p, const DevCtl& c, int grid, cudaStream_t s) {
-  (void)grid;
-  return launch_gemm_pair<kBnGrad, 1, true, true, 6, EpiDw>(tDzT, tDzT, tH, g, p, c, s);
+                      const DwParams& p, const DevCtl& c, cudaStream_t s) {
+  return launch_pair<256, 1, 1, 2, 1, true, true, 6, EpiDw>(tDzT, tDzT, tH, g, p, c, s);
 }
 
 // ----------------------------------------------------------------------------------------
