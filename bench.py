@@ -214,10 +214,9 @@ def run_ours(args):
     import torch
     import torch.distributed as dist
 
-    from lm_head_loss_streaming_b200 import synthetic
+    from lm_head_loss_streaming_b200 import _lib, dp, synthetic
     from lm_head_loss_streaming_b200.loss import (FwdResult, lm_head_loss_bwd,
                                                   lm_head_loss_fwd, workspace_bytes)
-    from lm_head_loss_streaming_b200 import _lib
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -247,20 +246,33 @@ def run_ours(args):
     dW = torch.empty(V, d, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
 
-    def step(ev=None):
-        if ev is not None:
-            ev[0].record(stream)
-        lm_head_loss_fwd(kind, Hq, W, lab, Hp, inp.ignore_index, workspace=ws,
-                         chunk_tokens=args.chunk_tokens, out=res)
-        if ev is not None:
-            ev[1].record(stream)
-        if world > 1:
-            dist.all_reduce(res.n_valid)
-        lm_head_loss_bwd(res, Hq, W, lab, Hp, inp.ignore_index, dH=dH, dW=dW,
-                         chunk_tokens=args.chunk_tokens)
-        if world > 1:
-            dist.all_reduce(dW)
-            dist.all_reduce(res.loss_sum)
+    def make_step(Hq_, W_, lab_, Hp_):
+        def _fwd(ev=None):
+            if ev is not None:
+                ev[0].record(stream)
+            r = lm_head_loss_fwd(kind, Hq_, W_, lab_, Hp_, inp.ignore_index, workspace=ws,
+                                 chunk_tokens=args.chunk_tokens, out=res)
+            if ev is not None:
+                ev[1].record(stream)
+            return r
+
+        def _bwd(r, n_valid_global):
+            r.n_valid.copy_(n_valid_global)
+            return lm_head_loss_bwd(r, Hq_, W_, lab_, Hp_, inp.ignore_index, dH=dH, dW=dW,
+                                    chunk_tokens=args.chunk_tokens)
+
+        def step(ev=None):
+            if world > 1:
+                # Data parallel over token rows: global valid count before the backward,
+                # dW and the loss sum summed after it (lm_head_loss_streaming_b200.dp).
+                dp.fwd_bwd(lambda: _fwd(ev), _bwd)
+            else:
+                r = _fwd(ev)
+                lm_head_loss_bwd(r, Hq_, W_, lab_, Hp_, inp.ignore_index, dH=dH, dW=dW,
+                                 chunk_tokens=args.chunk_tokens)
+        return step
+
+    step = make_step(Hq, W, lab, Hp)
 
     for _ in range(args.warmup):
         step()
@@ -310,6 +322,8 @@ def run_ours(args):
         h2d = hHq.numel() * 2 + hW.numel() * 2 + (hHp.numel() * 2 if hHp is not None else 0) \
             + (hlab.numel() * 4 if hlab is not None else 0)
 
+        dev_step = make_step(dHq, dWt, dlab, dHp)
+
         def e2e_step():
             dHq.copy_(hHq, non_blocking=True)
             dWt.copy_(hW, non_blocking=True)
@@ -317,15 +331,7 @@ def run_ours(args):
                 dHp.copy_(hHp, non_blocking=True)
             if dlab is not None:
                 dlab.copy_(hlab, non_blocking=True)
-            lm_head_loss_fwd(kind, dHq, dWt, dlab, dHp, inp.ignore_index, workspace=ws,
-                             chunk_tokens=args.chunk_tokens, out=res)
-            if world > 1:
-                dist.all_reduce(res.n_valid)
-            lm_head_loss_bwd(res, dHq, dWt, dlab, dHp, inp.ignore_index, dH=dH, dW=dW,
-                             chunk_tokens=args.chunk_tokens)
-            if world > 1:
-                dist.all_reduce(dW)
-                dist.all_reduce(res.loss_sum)
+            dev_step()
             hloss.copy_(res.loss_mean, non_blocking=True)
 
         e2e_step()

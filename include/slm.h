@@ -150,6 +150,15 @@ SLM_API int slm_loss_bwd(int kind, const void* Hq, const void* Hp, const void* W
  * word when it starts, so the status describes the most recent call. */
 SLM_API int slm_device_status(const void* workspace, void* stream);
 
+/* Test hook for the device-side failure path (not for production use).  fault_mode 1 makes
+ * every following launch withhold one internal pipeline release, so that a bounded wait in
+ * the kernel runs out: the kernel then records SLM_ERR_TIMEOUT in the workspace status word,
+ * lets its own copies and MMAs finish, frees its tensor memory and returns; results of that
+ * call are undefined.  fault_mode 0 restores normal operation.  timeout_cycles bounds every
+ * pipeline wait in SM clock cycles (0 = the default of 4e9, about 2 s).  Process-wide;
+ * takes effect at the next launch.  Returns SLM_ERR_SHAPE for an invalid mode or bound. */
+SLM_API int slm_debug_set(int fault_mode, long long timeout_cycles);
+
 /* Size of the device scratch array behind slm_loss_fwd_noalloc: 32 MiB per GPU that loads
  * the library's device code, held until the process exits. */
 #define SLM_NOALLOC_SCRATCH_BYTES (32u << 20)
@@ -162,7 +171,7 @@ SLM_API int slm_device_status(const void* workspace, void* stream);
  * Same arguments, outputs and results as slm_loss_fwd, without the workspace: the scratch
  * lives in a fixed __device__ array of SLM_NOALLOC_SCRATCH_BYTES.  Sizes whose forward
  * scratch exceeds it return SLM_ERR_WORKSPACE before anything is enqueued (at V = 128256
- * that is N > ~66,000 rows for SLM_CE and N > ~26,500 rows for the other kinds).
+ * that is N > ~65,000 rows for SLM_CE and N > ~26,000 rows for the other kinds).
  *   device_flags  int [1] device memory or NULL: receives the device status bits of this
  *                 call (0 = none; 1 = a CE label outside [0, V); 2 = a wait ran out of time).
  * The first call on each device looks up the array's device address (and may load the

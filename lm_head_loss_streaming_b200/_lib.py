@@ -40,6 +40,7 @@ SIGNATURES = {
     "slm_loss_bwd": (_INT, [_INT, _P, _P, _P, _P, _I32, _I64, _I64, _I64,
                             _P, _P, _P, _P, _P, _P, _INT, _I64, _P, _SZ, _P]),
     "slm_device_status": (_INT, [_P, _P]),
+    "slm_debug_set": (_INT, [_INT, ctypes.c_longlong]),
     "slm_loss_fwd_noalloc": (_INT, [_INT, _P, _P, _P, _P, _I32, _I64, _I64, _I64,
                                     _P, _P, _P, _P, _P, _P, _P, _P]),
 }
@@ -118,6 +119,12 @@ def slm_loss_bwd(kind, Hq, Hp, W, labels, ignore_index, N, d, V, grad_tok, grad_
 
 def slm_device_status(workspace, stream):
     return load().slm_device_status(workspace, stream)
+
+
+def slm_debug_set(fault_mode, timeout_cycles=0):
+    """Test hook: make the next launches run a bounded wait out (fault_mode=1), or restore
+    normal operation (0); timeout_cycles bounds every pipeline wait (0 = default)."""
+    return load().slm_debug_set(int(fault_mode), int(timeout_cycles))
 
 
 def slm_loss_fwd_noalloc(kind, Hq, Hp, W, labels, ignore_index, N, d, V, loss_tok, alpha_tok,

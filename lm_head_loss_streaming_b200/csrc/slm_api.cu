@@ -18,6 +18,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include "../../include/slm.h"
@@ -30,6 +31,14 @@ constexpr size_t kAlign = 256;
 constexpr int kPairM = 2 * kBM;   // M rows of one 2-SM tile
 constexpr int kGroupPairs = 8;    // pair M tiles per raster group (2048 token rows)
 constexpr long long kTimeoutCycles = 4000000000LL;  // ~2 s at the B200's boost clock
+
+// Test hooks set through slm_debug_set (process-wide, read at every launch).
+std::atomic<int> g_fault{0};
+std::atomic<long long> g_timeout{kTimeoutCycles};
+
+DevCtl make_ctl(int* status) {
+  return DevCtl{status, g_timeout.load(), g_fault.load()};
+}
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
@@ -246,7 +255,7 @@ int slm_loss_fwd(int kind, const void* Hq, const void* Hp, const void* W, const 
   float* part = reinterpret_cast<float*>(ws + L.part_off);
   float* zy = reinterpret_cast<float*>(ws + L.zy_off);
   SLM_TRY_CUDA(cudaMemsetAsync(status, 0, sizeof(int), s));
-  const DevCtl ctl{status, kTimeoutCycles};
+  const DevCtl ctl = make_ctl(status);
 
   if (N > 0) {
     const FwdSched f = fwd_sched(kind, V);
@@ -295,7 +304,7 @@ int slm_loss_bwd(int kind, const void* Hq, const void* Hp, const void* W, const 
   int* status = reinterpret_cast<int*>(ws + L.status_off);
   __nv_bfloat16* dz = reinterpret_cast<__nv_bfloat16*>(ws + L.dz_off);
   SLM_TRY_CUDA(cudaMemsetAsync(status, 0, sizeof(int), s));
-  const DevCtl ctl{status, kTimeoutCycles};
+  const DevCtl ctl = make_ctl(status);
 
   if (N == 0) {
     if (!accumulate_dW) SLM_TRY_CUDA(launch_zero_f32(dW, V * d, s));
@@ -337,6 +346,13 @@ int slm_loss_bwd(int kind, const void* Hq, const void* Hp, const void* W, const 
     DwParams pw{dW, V, d, (accumulate_dW || c0 > 0) ? 1 : 0};
     SLM_TRY_CUDA(launch_dw(tDz_mn, tH_mn, gw, pw, ctl, s));
   }
+  return SLM_OK;
+}
+
+int slm_debug_set(int fault_mode, long long timeout_cycles) {
+  if (fault_mode < 0 || fault_mode > 1 || timeout_cycles < 0) return SLM_ERR_SHAPE;
+  g_fault.store(fault_mode);
+  g_timeout.store(timeout_cycles > 0 ? timeout_cycles : kTimeoutCycles);
   return SLM_OK;
 }
 

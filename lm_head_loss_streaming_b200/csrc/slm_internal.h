@@ -44,6 +44,7 @@ struct GemmGeom {
 struct DevCtl {
   int* status;               // device status word (in the workspace)
   long long timeout_cycles;  // bound of every pipeline wait
+  int fault;                 // test hook: 1 = the epilogue withholds its first accumulator release
 };
 
 // Forward statistics (pass 1) and the alpha pass (pass 2).

@@ -317,7 +317,10 @@ __global__ void __launch_bounds__(64 + 128 * NWG, 1)
                                   static_cast<int64_t>(nt) * kTileN, c0, c1, row);
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(b ? tempty_leader1 : tempty_leader0);
+        // Test hook (fault == 1): withhold the release of the first accumulator, so that the
+        // MMA issuer's bounded wait for it runs out and the kernel unwinds with a timeout.
+        const bool withhold = ctl.fault == 1 && t == 0;
+        if (lane == 0 && !withhold) mbar_arrive_cluster(b ? tempty_leader1 : tempty_leader0);
       }
       if (!ok) break;
       epi.unit_end(ep, row0, j * NWG + wg, row);

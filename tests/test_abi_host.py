@@ -114,3 +114,9 @@ def test_bwd_output_pointer_errors(lib):
     assert _bwd(dW=None) == 1
     assert _bwd(dHq=None) == 1
     assert _bwd(dW=A + 4) == 3
+
+
+def test_debug_hook_arguments(lib):
+    assert _lib.slm_debug_set(2, 0) == 2     # SLM_ERR_SHAPE: unknown mode
+    assert _lib.slm_debug_set(0, -1) == 2    # SLM_ERR_SHAPE: negative bound
+    assert _lib.slm_debug_set(0, 0) == 0     # back to normal operation
