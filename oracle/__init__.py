@@ -9,6 +9,8 @@ from .slm_oracle import (  # noqa: F401
     KINDS,
     DISTRIBUTION_KINDS,
     ALPHA_KINDS,
+    TARGET_KINDS,
+    argmax_target,
     logits,
     log_softmax,
     token_terms,

@@ -24,13 +24,17 @@ Sources, cited by page title and section:
 [LF] "Loss Functions" (speculators user guide), table "Available Losses": p is the
      target distribution, q the draft distribution, alpha = sum_v min(p_v, q_v);
      kl_div = forward KL target->draft, rkl = reverse KL, jsd = Jensen-Shannon,
+     ce = cross entropy against argmax p (hard labels from the target),
      tv = 1 - alpha, nla = -log(alpha), lk_hybrid = lambda*KL + (1-lambda)*TV with
      lambda = exp(-3*alpha) detached.
 
 Readings taken where the pages are silent (each one is also listed in the design notes):
   * Row mask: a row whose label equals ``ignore_index`` is masked.  For "ce" the labels
     are required and every other label must lie in [0, V).  For the distribution losses
-    the labels are optional and only act as a row mask.
+    and "ce_argmax_p" the labels are optional and only act as a row mask.
+  * "ce_argmax_p" is the table's "ce" row (cross entropy against argmax p); it is named
+    apart from the hard-label "ce" of the streaming cross entropy page.  Ties of the
+    argmax go to the lowest vocabulary index.
   * Denominator: the number of unmasked rows.  With every row masked the loss is 0 and
     every gradient is 0 (the pages do not say; a mean over zero rows is undefined).
   * KL direction: "Forward KL, target to draft" is KL(p || q).
@@ -49,8 +53,10 @@ from __future__ import annotations
 
 import numpy as np
 
-KINDS = ("ce", "kl_div", "tv", "nla", "lk_hybrid", "rkl", "jsd")
+KINDS = ("ce", "kl_div", "tv", "nla", "lk_hybrid", "rkl", "jsd", "ce_argmax_p")
 DISTRIBUTION_KINDS = ("kl_div", "tv", "nla", "lk_hybrid", "rkl", "jsd")
+# Kinds that read the target logits z_p (every kind but hard-label "ce").
+TARGET_KINDS = DISTRIBUTION_KINDS + ("ce_argmax_p",)
 ALPHA_KINDS = ("tv", "nla", "lk_hybrid")
 
 GIB = float(1 << 30)
@@ -118,6 +124,12 @@ def token_terms(kind, zq, zp=None, labels=None):
         out["loss"] = -lq[np.arange(n), safe]
         return out
     zp = _f64(zp)
+    if kind == "ce_argmax_p":
+        # Cross entropy against the target's most likely token (lowest index on ties).
+        y = argmax_target(zp)
+        out["target"] = y
+        out["loss"] = -lq[np.arange(n), y]
+        return out
     out["lse_p"] = _logsumexp(zp)
     lp = zp - out["lse_p"][:, None]
     q = np.exp(lq)
@@ -149,6 +161,11 @@ def token_terms(kind, zq, zp=None, labels=None):
     return out
 
 
+def argmax_target(zp):
+    """Hard labels from the target: argmax_v z_p (first, i.e. lowest, index on ties)."""
+    return np.argmax(_f64(zp), axis=1)
+
+
 def dlogits(kind, zq, zp=None, labels=None):
     """d(per-token loss)/d z_q for one block of rows (upstream gradient 1 per row).
 
@@ -163,6 +180,10 @@ def dlogits(kind, zq, zp=None, labels=None):
         y = np.asarray(labels, dtype=np.int64)
         dz = q.copy()
         dz[np.arange(n), np.clip(y, 0, V - 1)] -= 1.0
+        return dz
+    if kind == "ce_argmax_p":
+        dz = q.copy()
+        dz[np.arange(n), argmax_target(zp)] -= 1.0
         return dz
     lp = log_softmax(zp)
     p = np.exp(lp)
@@ -220,7 +241,7 @@ def forward(kind, Hq, W, labels=None, Hp=None, ignore_index=-100, chunk_size=512
     Hp_ = _f64(Hp) if (kind != "ce") else None
     lab = _labels(labels, n)
     valid = _row_mask(kind, lab, n, V, ignore_index)
-    keys = ("lse_q", "lse_p", "kl", "alpha", "S")
+    keys = ("lse_q", "lse_p", "kl", "alpha", "S", "target")
     res = {k: np.zeros(n) for k in keys}
     res["loss_tok"] = np.zeros(n)
     total_loss = 0.0
@@ -238,6 +259,7 @@ def forward(kind, Hq, W, labels=None, Hp=None, ignore_index=-100, chunk_size=512
                 res[k][c0:c1] = terms[k]
         total_loss += tok.sum()          # chunk_loss_sum
         total_weight += int(v.sum())     # chunk_weight
+    res["target"] = res["target"].astype(np.int64)
     res["loss_sum"] = total_loss
     res["n_valid"] = total_weight
     res["loss"] = total_loss / total_weight if total_weight > 0 else 0.0

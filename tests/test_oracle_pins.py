@@ -374,3 +374,34 @@ def test_large_logits_are_finite_and_match_torch():
     assert np.allclose(out["loss_tok"], ref, rtol=1e-12)
     kl = orc.forward("kl_div", Hq, W, Hp=Hp)["loss_tok"]
     assert np.isfinite(kl).all()
+
+
+# --------------------------------------------------------------------------------------
+# "ce" row of the loss table: cross entropy against argmax p (hard labels from the target).
+# --------------------------------------------------------------------------------------
+def test_ce_argmax_p_matches_torch():
+    Hq, Hp, W, y = _rand(11, 9, 21, seed=40, w_std=0.8)
+    lab = y.copy()
+    lab[[2, 7]] = -100                      # optional row mask
+    H_t = torch.tensor(Hq, requires_grad=True)
+    W_t = torch.tensor(W, requires_grad=True)
+    zp = torch.tensor(Hp) @ W_t.T.detach()
+    target = torch.argmax(zp, dim=1)        # first maximal index on ties
+    target[[2, 7]] = -100
+    ref = F.cross_entropy(H_t @ W_t.T, target, ignore_index=-100, reduction="mean")
+    ref.backward()
+    L, dH, dW, f = orc.loss_and_grads("ce_argmax_p", Hq, W, lab, Hp)
+    assert abs(L - ref.item()) < 1e-13
+    assert np.allclose(dH, H_t.grad.numpy(), atol=1e-14)
+    assert np.allclose(dW, W_t.grad.numpy(), atol=1e-14)
+    assert f["n_valid"] == 9
+
+
+def test_ce_argmax_p_ties_go_to_lowest_index():
+    # Target logits with an exact three-way tie at columns 1, 3 and 4.
+    zp = np.array([[0.0, 2.0, 1.0, 2.0, 2.0]])
+    zq = np.array([[0.3, -0.1, 0.2, 0.5, 0.0]])
+    t = orc.token_terms("ce_argmax_p", zq, zp)
+    assert int(t["target"][0]) == 1
+    lse = math.log(sum(math.exp(v) for v in zq[0]))
+    assert abs(t["loss"][0] - (lse - zq[0, 1])) < 1e-14
