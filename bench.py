@@ -58,9 +58,10 @@ def parse_args():
 # ---------------------------------------------------------------------------------------
 def gemm_passes(kind):
     """Number of N x V x d logit-sized GEMMs per token in fwd + bwd (each 2NVd flops):
-    CE: fwd 1 + recompute 1 + dH 1 + dW 1 = 4;  KL: 2 + 2 + 1 + 1 = 6;
-    alpha losses: 2 + 2 (second pass) + 2 + 1 + 1 = 8."""
-    return {"ce": 4, "kl_div": 6}.get(kind, 8)
+    CE: fwd 1 + recompute 1 + dH 1 + dW 1 = 4;  KL, RKL: 2 + 2 + 1 + 1 = 6;
+    CE against argmax p: 2 + 1 + 1 + 1 = 5;
+    alpha losses and JSD: 2 + 2 (second pass) + 2 + 1 + 1 = 8."""
+    return {"ce": 4, "kl_div": 6, "rkl": 6, "ce_argmax_p": 5}.get(kind, 8)
 
 
 def fwd_gemm_passes(kind):
@@ -71,7 +72,8 @@ def launches_per_step(kind, N, d, chunk_tokens):
     """Kernels of libslm.so launched by one forward + backward (memsets excluded)."""
     if N == 0:
         return 1 + 1
-    fwd = 3 if kind in ("ce", "kl_div") else 5  # GEMM, combine, [alpha GEMM, combine], finalize
+    # GEMM, combine, [second GEMM pass, combine], finalize
+    fwd = 5 if kind in ("tv", "nla", "lk_hybrid", "jsd") else 3
     C = chunk_tokens if chunk_tokens > 0 else ((2 * d + 127) // 128) * 128
     C = max(1, min(C, N))
     chunks = (N + C - 1) // C

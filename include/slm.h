@@ -16,6 +16,11 @@
  *   SLM_NLA        negative log-acceptance  -log(alpha)   (alpha clamped at 1e-30)
  *   SLM_LK_HYBRID  lambda * KL + (1 - lambda) * TV,  lambda = exp(-3 alpha) per token,
  *                  detached (no gradient through lambda)
+ *   SLM_RKL        reverse KL, draft to target  KL(q || p)
+ *   SLM_JSD        Jensen-Shannon divergence  (KL(p || M) + KL(q || M)) / 2, M = (p + q) / 2,
+ *                  bounded by log 2
+ *   SLM_CE_ARGMAX_P  cross entropy against argmax p: hard labels from the target (the
+ *                  lowest vocabulary index wins a tie)
  * The target p is detached: gradients flow to H_q and to W through z_q only.
  *
  * Masking and normalisation ("Streaming Cross Entropy"; "Correctness: alignment before
@@ -61,7 +66,10 @@ typedef enum slm_loss_kind {
   SLM_KL = 1,
   SLM_TV = 2,
   SLM_NLA = 3,
-  SLM_LK_HYBRID = 4
+  SLM_LK_HYBRID = 4,
+  SLM_RKL = 5,
+  SLM_JSD = 6,
+  SLM_CE_ARGMAX_P = 7
 } slm_loss_kind;
 
 typedef enum slm_status {
@@ -86,8 +94,10 @@ SLM_API const char* slm_status_string(int status);
 /* Number of floats per token row of the `stats` array that slm_loss_fwd writes and
  * slm_loss_bwd reads (layout [k][N], field-major):
  *   SLM_CE: 1  (L_q = logsumexp z_q)
- *   SLM_KL: 3  (L_q, L_p, KL)
+ *   SLM_CE_ARGMAX_P: 2  (L_q, the argmax-p target as int32 bits; ignore_index if masked)
+ *   SLM_KL: 3  (L_q, L_p, KL);  SLM_RKL: 3  (L_q, L_p, RKL)
  *   SLM_TV, SLM_NLA, SLM_LK_HYBRID: 5  (L_q, L_p, KL, alpha, S = sum_{q_v < p_v} q_v)
+ *   SLM_JSD: 5  (L_q, L_p, KL, JSD, T = sum_v q_v (log q_v - log M_v) / 2)
  * Returns 0 for an unknown kind. */
 SLM_API size_t slm_stats_floats(int kind);
 
@@ -107,6 +117,7 @@ SLM_API size_t slm_workspace_bytes(int kind, int64_t N, int64_t d, int64_t V, in
  *                        to ignore_index masks the row, any other value outside [0, V)
  *                        sets SLM_ERR_LABEL_RANGE and masks the row.
  *                        Other kinds: optional row mask (NULL = every row valid).
+ *                        (SLM_CE_ARGMAX_P takes its targets from H_p; labels only mask.)
  *   loss_tok   float [N]  per-token loss (0 on masked rows); may be NULL.
  *   alpha_tok  float [N]  per-token alpha for TV / NLA / LK_HYBRID; may be NULL.
  *   loss_sum   double [1] masked loss sum; required.
@@ -115,8 +126,9 @@ SLM_API size_t slm_workspace_bytes(int kind, int64_t N, int64_t d, int64_t V, in
  *   stats      float [slm_stats_floats(kind) * N] per-token statistics kept for the
  *                        backward (layout above); required when N > 0.
  *   workspace  device scratch of at least slm_workspace_bytes(kind, N, d, V, *) bytes.
- * SLM_CE / SLM_KL make one pass of the LM-head GEMM over the vocabulary; the alpha-based
- * kinds make two (alpha needs the final log-sum-exps). */
+ * SLM_CE, SLM_KL, SLM_RKL and SLM_CE_ARGMAX_P make one pass of the LM-head GEMM over the
+ * vocabulary; the alpha-based kinds and SLM_JSD make two (they need the final
+ * log-sum-exps). */
 SLM_API int slm_loss_fwd(int kind, const void* Hq, const void* Hp, const void* W,
                  const int32_t* labels, int32_t ignore_index,
                  int64_t N, int64_t d, int64_t V,

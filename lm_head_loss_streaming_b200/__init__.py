@@ -8,7 +8,7 @@ only marshals arguments and allocates device memory through PyTorch.
 
 from .synthetic import IGNORE_INDEX  # noqa: F401
 
-KINDS = ("ce", "kl_div", "tv", "nla", "lk_hybrid")
+KINDS = ("ce", "kl_div", "tv", "nla", "lk_hybrid", "rkl", "jsd", "ce_argmax_p")
 
 
 def __getattr__(name):

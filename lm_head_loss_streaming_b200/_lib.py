@@ -14,8 +14,11 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libslm.so")
 
 SLM_CE, SLM_KL, SLM_TV, SLM_NLA, SLM_LK_HYBRID = 0, 1, 2, 3, 4
+SLM_RKL, SLM_JSD, SLM_CE_ARGMAX_P = 5, 6, 7
 KIND = {"ce": SLM_CE, "kl_div": SLM_KL, "tv": SLM_TV, "nla": SLM_NLA,
-        "lk_hybrid": SLM_LK_HYBRID}
+        "lk_hybrid": SLM_LK_HYBRID, "rkl": SLM_RKL, "jsd": SLM_JSD,
+        "ce_argmax_p": SLM_CE_ARGMAX_P}
+ALPHA_KINDS = (SLM_TV, SLM_NLA, SLM_LK_HYBRID)
 
 SLM_OK = 0
 STATUS_NAMES = {

@@ -43,9 +43,13 @@ DevCtl make_ctl(int* status) {
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
-bool valid_kind(int k) { return k >= SLM_CE && k <= SLM_LK_HYBRID; }
+bool valid_kind(int k) { return k >= SLM_CE && k <= SLM_CE_ARGMAX_P; }
+// Kinds whose forward reads the target logits z_p (all but hard-label CE).
 bool dual_kind(int k) { return k != SLM_CE; }
-bool alpha_kind(int k) { return k == SLM_TV || k == SLM_NLA || k == SLM_LK_HYBRID; }
+// Kinds whose loss needs the final log-sum-exps: a second pass over the vocabulary.
+bool two_pass_kind(int k) {
+  return k == SLM_TV || k == SLM_NLA || k == SLM_LK_HYBRID || k == SLM_JSD;
+}
 
 // Forward vocabulary schedule: tiles of `bn` columns, grouped into at most 32 runs per row
 // (so the per-row partials stay O(N)), each run at least 2048 columns long.  Each run
@@ -63,7 +67,7 @@ FwdSched fwd_sched(int kind, int64_t V) {
   f.vc = std::min(f.vc, f.num_n);
   f.units_n = static_cast<int>(ceil_div(f.num_n, f.vc));
   f.slots = f.units_n * kFwdPartsPerRun;
-  f.fields = dual_kind(kind) ? 5 : 2;
+  f.fields = kind == SLM_CE ? kCEFields : (kind == SLM_CE_ARGMAX_P ? kArgmaxFields : kDualFields);
   return f;
 }
 
@@ -229,7 +233,8 @@ const char* slm_status_string(int s) {
 size_t slm_stats_floats(int kind) {
   if (!valid_kind(kind)) return 0;
   if (kind == SLM_CE) return 1;
-  if (kind == SLM_KL) return 3;
+  if (kind == SLM_CE_ARGMAX_P) return 2;
+  if (kind == SLM_KL || kind == SLM_RKL) return 3;
   return 5;
 }
 
@@ -268,12 +273,18 @@ int slm_loss_fwd(int kind, const void* Hq, const void* Hp, const void* W, const 
       SLM_TRY_CUDA(launch_fwd_ce(tHq, tW, g, p, ctl, s));
     } else {
       if (!make_map(&tHp, Hp, d, N, d, kBK, kBM)) return SLM_ERR_CUDA;
-      SLM_TRY_CUDA(launch_fwd_dual(tHq, tHp, tW, g, p, ctl, s));
+      if (kind == SLM_CE_ARGMAX_P)
+        SLM_TRY_CUDA(launch_fwd_argmax(tHq, tHp, tW, g, p, ctl, s));
+      else
+        SLM_TRY_CUDA(launch_fwd_dual(tHq, tHp, tW, g, p, ctl, s));
     }
     SLM_TRY_CUDA(launch_combine(kind, 1, part, f.slots, zy, labels, ignore_index, N, V,
                                 loss_tok, alpha_tok, stats, blk_sum, blk_cnt, status, s));
-    if (alpha_kind(kind)) {
-      SLM_TRY_CUDA(launch_alpha(tHq, tHp, tW, g, p, ctl, s));
+    if (two_pass_kind(kind)) {
+      if (kind == SLM_JSD)
+        SLM_TRY_CUDA(launch_jsd(tHq, tHp, tW, g, p, ctl, s));
+      else
+        SLM_TRY_CUDA(launch_alpha(tHq, tHp, tW, g, p, ctl, s));
       SLM_TRY_CUDA(launch_combine(kind, 2, part, f.slots, zy, labels, ignore_index, N, V,
                                   loss_tok, alpha_tok, stats, blk_sum, blk_cnt, status, s));
     }
@@ -311,7 +322,14 @@ int slm_loss_bwd(int kind, const void* Hq, const void* Hp, const void* W, const 
     return SLM_OK;
   }
   const int64_t C = default_chunk(N, d, chunk_tokens);
-  const FwdSched f = fwd_sched(kind, V);
+  // CE against argmax p needs only the draft logits in the backward: it runs the CE
+  // logits-gradient kernel with the forward's argmax targets (ignore_index on masked rows)
+  // as labels.
+  const bool argmax_kind = kind == SLM_CE_ARGMAX_P;
+  const int dz_kind = argmax_kind ? SLM_CE : kind;
+  const int32_t* dz_labels =
+      argmax_kind ? reinterpret_cast<const int32_t*>(stats + N) : labels;
+  const FwdSched f = fwd_sched(dz_kind, V);
   CUtensorMap tW_k, tW_mn;
   if (!make_map(&tW_k, W, d, V, d, kBK, 128)) return SLM_ERR_CUDA;
   if (!make_map(&tW_mn, W, d, V, d, 64, 64)) return SLM_ERR_CUDA;
@@ -324,9 +342,9 @@ int slm_loss_bwd(int kind, const void* Hq, const void* Hp, const void* W, const 
     CUtensorMap tHq, tHp;
     if (!make_map(&tHq, hq, d, rows, d, kBK, kBM)) return SLM_ERR_CUDA;
     const GemmGeom gz = geom(rows, V, d, f.bn, f.vc, kGroupPairs, kPairM);
-    DzParams pz{kind, labels, ignore_index, c0, rows, N, V, stats, grad_tok, grad_scale,
+    DzParams pz{dz_kind, dz_labels, ignore_index, c0, rows, N, V, stats, grad_tok, grad_scale,
                 n_valid, dz, ldz};
-    if (!dual_kind(kind)) {
+    if (!dual_kind(dz_kind)) {
       SLM_TRY_CUDA(launch_dz_ce(tHq, tW_k, gz, pz, ctl, s));
     } else {
       const __nv_bfloat16* hp = static_cast<const __nv_bfloat16*>(Hp) + c0 * d;

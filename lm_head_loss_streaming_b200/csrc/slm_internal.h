@@ -26,7 +26,13 @@ constexpr int kFwdPartsPerRun = 2;
 constexpr int kFlagLabelRange = 1;
 constexpr int kFlagTimeout = 2;
 
-enum LossKind : int { kCE = 0, kKL = 1, kTV = 2, kNLA = 3, kLK = 4 };
+enum LossKind : int { kCE = 0, kKL = 1, kTV = 2, kNLA = 3, kLK = 4, kRKL = 5, kJSD = 6,
+                      kCEArgmax = 7 };
+
+// Fields of the forward's per-row partial statistics (per vocabulary-run slot).
+constexpr int kDualFields = 6;    // m_q, s_q, m_p, s_p, A (p-weighted z_p - z_q), B (q-weighted z_q - z_p)
+constexpr int kArgmaxFields = 5;  // m_q, s_q, max z_p, its column, z_q at that column
+constexpr int kCEFields = 2;      // m, s
 
 // Persistent tile schedule.  Work units are (M tile, run of `vc` consecutive N tiles);
 // units are ordered in groups of `group_m` M tiles: for each N run, every M tile of the
@@ -90,6 +96,11 @@ cudaError_t launch_fwd_ce(const CUtensorMap& tH, const CUtensorMap& tW, const Ge
 cudaError_t launch_fwd_dual(const CUtensorMap& tHq, const CUtensorMap& tHp,
                             const CUtensorMap& tW, const GemmGeom& g, const FwdParams& p,
                             const DevCtl& c, cudaStream_t s);
+cudaError_t launch_fwd_argmax(const CUtensorMap& tHq, const CUtensorMap& tHp,
+                              const CUtensorMap& tW, const GemmGeom& g, const FwdParams& p,
+                              const DevCtl& c, cudaStream_t s);
+cudaError_t launch_jsd(const CUtensorMap& tHq, const CUtensorMap& tHp, const CUtensorMap& tW,
+                       const GemmGeom& g, const FwdParams& p, const DevCtl& c, cudaStream_t s);
 cudaError_t launch_alpha(const CUtensorMap& tHq, const CUtensorMap& tHp, const CUtensorMap& tW,
                          const GemmGeom& g, const FwdParams& p, const DevCtl& c,
                          cudaStream_t s);

@@ -18,9 +18,12 @@
 // removing the logits and attention bottlenecks", "Streaming Cross Entropy" and
 // "Backward pass"): logits tiles live only in TMEM and registers.
 //   EpiFwdCE    online row max / sum of exp and the label logit          (CE forward)
-//   EpiFwdDual  the same for target and draft plus the KL accumulator    (KL forward,
-//               first pass of the alpha losses)
+//   EpiFwdDual  the same for target and draft plus the forward- and reverse-KL
+//               accumulators                                             (KL / RKL forward,
+//               first pass of the alpha losses and of JSD)
+//   EpiFwdArgmax draft log-sum-exp plus the target's running argmax      (CE against argmax p)
 //   EpiAlpha    alpha = sum min(p, q) and S = sum_{q<p} q                 (second pass)
+//   EpiJsd      the two halves of the Jensen-Shannon divergence         (second pass)
 //   EpiDz       the logits gradient, rounded to bf16 into the chunk buffer (backward)
 //   EpiDh       dH chunk rows (bf16)                                      (dH = dZ W)
 //   EpiDw       fp32 read-add-write of disjoint dW tiles, no atomics      (dW += dZ^T H)
@@ -418,18 +421,19 @@ struct EpiFwdCE {
   }
 };
 
-// KL forward (and the first pass of the alpha losses): per row and for both the draft
-// (q, accumulator 0) and the target (p, accumulator 1): online max and sum of exp; plus
-// A = sum_v 2^(z_p log2e - m_p) (z_p - z_q), rescaled whenever m_p grows.
+// KL / RKL forward (and the first pass of the alpha losses and of JSD): per row and for
+// both the draft (q, accumulator 0) and the target (p, accumulator 1): online max and sum
+// of exp; plus A = sum_v 2^(z_p log2e - m_p) (z_p - z_q), rescaled whenever m_p grows, and
+// B = sum_v 2^(z_q log2e - m_q) (z_q - z_p), rescaled whenever m_q grows.
 struct EpiFwdDual {
   using Params = FwdParams;
-  float mq, sq, mp, sp, A;
+  float mq, sq, mp, sp, A, B;
   bool row_ok;
   int64_t grow;
 
   __device__ __forceinline__ void unit_begin(const Params& p, int row0, int row) {
     mq = mp = -INFINITY;
-    sq = sp = A = 0.f;
+    sq = sp = A = B = 0.f;
     grow = static_cast<int64_t>(row0) + row;
     row_ok = grow < p.N;
   }
@@ -439,7 +443,9 @@ struct EpiFwdDual {
     const float xq = max32(vq) * kLog2e;
     const float xp = max32(vp) * kLog2e;
     if (xq > mq) {
-      sq *= exp2f(mq - xq);
+      const float r = exp2f(mq - xq);
+      sq *= r;
+      B *= r;
       mq = xq;
     }
     if (xp > mp) {
@@ -456,9 +462,13 @@ struct EpiFwdDual {
       sq += eq;
       sp += e;
       if (TAIL) {
+        // Masked columns are -inf in both: their weights are 0 and their difference NaN.
         if (e > 0.f) A = fmaf(e, vp[i] - vq[i], A);
+        if (eq > 0.f) B = fmaf(eq, vq[i] - vp[i], B);
       } else {
-        A = fmaf(e, vp[i] - vq[i], A);
+        const float dpq = vp[i] - vq[i];
+        A = fmaf(e, dpq, A);
+        B = fmaf(-eq, dpq, B);
       }
     }
   }
@@ -484,12 +494,81 @@ struct EpiFwdDual {
 
   __device__ __forceinline__ void unit_end(const Params& p, int, int slot, int) {
     if (!row_ok) return;
-    float* base = p.part + static_cast<int64_t>(slot) * 5 * p.N + grow;
+    float* base = p.part + static_cast<int64_t>(slot) * kDualFields * p.N + grow;
     base[0 * p.N] = mq;
     base[1 * p.N] = sq;
     base[2 * p.N] = mp;
     base[3 * p.N] = sp;
     base[4 * p.N] = A;
+    base[5 * p.N] = B;
+  }
+};
+
+// CE against argmax p (forward): online max / sum of exp of the draft logits, and the
+// target's running argmax over the slot's columns (the first, i.e. lowest, column wins
+// ties: columns are visited in increasing order and only a strictly larger value
+// replaces), with the draft logit at that column.
+struct EpiFwdArgmax {
+  using Params = FwdParams;
+  float mq, sq, pmax, zqa;
+  int pidx;
+  bool row_ok;
+  int64_t grow;
+
+  __device__ __forceinline__ void unit_begin(const Params& p, int row0, int row) {
+    mq = pmax = -INFINITY;
+    sq = zqa = 0.f;
+    pidx = -1;
+    grow = static_cast<int64_t>(row0) + row;
+    row_ok = grow < p.N;
+  }
+
+  template <int TN>
+  __device__ __forceinline__ void tile(const Params& p, uint32_t tb, int, int64_t n0, int c0,
+                                       int c1, int) {
+#pragma unroll 1
+    for (int c = c0; c < c1; c += 32) {
+      float vq[32], vp[32];
+      tmem_ld32(tb + c, vq);
+      tmem_ld32(tb + TN + c, vp);
+      tmem_ld_wait();
+      if (n0 + c + 32 > p.V) {
+        mask_tail(vq, n0 + c, p.V);
+        mask_tail(vp, n0 + c, p.V);
+      }
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        if (vp[i] > pmax) {
+          pmax = vp[i];
+          pidx = static_cast<int>(n0 + c + i);
+          zqa = vq[i];
+        }
+      }
+      const float mx = max32(vq) * kLog2e;
+      if (mx > mq) {
+        sq *= exp2f(mq - mx);
+        mq = mx;
+      }
+      if (mq != -INFINITY) {
+        float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          a0 += exp2f(fmaf(vq[i], kLog2e, -mq));
+          a1 += exp2f(fmaf(vq[i + 1], kLog2e, -mq));
+        }
+        sq += a0 + a1;
+      }
+    }
+  }
+
+  __device__ __forceinline__ void unit_end(const Params& p, int, int slot, int) {
+    if (!row_ok) return;
+    float* base = p.part + static_cast<int64_t>(slot) * kArgmaxFields * p.N + grow;
+    base[0 * p.N] = mq;
+    base[1 * p.N] = sq;
+    base[2 * p.N] = pmax;
+    base[3 * p.N] = __int_as_float(pidx);
+    base[4 * p.N] = zqa;
   }
 };
 
@@ -539,6 +618,60 @@ struct EpiAlpha {
   }
 };
 
+// Second pass of JSD: with L_q and L_p known, per column p, q and M = (p + q) / 2;
+// jp += p (log p - log M) and jq += q (log q - log M), where log p = z_p - L_p exactly.
+// JSD = (jp + jq) / 2; the backward also needs T = sum_v q_v a_v = jq / 2 with
+// a_v = (log q_v - log M_v) / 2.
+struct EpiJsd {
+  using Params = FwdParams;
+  float lq, lp, lq2, lp2, jp, jq;
+  bool row_ok;
+  int64_t grow;
+
+  __device__ __forceinline__ void unit_begin(const Params& p, int row0, int row) {
+    jp = jq = 0.f;
+    grow = static_cast<int64_t>(row0) + row;
+    row_ok = grow < p.N;
+    lq = row_ok ? p.stats[grow] : 0.f;
+    lp = row_ok ? p.stats[p.N + grow] : 0.f;
+    lq2 = lq * kLog2e;
+    lp2 = lp * kLog2e;
+  }
+
+  template <int TN>
+  __device__ __forceinline__ void tile(const Params& p, uint32_t tb, int, int64_t n0, int c0,
+                                       int c1, int) {
+#pragma unroll 1
+    for (int c = c0; c < c1; c += 32) {
+      float vq[32], vp[32];
+      tmem_ld32(tb + c, vq);
+      tmem_ld32(tb + TN + c, vp);
+      tmem_ld_wait();
+      if (n0 + c + 32 > p.V) {
+        mask_tail(vq, n0 + c, p.V);
+        mask_tail(vp, n0 + c, p.V);
+      }
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float qv = exp2f(fmaf(vq[i], kLog2e, -lq2));
+        const float pv = exp2f(fmaf(vp[i], kLog2e, -lp2));
+        const float ms = pv + qv;
+        if (ms > 0.f) {  // both 0 (masked or underflowed) contributes nothing
+          const float lm = log2f(0.5f * ms) * kLn2;
+          jp = fmaf(pv, (vp[i] - lp) - lm, jp);
+          jq = fmaf(qv, (vq[i] - lq) - lm, jq);
+        }
+      }
+    }
+  }
+
+  __device__ __forceinline__ void unit_end(const Params& p, int, int slot, int) {
+    if (!row_ok) return;
+    p.part[(static_cast<int64_t>(slot) * 2 + 0) * p.N + grow] = jp;
+    p.part[(static_cast<int64_t>(slot) * 2 + 1) * p.N + grow] = jq;
+  }
+};
+
 // Upstream gradient of one row: valid * grad_tok * grad_scale / max(n_valid, 1).
 __device__ __forceinline__ float row_grad(const DzParams& p, int64_t n, bool valid) {
   if (!valid) return 0.f;
@@ -573,15 +706,20 @@ __device__ __forceinline__ void store_bf16_row32(__nv_bfloat16* dst, const float
 }
 
 // Backward logits-gradient tile: recomputed logits -> dZ (bf16) of the token chunk.
-//   CE:      dz_j = g (q_j - [j = y])
-//   others:  dz_j = ck (q_j - p_j) + cm q_j (m_j - S),  m_j = [q_j < p_j]
+//   CE (and CE against argmax p, whose targets come from the forward):
+//            dz_j = g (q_j - [j = y])
+//   KL, TV, NLA, LK (mode 0):  dz_j = ck (q_j - p_j) + cm q_j (m_j - S),  m_j = [q_j < p_j]
 //            KL: ck = g, cm = 0;  TV: ck = 0, cm = -g;  NLA: ck = 0, cm = -g / alpha;
 //            LK: ck = g lambda, cm = -g (1 - lambda), lambda = exp(-3 alpha) (detached).
+//   RKL (mode 1):  dz_j = g q_j (log q_j - log p_j - RKL) = g q_j (z_q - z_p - c),
+//            c = L_q - L_p + RKL.
+//   JSD (mode 2):  dz_j = g q_j (a_j - T),  a_j = (log q_j - log M_j) / 2.
 template <bool DUAL>
 struct EpiDz {
   using Params = DzParams;
-  float lq2, lp2, g, ck, cm, S;
+  float lq, lp, lq2, lp2, g, ck, cm, S;
   int32_t lab;
+  int mode;
   bool row_ok;
   int64_t lrow;
 
@@ -589,8 +727,9 @@ struct EpiDz {
     lrow = static_cast<int64_t>(row0) + row;
     row_ok = lrow < p.rows;
     const int64_t n = p.row0 + lrow;
-    lq2 = lp2 = g = ck = cm = S = 0.f;
+    lq = lp = lq2 = lp2 = g = ck = cm = S = 0.f;
     lab = -1;
+    mode = 0;
     if (!row_ok) return;
     bool valid = true;
     if (p.labels) {
@@ -599,11 +738,21 @@ struct EpiDz {
       if (!DUAL && (lab < 0 || lab >= p.V)) valid = false;
     }
     g = row_grad(p, n, valid);
-    lq2 = p.stats[n] * kLog2e;
+    lq = p.stats[n];
+    lq2 = lq * kLog2e;
     if (DUAL) {
-      lp2 = p.stats[p.N + n] * kLog2e;
+      lp = p.stats[p.N + n];
+      lp2 = lp * kLog2e;
       if (p.kind == kKL) {
         ck = g;
+      } else if (p.kind == kRKL) {
+        mode = 1;
+        ck = g;
+        cm = lq - lp + p.stats[2 * p.N + n];  // c
+      } else if (p.kind == kJSD) {
+        mode = 2;
+        ck = g;
+        S = p.stats[4 * p.N + n];  // T
       } else {
         const float al = p.stats[3 * p.N + n];
         S = p.stats[4 * p.N + n];
@@ -632,12 +781,32 @@ struct EpiDz {
         float vp[32];
         tmem_ld32(tb + TN + c, vp);
         tmem_ld_wait();
+        if (mode == 0) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float qv = exp2f(fmaf(vq[i], kLog2e, -lq2));
-          const float pv = exp2f(fmaf(vp[i], kLog2e, -lp2));
-          const float mS = ((qv < pv) ? 1.f : 0.f) - S;
-          vq[i] = fmaf(ck, qv - pv, cm * qv * mS);
+          for (int i = 0; i < 32; ++i) {
+            const float qv = exp2f(fmaf(vq[i], kLog2e, -lq2));
+            const float pv = exp2f(fmaf(vp[i], kLog2e, -lp2));
+            const float mS = ((qv < pv) ? 1.f : 0.f) - S;
+            vq[i] = fmaf(ck, qv - pv, cm * qv * mS);
+          }
+        } else if (mode == 1) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float qv = exp2f(fmaf(vq[i], kLog2e, -lq2));
+            vq[i] = ck * qv * ((vq[i] - vp[i]) - cm);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float qv = exp2f(fmaf(vq[i], kLog2e, -lq2));
+            const float pv = exp2f(fmaf(vp[i], kLog2e, -lp2));
+            float dz = 0.f;
+            if (qv > 0.f) {
+              const float lm = log2f(0.5f * (pv + qv)) * kLn2;
+              dz = ck * qv * (0.5f * ((vq[i] - lq) - lm) - S);
+            }
+            vq[i] = dz;
+          }
         }
       } else {
         tmem_ld_wait();
@@ -780,6 +949,15 @@ cudaError_t launch_fwd_dual(const CUtensorMap& tHq, const CUtensorMap& tHp, cons
                             cudaStream_t s) {
   return launch_pair<256, 1, 2, 1, 2, false, false, 4, EpiFwdDual>(tHq, tHp, tW, g, p, c, s);
 }
+cudaError_t launch_fwd_argmax(const CUtensorMap& tHq, const CUtensorMap& tHp,
+                              const CUtensorMap& tW, const GemmGeom& g, const FwdParams& p,
+                              const DevCtl& c, cudaStream_t s) {
+  return launch_pair<256, 1, 2, 1, 2, false, false, 4, EpiFwdArgmax>(tHq, tHp, tW, g, p, c, s);
+}
+cudaError_t launch_jsd(const CUtensorMap& tHq, const CUtensorMap& tHp, const CUtensorMap& tW,
+                       const GemmGeom& g, const FwdParams& p, const DevCtl& c, cudaStream_t s) {
+  return launch_pair<256, 1, 2, 1, 2, false, false, 4, EpiJsd>(tHq, tHp, tW, g, p, c, s);
+}
 cudaError_t launch_alpha(const CUtensorMap& tHq, const CUtensorMap& tHp, const CUtensorMap& tW,
                          const GemmGeom& g, const FwdParams& p, const DevCtl& c,
                          cudaStream_t s) {
@@ -864,28 +1042,68 @@ __global__ void __launch_bounds__(kCombineThreads)
       const float L = (M + log2f(S)) * kLn2;
       stats[n] = L;
       loss = valid ? (L - zy[n]) : 0.f;
+    } else if (kind == kCEArgmax) {
+      // Log-sum-exp of the draft; the target's argmax over all slots (the largest value,
+      // the lowest column on ties) and the draft logit there.
+      float Mq = -INFINITY, best = -INFINITY, zq_best = 0.f;
+      int idx = -1;
+      for (int j = 0; j < nch; ++j) {
+        const float* b = part + (int64_t)j * kArgmaxFields * N + n;
+        Mq = fmaxf(Mq, b[0]);
+        const float v = b[2 * N];
+        const int k = __float_as_int(b[3 * N]);
+        if (k >= 0 && (v > best || (v == best && k < idx))) {
+          best = v;
+          idx = k;
+          zq_best = b[4 * N];
+        }
+      }
+      float Sq = 0.f;
+      for (int j = 0; j < nch; ++j) {
+        const float* b = part + (int64_t)j * kArgmaxFields * N + n;
+        Sq += b[N] * exp2f(b[0] - Mq);
+      }
+      const float Lq = (Mq + log2f(Sq)) * kLn2;
+      if (idx < 0) valid = false;
+      stats[n] = Lq;
+      stats[N + n] = __int_as_float(valid ? idx : ignore_index);
+      loss = valid ? (Lq - zq_best) : 0.f;
     } else if (pass == 1) {
       float Mq = -INFINITY, Mp = -INFINITY;
       for (int j = 0; j < nch; ++j) {
-        const float* b = part + (int64_t)j * 5 * N + n;
+        const float* b = part + (int64_t)j * kDualFields * N + n;
         Mq = fmaxf(Mq, b[0]);
         Mp = fmaxf(Mp, b[2 * N]);
       }
-      float Sq = 0.f, Sp = 0.f, A = 0.f;
+      float Sq = 0.f, Sp = 0.f, A = 0.f, B = 0.f;
       for (int j = 0; j < nch; ++j) {
-        const float* b = part + (int64_t)j * 5 * N + n;
-        Sq += b[N] * exp2f(b[0] - Mq);
-        const float r = exp2f(b[2 * N] - Mp);
-        Sp += b[3 * N] * r;
-        A += b[4 * N] * r;
+        const float* b = part + (int64_t)j * kDualFields * N + n;
+        const float rq = exp2f(b[0] - Mq);
+        const float rp = exp2f(b[2 * N] - Mp);
+        Sq += b[N] * rq;
+        B += b[5 * N] * rq;
+        Sp += b[3 * N] * rp;
+        A += b[4 * N] * rp;
       }
       const float Lq = (Mq + log2f(Sq)) * kLn2;
       const float Lp = (Mp + log2f(Sp)) * kLn2;
+      // KL(p||q) = sum p (z_p - z_q) - L_p + L_q;  KL(q||p) = sum q (z_q - z_p) - L_q + L_p.
       const float kl = A / Sp - Lp + Lq;
+      const float rkl = B / Sq - Lq + Lp;
       stats[n] = Lq;
       stats[N + n] = Lp;
-      stats[2 * N + n] = kl;
-      loss = valid ? kl : 0.f;
+      stats[2 * N + n] = (kind == kRKL) ? rkl : kl;
+      loss = valid ? ((kind == kRKL) ? rkl : kl) : 0.f;
+    } else if (kind == kJSD) {
+      float jp = 0.f, jq = 0.f;
+      for (int j = 0; j < nch; ++j) {
+        jp += part[(2 * (int64_t)j) * N + n];
+        jq += part[(2 * (int64_t)j + 1) * N + n];
+      }
+      const float jsd = 0.5f * (jp + jq);
+      stats[3 * N + n] = jsd;
+      stats[4 * N + n] = 0.5f * jq;
+      loss = valid ? jsd : 0.f;
     } else {
       float al = 0.f, S = 0.f;
       for (int j = 0; j < nch; ++j) {

@@ -84,7 +84,7 @@ def lm_head_loss_fwd(kind, hidden, weight, labels=None, target_hidden=None,
             torch.empty(1, dtype=torch.float64, device=dev),
             torch.empty(1, dtype=torch.int64, device=dev),
             torch.empty(N, dtype=torch.float32, device=dev),
-            torch.empty(N, dtype=torch.float32, device=dev) if k >= _lib.SLM_TV else None,
+            torch.empty(N, dtype=torch.float32, device=dev) if k in _lib.ALPHA_KINDS else None,
             torch.empty(nk, N, dtype=torch.float32, device=dev),
             workspace)
     else:

@@ -53,7 +53,8 @@ def gpu_fwd_bwd(inp, kind=None, chunk_tokens=0, grad_tok=None, normalize=True,
     out = dict(
         loss_tok=_np64(fwd.loss_tok), loss_mean=float(fwd.loss_mean.item()),
         loss_sum=float(fwd.loss_sum.item()), n_valid=int(fwd.n_valid.item()),
-        stats=_np64(fwd.stats), alpha=None if fwd.alpha_tok is None else _np64(fwd.alpha_tok),
+        stats=_np64(fwd.stats), stats32=fwd.stats.cpu().numpy(),
+        alpha=None if fwd.alpha_tok is None else _np64(fwd.alpha_tok),
         dH=_np64(dH), dW=_np64(dW), st_fwd=st_fwd, st_bwd=st_bwd,
     )
     assert _lib.SLM_OK == 0
@@ -144,3 +145,36 @@ def assert_grad_close(g, r, what="", slack=0.0):
         assert err <= 1e-6, f"{what}: expected zero gradient, max {err:.3e}"
         return
     assert err / den <= GRAD_RTOL, f"{what}: grad rel err {err / den:.3e} > {GRAD_RTOL}"
+
+
+# Band inside which the GPU's fp32 argmax of the target logits may pick another column
+# than the float64 one: the GPU's z_p carry an absolute error of a few 1e-6 (fp32
+# accumulation over d products), far below this band.
+ARGMAX_BAND = 1e-4
+
+
+def argmax_targets_valid(inp, y_gpu, rows=None):
+    """Check every GPU target is an argmax of the oracle's float64 target logits up to
+    ARGMAX_BAND (masked rows carry ignore_index).  Returns the fraction of rows where the
+    GPU picked another column than the float64 argmax (a near-tie)."""
+    sl = slice(None) if rows is None else rows
+    zp = oracle.logits(inp.Hp[sl], inp.W)
+    y_ref = oracle.argmax_target(zp)
+    y = np.asarray(y_gpu, dtype=np.int64)
+    valid = np.ones(len(y), dtype=bool)
+    if inp.labels is not None:
+        valid = inp.labels[sl].numpy() != inp.ignore_index
+    assert (y[~valid] == inp.ignore_index).all()
+    yv = y[valid]
+    assert ((yv >= 0) & (yv < inp.V)).all()
+    top = zp[valid].max(axis=1)
+    picked = zp[valid][np.arange(valid.sum()), yv]
+    assert (top - picked <= ARGMAX_BAND * np.maximum(1.0, np.abs(top))).all()
+    return float((yv != y_ref[valid]).mean()) if valid.any() else 0.0
+
+
+def with_labels(inp, y):
+    """The same inputs as a hard-label CE problem with labels y."""
+    from lm_head_loss_streaming_b200 import synthetic
+    return synthetic.Inputs("ce", inp.Hq, inp.W, torch.as_tensor(np.asarray(y, np.int32)), None,
+                            inp.ignore_index, dict(inp.meta))

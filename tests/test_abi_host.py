@@ -49,7 +49,10 @@ def test_status_strings_and_sizes(lib):
     assert _lib.slm_stats_floats(_lib.SLM_KL) == 3
     for k in (_lib.SLM_TV, _lib.SLM_NLA, _lib.SLM_LK_HYBRID):
         assert _lib.slm_stats_floats(k) == 5
-    assert _lib.slm_stats_floats(7) == 0
+    assert _lib.slm_stats_floats(_lib.SLM_RKL) == 3
+    assert _lib.slm_stats_floats(_lib.SLM_JSD) == 5
+    assert _lib.slm_stats_floats(_lib.SLM_CE_ARGMAX_P) == 2
+    assert _lib.slm_stats_floats(8) == 0
     assert _lib.slm_workspace_bytes(_lib.SLM_CE, 16, 12, 100) == 0  # d % 8 != 0
     assert _lib.slm_workspace_bytes(9, 16, 16, 100) == 0
 
@@ -87,7 +90,7 @@ def _bwd(**kw):
 
 @pytest.mark.parametrize("fn", [_fwd, _bwd])
 def test_host_errors(lib, fn):
-    assert fn(kind=5) == 4                   # SLM_ERR_KIND
+    assert fn(kind=8) == 4                   # SLM_ERR_KIND
     assert fn(kind=-1) == 4
     assert fn(d=12) == 2                     # SLM_ERR_SHAPE: d % 8
     assert fn(d=0) == 2
@@ -97,6 +100,7 @@ def test_host_errors(lib, fn):
     assert fn(Hq=None) == 1
     assert fn(labels=None) == 1              # CE needs labels
     assert fn(kind=1) == 1                   # KL needs Hp
+    assert fn(kind=7) == 1                   # CE against argmax p needs Hp
     assert fn(workspace=None) == 1
     assert fn(W=A + 8) == 3                  # SLM_ERR_ALIGN
     assert fn(Hq=A + 2) == 3

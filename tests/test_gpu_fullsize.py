@@ -15,12 +15,14 @@ import pytest
 import torch
 
 from lm_head_loss_streaming_b200 import synthetic
-from parity_util import assert_grad_close, assert_loss_close, oracle_fwd_bwd, tie_slack
+from parity_util import (argmax_targets_valid, assert_grad_close, assert_loss_close,
+                         oracle_fwd_bwd, tie_slack, with_labels)
 
 pytestmark = pytest.mark.gpu
 
 CASES = [("llama1b_ce", "ce"), ("llama8b_kl", "kl_div"), ("alpha_losses", "tv"),
-         ("alpha_losses", "nla"), ("alpha_losses", "lk_hybrid"), ("llama405b_ce", "ce")]
+         ("alpha_losses", "nla"), ("alpha_losses", "lk_hybrid"), ("llama405b_ce", "ce"),
+         ("llama8b_kl", "rkl"), ("llama8b_kl", "jsd"), ("llama8b_kl", "ce_argmax_p")]
 R = 48
 
 
@@ -79,7 +81,13 @@ def test_full_size_sampled_rows(name, kind):
     else:
         assert nv == inp.N
 
-    ref = oracle_fwd_bwd(inp, kind, rows=torch.from_numpy(rows),
+    ref_inp, ref_kind = inp, kind
+    if kind == "ce_argmax_p":
+        # The targets are an fp32 argmax: check them, then compare against hard-label CE.
+        y = fwd.stats[1].cpu().numpy().view(np.int32)
+        assert argmax_targets_valid(inp, y[rows], rows=torch.from_numpy(rows)) <= 0.05
+        ref_inp, ref_kind = with_labels(inp, y), "ce"
+    ref = oracle_fwd_bwd(ref_inp, ref_kind, rows=torch.from_numpy(rows),
                          grad_tok=np.ones(len(rows)))
     assert_loss_close(loss_tok[rows], ref["loss_tok"], what=f"{name} {kind} loss")
     sh, sw = tie_slack(inp, kind, rows=torch.from_numpy(rows), grad_tok=np.ones(len(rows)))

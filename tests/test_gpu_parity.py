@@ -9,15 +9,34 @@ import pytest
 import torch
 
 from lm_head_loss_streaming_b200 import synthetic
-from parity_util import (assert_grad_close, assert_loss_close, gpu_fwd_bwd, oracle_fwd_bwd,
-                         tie_slack)
+from parity_util import (argmax_targets_valid, assert_grad_close, assert_loss_close,
+                         gpu_fwd_bwd, oracle_fwd_bwd, tie_slack, with_labels)
 
 pytestmark = pytest.mark.gpu
 
-KINDS = ["ce", "kl_div", "tv", "nla", "lk_hybrid"]
+KINDS = ["ce", "kl_div", "tv", "nla", "lk_hybrid", "rkl", "jsd", "ce_argmax_p"]
+
+
+def _compare_argmax(inp, chunk_tokens=0, what=""):
+    """CE against argmax p: the targets are an argmax decided in fp32 on the GPU.  Check
+    they are valid argmaxes of the float64 target logits, then compare the loss and the
+    gradients with the oracle's hard-label CE on the GPU's targets."""
+    g = gpu_fwd_bwd(inp, "ce_argmax_p", chunk_tokens=chunk_tokens)
+    assert g["st_fwd"] == 0 and g["st_bwd"] == 0, (g["st_fwd"], g["st_bwd"])
+    y = g["stats32"][1].view(np.int32)
+    assert argmax_targets_valid(inp, y) <= 0.01, what
+    r = oracle_fwd_bwd(with_labels(inp, y), "ce")
+    assert g["n_valid"] == r["n_valid"]
+    assert_loss_close(g["loss_tok"], r["loss_tok"], g["loss_mean"], r["loss"], what)
+    assert np.allclose(g["stats"][0], r["lse_q"], rtol=1e-5, atol=1e-4), what
+    assert_grad_close(g["dH"], r["dH"], what + " dH")
+    assert_grad_close(g["dW"], r["dW"], what + " dW")
+    return g, r
 
 
 def _compare(inp, kind, chunk_tokens=0, what=""):
+    if kind == "ce_argmax_p":
+        return _compare_argmax(inp, chunk_tokens, what)
     g = gpu_fwd_bwd(inp, kind, chunk_tokens=chunk_tokens)
     r = oracle_fwd_bwd(inp, kind)
     assert g["st_fwd"] == 0 and g["st_bwd"] == 0, (g["st_fwd"], g["st_bwd"])
@@ -58,7 +77,7 @@ def test_edge_shapes(kind, shape):
     _compare(inp, kind, what=f"edge {kind} {shape}")
 
 
-@pytest.mark.parametrize("kind", ["ce", "kl_div", "lk_hybrid"])
+@pytest.mark.parametrize("kind", ["ce", "kl_div", "lk_hybrid", "jsd", "ce_argmax_p"])
 def test_chunked_backward_matches(kind):
     """The backward's token chunking does not change the result (only reduction order)."""
     inp = synthetic.make(kind, 700, 128, 3000, w_std=0.05, ignore_frac=0.05, seed=3)
@@ -77,9 +96,9 @@ def test_zero_weight_gives_log_v():
     assert np.abs(g["dH"]).max() == 0.0
 
 
-@pytest.mark.parametrize("kind", ["kl_div", "tv", "nla", "lk_hybrid"])
+@pytest.mark.parametrize("kind", ["kl_div", "tv", "nla", "lk_hybrid", "rkl", "jsd"])
 def test_identical_target_and_draft(kind):
-    """p = q: KL = TV = nla = lk = 0, alpha = 1, gradients vanish."""
+    """p = q: KL = TV = nla = lk = RKL = JSD = 0, alpha = 1, gradients vanish."""
     inp = synthetic.make(kind, 150, 128, 2000, w_std=0.05, draft=("none",), seed=5)
     g = gpu_fwd_bwd(inp, kind)
     assert np.abs(g["loss_tok"]).max() <= 2e-3 * 1e-2 * 50
@@ -147,3 +166,12 @@ def test_autograd_wrapper():
     assert abs(loss.item() - r["loss"]) <= 2e-3 * abs(r["loss"])
     assert_grad_close(Hq.grad.double().cpu().numpy(), 2 * r["dH"], "autograd dH")
     assert_grad_close(W.grad.double().cpu().numpy(), 2 * r["dW"], "autograd dW")
+
+
+def test_jsd_bounded_by_log2_on_disjoint_targets():
+    """Target and draft concentrated on different tokens: JSD approaches log 2."""
+    inp = synthetic.make("jsd", 128, 64, 512, w_std=1.5, draft=("mix", -1.0, 0.0), seed=12)
+    g = gpu_fwd_bwd(inp, "jsd")
+    r = oracle_fwd_bwd(inp, "jsd")
+    assert (g["loss_tok"] <= math.log(2) + 2e-3).all() and (g["loss_tok"] >= -2e-3).all()
+    assert_loss_close(g["loss_tok"], r["loss_tok"], g["loss_mean"], r["loss"], "jsd disjoint")

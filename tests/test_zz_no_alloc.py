@@ -33,7 +33,7 @@ def _noalloc_fwd(inp):
     dev = Hq.device
     N, d, V = inp.N, inp.d, inp.V
     loss_tok = torch.full((N,), float("nan"), device=dev)
-    alpha = torch.full((N,), float("nan"), device=dev) if k >= _lib.SLM_TV else None
+    alpha = torch.full((N,), float("nan"), device=dev) if k in _lib.ALPHA_KINDS else None
     loss_sum = torch.zeros(1, dtype=torch.float64, device=dev)
     n_valid = torch.zeros(1, dtype=torch.int64, device=dev)
     loss_mean = torch.zeros(1, device=dev)
