@@ -150,11 +150,13 @@ def make(kind, N, d, V, *, w_std=0.02, h_std=1.0, ignore_frac=0.0, draft=None,
 
 
 def workload(name, *, kind=None, seed=0, device="cpu", N=None) -> Inputs:
-    """Draw the named workload (optionally with fewer token rows ``N``)."""
+    """Draw the named workload (optionally with fewer token rows ``N``).
+
+    ``kind`` defaults to the workload's first kind.  Any other kind draws the workload's
+    shapes and distributions: hard-label CE adds uniform labels; the distribution kinds
+    draw a draft with the workload's recipe (H_q = H_p + 0.5 eps when it has none)."""
     cfg = WORKLOADS[name]
     k = kind or cfg["kinds"][0]
-    if k not in cfg["kinds"]:
-        raise ValueError(f"workload {name} is defined for kinds {cfg['kinds']}")
     inp = make(k, N or cfg["N"], cfg["d"], cfg["V"], w_std=cfg["w_std"],
                ignore_frac=cfg["ignore_frac"], draft=cfg["draft"], seed=seed,
                device=device)
