@@ -65,7 +65,11 @@ def gemm_passes(kind):
 
 
 def fwd_gemm_passes(kind):
-    return 1 if kind == "ce" else 2
+    """Logit-sized GEMMs (2NVd each) in the forward alone: one per operand (draft, and the
+    target for every kind but CE), twice over for the two-pass kinds."""
+    if kind == "ce":
+        return 1
+    return 4 if kind in ("tv", "nla", "lk_hybrid", "jsd") else 2
 
 
 def launches_per_step(kind, N, d, chunk_tokens):
