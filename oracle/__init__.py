@@ -18,6 +18,8 @@ from .slm_oracle import (  # noqa: F401
     forward,
     backward,
     loss_and_grads,
+    combo_forward,
+    combo_backward,
     logits_bytes,
     chunk_buffer_bytes,
 )

@@ -317,3 +317,38 @@ def logits_bytes(batch, seq, vocab, dtype_bytes=4):
 def chunk_buffer_bytes(chunk, vocab, dtype_bytes=4):
     """Peak bytes of one chunk's logits plus their gradient: chunk x vocab x dtype x 2."""
     return int(chunk) * int(vocab) * int(dtype_bytes) * 2
+
+
+# ----------------------------------------------------------------------------------------
+# [LF] "Weighted Combinations": a weighted sum of several losses; the weights are used as
+# given (not normalised) and every term is also reported on its own, before weighting.
+# ----------------------------------------------------------------------------------------
+def combo_forward(weights, Hq, W, labels=None, Hp=None, ignore_index=-100, chunk_size=512):
+    """Weighted combination {kind: weight}.  Every term shares the row mask and the valid
+    count; the combined per-token loss is sum_k w_k l_k and the mean divides it by the
+    valid count.  Returns the combined results plus ``terms`` = {kind: per-term forward}."""
+    terms = {}
+    for kind, w in weights.items():
+        if kind not in KINDS:
+            raise ValueError(f"unknown loss kind {kind!r}")
+        terms[kind] = forward(kind, Hq, W, labels, Hp if kind != "ce" else None, ignore_index,
+                              chunk_size)
+    first = next(iter(terms.values()))
+    tok = sum(float(w) * terms[k]["loss_tok"] for k, w in weights.items())
+    n_valid = first["n_valid"]
+    loss_sum = float(tok.sum())
+    return {"loss_tok": tok, "loss_sum": loss_sum, "n_valid": n_valid,
+            "loss": loss_sum / n_valid if n_valid > 0 else 0.0, "terms": terms}
+
+
+def combo_backward(weights, Hq, W, labels=None, Hp=None, grad_tok=None, ignore_index=-100,
+                   chunk_size=512):
+    """Gradients of the weighted combination: the weighted sum of the terms' gradients."""
+    dH = np.zeros(np.shape(Hq))
+    dW = np.zeros(np.shape(W))
+    for kind, w in weights.items():
+        h, g = backward(kind, Hq, W, labels, Hp if kind != "ce" else None, grad_tok,
+                        ignore_index, chunk_size)
+        dH += float(w) * h
+        dW += float(w) * g
+    return dH, dW

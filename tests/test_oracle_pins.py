@@ -405,3 +405,37 @@ def test_ce_argmax_p_ties_go_to_lowest_index():
     assert int(t["target"][0]) == 1
     lse = math.log(sum(math.exp(v) for v in zq[0]))
     assert abs(t["loss"][0] - (lse - zq[0, 1])) < 1e-14
+
+
+# --------------------------------------------------------------------------------------
+# "Weighted Combinations": weights used as given, each term reported before weighting.
+# --------------------------------------------------------------------------------------
+def test_combination_against_torch_autograd():
+    # {"ce": 0.1, "tv": 0.9} as on the page, plus a three-term mix, against torch.
+    Hq, Hp, W, y = _rand(8, 10, 19, seed=50, w_std=0.7)
+    y[3] = -100
+    for weights in ({"ce": 0.1, "tv": 0.9}, {"kl_div": 1.0, "rkl": 0.5, "jsd": 2.0}):
+        H_t = torch.tensor(Hq, requires_grad=True)
+        W_t = torch.tensor(W, requires_grad=True)
+        zq = H_t @ W_t.T
+        zp = (torch.tensor(Hp) @ W_t.T).detach()
+        valid = torch.tensor(y != -100)
+        total = torch.zeros(8, dtype=torch.float64)
+        for k, w in weights.items():
+            if k == "ce":
+                per = F.cross_entropy(zq, torch.tensor(y), ignore_index=-100, reduction="none")
+            else:
+                per = _torch_loss(k, zq, zp)
+            total = total + w * torch.where(valid, per, torch.zeros_like(per))
+        L = total.sum() / valid.sum()
+        L.backward()
+        out = orc.combo_forward(weights, Hq, W, y, Hp)
+        dH, dW = orc.combo_backward(weights, Hq, W, y, Hp)
+        assert abs(out["loss"] - L.item()) < 1e-12
+        assert np.allclose(out["loss_tok"], total.detach().numpy(), atol=1e-12)
+        assert np.allclose(dH, H_t.grad.numpy(), atol=1e-12)
+        assert np.allclose(dW, W_t.grad.numpy(), atol=1e-12)
+        assert set(out["terms"]) == set(weights)   # each term also reported on its own
+        for k in weights:
+            assert np.allclose(out["terms"][k]["loss_tok"],
+                               orc.forward(k, Hq, W, y, Hp)["loss_tok"], atol=0)
