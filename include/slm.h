@@ -162,6 +162,45 @@ SLM_API int slm_loss_bwd(int kind, const void* Hq, const void* Hp, const void* W
  * word when it starts, so the status describes the most recent call. */
 SLM_API int slm_device_status(const void* workspace, void* stream);
 
+/* ---------------------------------------------------------------------------------------
+ * Weighted combinations ("Loss Functions", section "Weighted Combinations"): the loss is
+ * sum_k w_k * loss_k over the kinds above, with the weights used as given (not
+ * normalised); each term is also reported on its own, before its weight is applied.  Every
+ * term shares the row mask and the valid count, and one logit pass: the forward makes one
+ * pass over the vocabulary (two when a TV, NLA, LK_HYBRID or JSD term is present), the
+ * backward one logit recompute that forms sum_k w_k dz_k, then one dH and one dW GEMM.
+ *   weights  HOST float [SLM_NUM_KINDS], indexed by slm_loss_kind; 0 = term absent; at
+ *            least one nonzero; no NaN or infinity (else SLM_ERR_KIND).
+ *   Hp       required when any term but SLM_CE is present.
+ *   labels   required when the SLM_CE term is present; otherwise an optional row mask.
+ *   term_loss_tok  float [SLM_NUM_KINDS][N] per-term per-token losses before weighting
+ *            (0 for absent terms and masked rows); may be NULL.
+ *   term_loss_sum  double [SLM_NUM_KINDS] per-term loss sums; may be NULL.
+ *   stats    float [SLM_COMBO_STATS][N]: L_q, L_p, KL, RKL, alpha, S, JSD, T, argmax-p
+ *            target (int32 bits; ignore_index on masked rows).
+ * Everything else is as for slm_loss_fwd / slm_loss_bwd; the workspace size comes from
+ * slm_combo_workspace_bytes.
+ * ------------------------------------------------------------------------------------- */
+#define SLM_NUM_KINDS 8
+#define SLM_COMBO_STATS 9
+
+SLM_API size_t slm_combo_workspace_bytes(int64_t N, int64_t d, int64_t V, int64_t chunk_tokens);
+
+SLM_API int slm_combo_fwd(const float* weights, const void* Hq, const void* Hp, const void* W,
+                          const int32_t* labels, int32_t ignore_index,
+                          int64_t N, int64_t d, int64_t V,
+                          float* loss_tok, float* term_loss_tok, double* loss_sum,
+                          double* term_loss_sum, int64_t* n_valid, float* loss_mean,
+                          float* stats, void* workspace, size_t ws_bytes, void* stream);
+
+SLM_API int slm_combo_bwd(const float* weights, const void* Hq, const void* Hp, const void* W,
+                          const int32_t* labels, int32_t ignore_index,
+                          int64_t N, int64_t d, int64_t V,
+                          const float* grad_tok, const float* grad_scale,
+                          const int64_t* n_valid, const float* stats, void* dHq, float* dW,
+                          int accumulate_dW, int64_t chunk_tokens, void* workspace,
+                          size_t ws_bytes, void* stream);
+
 /* Test hook for the device-side failure path (not for production use).  fault_mode 1 makes
  * every following launch withhold one internal pipeline release, so that a bounded wait in
  * the kernel runs out: the kernel then records SLM_ERR_TIMEOUT in the workspace status word,

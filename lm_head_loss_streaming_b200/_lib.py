@@ -19,6 +19,8 @@ KIND = {"ce": SLM_CE, "kl_div": SLM_KL, "tv": SLM_TV, "nla": SLM_NLA,
         "lk_hybrid": SLM_LK_HYBRID, "rkl": SLM_RKL, "jsd": SLM_JSD,
         "ce_argmax_p": SLM_CE_ARGMAX_P}
 ALPHA_KINDS = (SLM_TV, SLM_NLA, SLM_LK_HYBRID)
+SLM_NUM_KINDS = 8
+SLM_COMBO_STATS = 9
 
 SLM_OK = 0
 STATUS_NAMES = {
@@ -44,6 +46,11 @@ SIGNATURES = {
                             _P, _P, _P, _P, _P, _P, _INT, _I64, _P, _SZ, _P]),
     "slm_device_status": (_INT, [_P, _P]),
     "slm_debug_set": (_INT, [_INT, ctypes.c_longlong]),
+    "slm_combo_workspace_bytes": (_SZ, [_I64, _I64, _I64, _I64]),
+    "slm_combo_fwd": (_INT, [_P, _P, _P, _P, _P, _I32, _I64, _I64, _I64,
+                             _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "slm_combo_bwd": (_INT, [_P, _P, _P, _P, _P, _I32, _I64, _I64, _I64,
+                             _P, _P, _P, _P, _P, _P, _INT, _I64, _P, _SZ, _P]),
     "slm_loss_fwd_noalloc": (_INT, [_INT, _P, _P, _P, _P, _I32, _I64, _I64, _I64,
                                     _P, _P, _P, _P, _P, _P, _P, _P]),
 }
@@ -138,3 +145,33 @@ def slm_loss_fwd_noalloc(kind, Hq, Hp, W, labels, ignore_index, N, d, V, loss_to
                                        int(N), int(d), int(V), loss_tok, alpha_tok,
                                        loss_sum, n_valid, loss_mean, stats, device_flags,
                                        stream)
+
+
+def _weights(weights):
+    """Host float[SLM_NUM_KINDS] array from a {kind name or id: weight} mapping."""
+    arr = (ctypes.c_float * SLM_NUM_KINDS)()
+    for k, w in weights.items():
+        arr[KIND[k] if isinstance(k, str) else int(k)] = float(w)
+    return arr
+
+
+def slm_combo_workspace_bytes(N, d, V, chunk_tokens=0):
+    return load().slm_combo_workspace_bytes(int(N), int(d), int(V), int(chunk_tokens))
+
+
+def slm_combo_fwd(weights, Hq, Hp, W, labels, ignore_index, N, d, V, loss_tok, term_loss_tok,
+                  loss_sum, term_loss_sum, n_valid, loss_mean, stats, workspace, ws_bytes,
+                  stream):
+    return load().slm_combo_fwd(_weights(weights), Hq, Hp, W, labels, int(ignore_index),
+                                int(N), int(d), int(V), loss_tok, term_loss_tok, loss_sum,
+                                term_loss_sum, n_valid, loss_mean, stats, workspace,
+                                int(ws_bytes), stream)
+
+
+def slm_combo_bwd(weights, Hq, Hp, W, labels, ignore_index, N, d, V, grad_tok, grad_scale,
+                  n_valid, stats, dHq, dW, accumulate_dW, chunk_tokens, workspace, ws_bytes,
+                  stream):
+    return load().slm_combo_bwd(_weights(weights), Hq, Hp, W, labels, int(ignore_index),
+                                int(N), int(d), int(V), grad_tok, grad_scale, n_valid, stats,
+                                dHq, dW, int(accumulate_dW), int(chunk_tokens), workspace,
+                                int(ws_bytes), stream)

@@ -200,6 +200,82 @@ int common_checks(int kind, const void* Hq, const void* Hp, const void* W, const
   return SLM_OK;
 }
 
+// Weighted combinations: a workspace laid out like the single-kind one, with union
+// partials (kUnionFields per slot), the label logits, the per-term losses [kNumKinds][N],
+// and per-block sums of the total and of every term.
+struct ComboLayout {
+  size_t status_off, red_off, nblk, cnt_off, part_off, zy_off, tl_off, dz_off, ldz;
+  size_t fwd_total, bwd_total, total;
+};
+
+ComboLayout combo_layout(int64_t N, int64_t d, int64_t V, int64_t chunk_tokens) {
+  ComboLayout L{};
+  L.status_off = 0;
+  L.nblk = static_cast<size_t>(std::max<int64_t>(1, ceil_div(N, kCombineThreads)));
+  L.red_off = kAlign;
+  L.cnt_off = align_up(L.red_off + L.nblk * (1 + kNumKinds) * sizeof(double), 16);
+  const size_t big = align_up(L.cnt_off + L.nblk * sizeof(long long), kAlign);
+  const FwdSched f = fwd_sched(SLM_KL, V);
+  L.part_off = big;
+  const size_t part = static_cast<size_t>(f.slots) * kUnionFields * static_cast<size_t>(N) * 4;
+  L.zy_off = align_up(L.part_off + part, kAlign);
+  L.tl_off = align_up(L.zy_off + static_cast<size_t>(N) * 4, kAlign);
+  L.fwd_total = align_up(L.tl_off + static_cast<size_t>(kNumKinds) * N * 4, kAlign);
+  L.ldz = align_up(static_cast<size_t>(V), 8);
+  L.dz_off = big;
+  L.bwd_total =
+      align_up(L.dz_off + static_cast<size_t>(default_chunk(N, d, chunk_tokens)) * L.ldz * 2,
+               kAlign);
+  L.total = std::max(L.fwd_total, L.bwd_total);
+  return L;
+}
+
+// Validates a weight vector; fills the device copy and reports which operands it needs.
+int combo_weights(const float* weights, ComboW* cw, bool* needs_p, bool* needs_labels,
+                  bool* two_pass) {
+  if (!weights) return SLM_ERR_NULL;
+  bool any = false;
+  *needs_p = false;
+  for (int k = 0; k < kNumKinds; ++k) {
+    const float w = weights[k];
+    if (!(w == w) || w > 3.0e38f || w < -3.0e38f) return SLM_ERR_KIND;  // NaN or inf
+    cw->w[k] = w;
+    if (w != 0.f) {
+      any = true;
+      if (k != SLM_CE) *needs_p = true;
+    }
+  }
+  if (!any) return SLM_ERR_KIND;
+  *needs_labels = weights[SLM_CE] != 0.f;
+  *two_pass = weights[SLM_TV] != 0.f || weights[SLM_NLA] != 0.f ||
+              weights[SLM_LK_HYBRID] != 0.f || weights[SLM_JSD] != 0.f;
+  return SLM_OK;
+}
+
+int combo_checks(const float* weights, ComboW* cw, bool* two_pass, const void* Hq,
+                 const void* Hp, const void* W, const int32_t* labels, int64_t N, int64_t d,
+                 int64_t V, const void* workspace, size_t ws_bytes, int64_t chunk_tokens,
+                 bool backward) {
+  bool needs_p = false, needs_labels = false;
+  int st = combo_weights(weights, cw, &needs_p, &needs_labels, two_pass);
+  if (st != SLM_OK) return st;
+  if (N < 0 || d <= 0 || V <= 0 || (d % 8) != 0) return SLM_ERR_SHAPE;
+  if (N >= (int64_t(1) << 31) || V >= (int64_t(1) << 31) || d >= (int64_t(1) << 31))
+    return SLM_ERR_SHAPE;
+  if (!W || !workspace) return SLM_ERR_NULL;
+  if (N > 0) {
+    if (!Hq) return SLM_ERR_NULL;
+    if (needs_p && !Hp) return SLM_ERR_NULL;
+    if (needs_labels && !labels) return SLM_ERR_NULL;
+  }
+  if (misaligned(W, 16) || (Hq && misaligned(Hq, 16)) || (Hp && misaligned(Hp, 16)))
+    return SLM_ERR_ALIGN;
+  if (misaligned(workspace, kAlign)) return SLM_ERR_WORKSPACE;
+  const ComboLayout L = combo_layout(N, d, V, chunk_tokens);
+  if (ws_bytes < (backward ? L.bwd_total : L.fwd_total)) return SLM_ERR_WORKSPACE;
+  return SLM_OK;
+}
+
 #define SLM_TRY_CUDA(expr)                  \
   do {                                      \
     if ((expr) != cudaSuccess) return SLM_ERR_CUDA; \
@@ -268,7 +344,7 @@ int slm_loss_fwd(int kind, const void* Hq, const void* Hp, const void* W, const 
     CUtensorMap tHq, tHp, tW;
     if (!make_map(&tHq, Hq, d, N, d, kBK, kBM)) return SLM_ERR_CUDA;
     if (!make_map(&tW, W, d, V, d, kBK, 128)) return SLM_ERR_CUDA;
-    FwdParams p{labels, ignore_index, N, V, part, zy, stats};
+    FwdParams p{labels, ignore_index, N, V, part, zy, stats, kind == SLM_JSD ? 1 : 0};
     if (!dual_kind(kind)) {
       SLM_TRY_CUDA(launch_fwd_ce(tHq, tW, g, p, ctl, s));
     } else {
@@ -343,7 +419,7 @@ int slm_loss_bwd(int kind, const void* Hq, const void* Hp, const void* W, const 
     if (!make_map(&tHq, hq, d, rows, d, kBK, kBM)) return SLM_ERR_CUDA;
     const GemmGeom gz = geom(rows, V, d, f.bn, f.vc, kGroupPairs, kPairM);
     DzParams pz{dz_kind, dz_labels, ignore_index, c0, rows, N, V, stats, grad_tok, grad_scale,
-                n_valid, dz, ldz};
+                n_valid, dz, ldz, ComboW{}};
     if (!dual_kind(dz_kind)) {
       SLM_TRY_CUDA(launch_dz_ce(tHq, tW_k, gz, pz, ctl, s));
     } else {
@@ -358,6 +434,116 @@ int slm_loss_bwd(int kind, const void* Hq, const void* Hp, const void* W, const 
     DhParams ph{static_cast<__nv_bfloat16*>(dHq), c0, rows, d};
     SLM_TRY_CUDA(launch_dh(tDz_k, tW_mn, gh, ph, ctl, s));
     // 3) dW (+)= dZ^T H[chunk]   (M = V, N = d, K = rows; both operands MN-major).
+    if (!make_map(&tDz_mn, dz, V, rows, ldz, 64, 64)) return SLM_ERR_CUDA;
+    if (!make_map(&tH_mn, hq, d, rows, d, 64, 64)) return SLM_ERR_CUDA;
+    const GemmGeom gw = geom(V, d, rows, kTileDw, 1, 1, kPairM);
+    DwParams pw{dW, V, d, (accumulate_dW || c0 > 0) ? 1 : 0};
+    SLM_TRY_CUDA(launch_dw(tDz_mn, tH_mn, gw, pw, ctl, s));
+  }
+  return SLM_OK;
+}
+
+size_t slm_combo_workspace_bytes(int64_t N, int64_t d, int64_t V, int64_t chunk_tokens) {
+  if (N < 0 || d <= 0 || V <= 0 || (d % 8) != 0) return 0;
+  return combo_layout(N, d, V, chunk_tokens).total;
+}
+
+int slm_combo_fwd(const float* weights, const void* Hq, const void* Hp, const void* W,
+                  const int32_t* labels, int32_t ignore_index, int64_t N, int64_t d, int64_t V,
+                  float* loss_tok, float* term_loss_tok, double* loss_sum,
+                  double* term_loss_sum, int64_t* n_valid, float* loss_mean, float* stats,
+                  void* workspace, size_t ws_bytes, void* stream) {
+  ComboW cw;
+  bool two_pass = false;
+  int st = combo_checks(weights, &cw, &two_pass, Hq, Hp, W, labels, N, d, V, workspace,
+                        ws_bytes, 0, false);
+  if (st != SLM_OK) return st;
+  if (!loss_sum || !n_valid || (N > 0 && !stats)) return SLM_ERR_NULL;
+  if ((st = check_device()) != SLM_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const ComboLayout L = combo_layout(N, d, V, 0);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int* status = reinterpret_cast<int*>(ws + L.status_off);
+  double* blk_sums = reinterpret_cast<double*>(ws + L.red_off);
+  long long* blk_cnt = reinterpret_cast<long long*>(ws + L.cnt_off);
+  float* part = reinterpret_cast<float*>(ws + L.part_off);
+  float* zy = reinterpret_cast<float*>(ws + L.zy_off);
+  float* tl = reinterpret_cast<float*>(ws + L.tl_off);
+  SLM_TRY_CUDA(cudaMemsetAsync(status, 0, sizeof(int), s));
+  const DevCtl ctl = make_ctl(status);
+  if (N > 0) {
+    const FwdSched f = fwd_sched(SLM_KL, V);
+    const GemmGeom g = geom(N, V, d, f.bn, f.vc, kGroupPairs, kPairM);
+    // A CE-only combination has no target: the draft stands in for it (its statistics are
+    // computed and unused).
+    const void* hp = Hp ? Hp : Hq;
+    CUtensorMap tHq, tHp, tW;
+    if (!make_map(&tHq, Hq, d, N, d, kBK, kBM)) return SLM_ERR_CUDA;
+    if (!make_map(&tHp, hp, d, N, d, kBK, kBM)) return SLM_ERR_CUDA;
+    if (!make_map(&tW, W, d, V, d, kBK, 128)) return SLM_ERR_CUDA;
+    FwdParams p{labels, ignore_index, N, V, part, zy, stats, cw.w[SLM_JSD] != 0.f ? 1 : 0};
+    SLM_TRY_CUDA(launch_fwd_union(tHq, tHp, tW, g, p, ctl, s));
+    SLM_TRY_CUDA(launch_combo_combine(1, cw, part, f.slots, zy, labels, ignore_index, N, V,
+                                      stats, tl, status, s));
+    if (two_pass) {
+      SLM_TRY_CUDA(launch_pass2_union(tHq, tHp, tW, g, p, ctl, s));
+      SLM_TRY_CUDA(launch_combo_combine(2, cw, part, f.slots, zy, labels, ignore_index, N, V,
+                                        stats, tl, status, s));
+    }
+  }
+  SLM_TRY_CUDA(launch_combo_total(cw, tl, labels, ignore_index, N, V, loss_tok, term_loss_tok,
+                                  blk_sums, blk_cnt, s));
+  SLM_TRY_CUDA(launch_combo_finalize(blk_sums, blk_cnt, static_cast<int>(L.nblk), loss_sum,
+                                     term_loss_sum, n_valid, loss_mean, s));
+  return SLM_OK;
+}
+
+int slm_combo_bwd(const float* weights, const void* Hq, const void* Hp, const void* W,
+                  const int32_t* labels, int32_t ignore_index, int64_t N, int64_t d, int64_t V,
+                  const float* grad_tok, const float* grad_scale, const int64_t* n_valid,
+                  const float* stats, void* dHq, float* dW, int accumulate_dW,
+                  int64_t chunk_tokens, void* workspace, size_t ws_bytes, void* stream) {
+  ComboW cw;
+  bool two_pass = false;
+  int st = combo_checks(weights, &cw, &two_pass, Hq, Hp, W, labels, N, d, V, workspace,
+                        ws_bytes, chunk_tokens, true);
+  if (st != SLM_OK) return st;
+  if (!dW || (N > 0 && (!dHq || !stats))) return SLM_ERR_NULL;
+  if ((N > 0 && misaligned(dHq, 16)) || misaligned(dW, 16)) return SLM_ERR_ALIGN;
+  if ((st = check_device()) != SLM_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const ComboLayout L = combo_layout(N, d, V, chunk_tokens);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int* status = reinterpret_cast<int*>(ws + L.status_off);
+  __nv_bfloat16* dz = reinterpret_cast<__nv_bfloat16*>(ws + L.dz_off);
+  SLM_TRY_CUDA(cudaMemsetAsync(status, 0, sizeof(int), s));
+  const DevCtl ctl = make_ctl(status);
+  if (N == 0) {
+    if (!accumulate_dW) SLM_TRY_CUDA(launch_zero_f32(dW, V * d, s));
+    return SLM_OK;
+  }
+  const int64_t C = default_chunk(N, d, chunk_tokens);
+  const FwdSched f = fwd_sched(SLM_KL, V);
+  const int64_t ldz = static_cast<int64_t>(L.ldz);
+  const void* hp_all = Hp ? Hp : Hq;
+  CUtensorMap tW_k, tW_mn;
+  if (!make_map(&tW_k, W, d, V, d, kBK, 128)) return SLM_ERR_CUDA;
+  if (!make_map(&tW_mn, W, d, V, d, 64, 64)) return SLM_ERR_CUDA;
+  for (int64_t c0 = 0; c0 < N; c0 += C) {
+    const int64_t rows = std::min<int64_t>(C, N - c0);
+    const __nv_bfloat16* hq = static_cast<const __nv_bfloat16*>(Hq) + c0 * d;
+    const __nv_bfloat16* hp = static_cast<const __nv_bfloat16*>(hp_all) + c0 * d;
+    CUtensorMap tHq, tHp, tDz_k, tDz_mn, tH_mn;
+    if (!make_map(&tHq, hq, d, rows, d, kBK, kBM)) return SLM_ERR_CUDA;
+    if (!make_map(&tHp, hp, d, rows, d, kBK, kBM)) return SLM_ERR_CUDA;
+    const GemmGeom gz = geom(rows, V, d, f.bn, f.vc, kGroupPairs, kPairM);
+    DzParams pz{-1, labels, ignore_index, c0, rows, N, V, stats, grad_tok, grad_scale,
+                n_valid, dz, ldz, cw};
+    SLM_TRY_CUDA(launch_dz_combo(tHq, tHp, tW_k, gz, pz, ctl, s));
+    if (!make_map(&tDz_k, dz, V, rows, ldz, kBK, kBM)) return SLM_ERR_CUDA;
+    const GemmGeom gh = geom(rows, d, V, kTileDh, 1, 1, kPairM);
+    DhParams ph{static_cast<__nv_bfloat16*>(dHq), c0, rows, d};
+    SLM_TRY_CUDA(launch_dh(tDz_k, tW_mn, gh, ph, ctl, s));
     if (!make_map(&tDz_mn, dz, V, rows, ldz, 64, 64)) return SLM_ERR_CUDA;
     if (!make_map(&tH_mn, hq, d, rows, d, 64, 64)) return SLM_ERR_CUDA;
     const GemmGeom gw = geom(V, d, rows, kTileDw, 1, 1, kPairM);

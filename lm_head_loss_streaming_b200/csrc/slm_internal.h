@@ -34,6 +34,15 @@ constexpr int kDualFields = 6;    // m_q, s_q, m_p, s_p, A (p-weighted z_p - z_q
 constexpr int kArgmaxFields = 5;  // m_q, s_q, max z_p, its column, z_q at that column
 constexpr int kCEFields = 2;      // m, s
 
+// Weighted combinations: one weight per loss kind (0 = term absent).
+constexpr int kNumKinds = 8;
+constexpr int kUnionFields = 9;   // pass 1: the dual fields + max z_p, its column, z_q there
+constexpr int kPass2Fields = 4;   // pass 2: alpha, S, jp, jq
+constexpr int kComboStats = 9;    // L_q, L_p, KL, RKL, alpha, S, JSD, T, argmax target
+struct ComboW {
+  float w[kNumKinds];
+};
+
 // Persistent tile schedule.  Work units are (M tile, run of `vc` consecutive N tiles);
 // units are ordered in groups of `group_m` M tiles: for each N run, every M tile of the
 // group, so that CTAs running at the same time share the N-operand tiles in L2.
@@ -61,6 +70,7 @@ struct FwdParams {
   float* part;         // [units_n * kFwdPartsPerRun][fields][N]
   float* zy;           // [N] label logit (CE)
   const float* stats;  // pass 2: L_q, L_p
+  int with_jsd;        // combination pass 2: accumulate the JSD halves too
 };
 
 // Logits-gradient tile (backward recompute + dZ epilogue).
@@ -76,6 +86,7 @@ struct DzParams {
   const int64_t* n_valid;
   __nv_bfloat16* dz;  // [rows][ldz]
   int64_t ldz;
+  ComboW cw;          // weighted combination (EpiDzCombo only)
 };
 
 struct DhParams {
@@ -113,6 +124,32 @@ cudaError_t launch_dh(const CUtensorMap& tDz, const CUtensorMap& tW, const GemmG
                       const DhParams& p, const DevCtl& c, cudaStream_t s);
 cudaError_t launch_dw(const CUtensorMap& tDzT, const CUtensorMap& tH, const GemmGeom& g,
                       const DwParams& p, const DevCtl& c, cudaStream_t s);
+
+// Weighted combinations.
+cudaError_t launch_fwd_union(const CUtensorMap& tHq, const CUtensorMap& tHp,
+                             const CUtensorMap& tW, const GemmGeom& g, const FwdParams& p,
+                             const DevCtl& c, cudaStream_t s);
+cudaError_t launch_pass2_union(const CUtensorMap& tHq, const CUtensorMap& tHp,
+                               const CUtensorMap& tW, const GemmGeom& g, const FwdParams& p,
+                               const DevCtl& c, cudaStream_t s);
+cudaError_t launch_dz_combo(const CUtensorMap& tHq, const CUtensorMap& tHp,
+                            const CUtensorMap& tW, const GemmGeom& g, const DzParams& p,
+                            const DevCtl& c, cudaStream_t s);
+// pass 1: stats 0-3 and 8, per-term losses of ce / kl / rkl / argmax; pass 2: stats 4-7 and
+// the per-term losses of tv / nla / lk / jsd.  term_tok is [kNumKinds][N].
+cudaError_t launch_combo_combine(int pass, const ComboW& cw, const float* part, int nch,
+                                 const float* zy, const int32_t* labels, int32_t ignore_index,
+                                 int64_t N, int64_t V, float* stats, float* term_tok,
+                                 int* status, cudaStream_t s);
+// Weighted per-token total, optional copy of the per-term losses, per-block sums of the
+// total and of every term ([nblk][1 + kNumKinds] doubles) and valid counts.
+cudaError_t launch_combo_total(const ComboW& cw, const float* term_tok, const int32_t* labels,
+                               int32_t ignore_index, int64_t N, int64_t V, float* loss_tok,
+                               float* term_out, double* blk_sums, long long* blk_cnt,
+                               cudaStream_t s);
+cudaError_t launch_combo_finalize(const double* blk_sums, const long long* blk_cnt, int nblk,
+                                  double* loss_sum, double* term_sum, int64_t* n_valid,
+                                  float* loss_mean, cudaStream_t s);
 
 // Row combines and the deterministic loss reduction.
 cudaError_t launch_combine(int kind, int pass, const float* part, int nch, const float* zy,

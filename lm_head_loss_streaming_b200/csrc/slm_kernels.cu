@@ -882,6 +882,238 @@ struct EpiDw {
 };
 
 // ----------------------------------------------------------------------------------------
+// Weighted combinations ("Loss Functions", "Weighted Combinations"): every term shares one
+// logit pass.  Pass 1 gathers the union of the one-pass statistics; pass 2 (only when a
+// term needs the final log-sum-exps) the union of alpha, S and the JSD halves; the
+// backward forms sum_k w_k dz_k in one epilogue.
+// ----------------------------------------------------------------------------------------
+struct EpiFwdUnion {
+  using Params = FwdParams;
+  EpiFwdDual dual;
+  float pmax, zqa, zyv;
+  int pidx;
+  int32_t lab;
+  bool has_zy;
+
+  __device__ __forceinline__ void unit_begin(const Params& p, int row0, int row) {
+    dual.unit_begin(p, row0, row);
+    pmax = -INFINITY;
+    zqa = zyv = 0.f;
+    pidx = -1;
+    has_zy = false;
+    lab = (dual.row_ok && p.labels) ? p.labels[dual.grow] : -1;
+  }
+
+  template <int TN>
+  __device__ __forceinline__ void tile(const Params& p, uint32_t tb, int, int64_t n0, int c0,
+                                       int c1, int) {
+    const int64_t rel = static_cast<int64_t>(lab) - n0;
+#pragma unroll 1
+    for (int c = c0; c < c1; c += 32) {
+      float vq[32], vp[32];
+      tmem_ld32(tb + c, vq);
+      tmem_ld32(tb + TN + c, vp);
+      tmem_ld_wait();
+      const bool tail = n0 + c + 32 > p.V;
+      if (tail) {
+        mask_tail(vq, n0 + c, p.V);
+        mask_tail(vp, n0 + c, p.V);
+      }
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        if (vp[i] > pmax) {
+          pmax = vp[i];
+          pidx = static_cast<int>(n0 + c + i);
+          zqa = vq[i];
+        }
+      }
+      if (static_cast<uint64_t>(rel - c) < 32u) {
+        const int o = static_cast<int>(rel - c);
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          if (i == o) zyv = vq[i];
+        has_zy = true;
+      }
+      if (tail)
+        dual.template chunk<true>(vq, vp);
+      else
+        dual.template chunk<false>(vq, vp);
+    }
+  }
+
+  __device__ __forceinline__ void unit_end(const Params& p, int, int slot, int) {
+    if (!dual.row_ok) return;
+    float* base = p.part + static_cast<int64_t>(slot) * kUnionFields * p.N + dual.grow;
+    base[0 * p.N] = dual.mq;
+    base[1 * p.N] = dual.sq;
+    base[2 * p.N] = dual.mp;
+    base[3 * p.N] = dual.sp;
+    base[4 * p.N] = dual.A;
+    base[5 * p.N] = dual.B;
+    base[6 * p.N] = pmax;
+    base[7 * p.N] = __int_as_float(pidx);
+    base[8 * p.N] = zqa;
+    if (has_zy) p.zy[dual.grow] = zyv;
+  }
+};
+
+struct EpiPass2Union {
+  using Params = FwdParams;
+  float lq, lp, lq2, lp2, al, S, jp, jq;
+  bool row_ok;
+  int64_t grow;
+
+  __device__ __forceinline__ void unit_begin(const Params& p, int row0, int row) {
+    al = S = jp = jq = 0.f;
+    grow = static_cast<int64_t>(row0) + row;
+    row_ok = grow < p.N;
+    lq = row_ok ? p.stats[grow] : 0.f;
+    lp = row_ok ? p.stats[p.N + grow] : 0.f;
+    lq2 = lq * kLog2e;
+    lp2 = lp * kLog2e;
+  }
+
+  template <int TN>
+  __device__ __forceinline__ void tile(const Params& p, uint32_t tb, int, int64_t n0, int c0,
+                                       int c1, int) {
+#pragma unroll 1
+    for (int c = c0; c < c1; c += 32) {
+      float vq[32], vp[32];
+      tmem_ld32(tb + c, vq);
+      tmem_ld32(tb + TN + c, vp);
+      tmem_ld_wait();
+      if (n0 + c + 32 > p.V) {
+        mask_tail(vq, n0 + c, p.V);
+        mask_tail(vp, n0 + c, p.V);
+      }
+      if (p.with_jsd) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float qv = exp2f(fmaf(vq[i], kLog2e, -lq2));
+          const float pv = exp2f(fmaf(vp[i], kLog2e, -lp2));
+          al += fminf(pv, qv);
+          S += (qv < pv) ? qv : 0.f;
+          const float ms = pv + qv;
+          if (ms > 0.f) {
+            const float lm = log2f(0.5f * ms) * kLn2;
+            jp = fmaf(pv, (vp[i] - lp) - lm, jp);
+            jq = fmaf(qv, (vq[i] - lq) - lm, jq);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float qv = exp2f(fmaf(vq[i], kLog2e, -lq2));
+          const float pv = exp2f(fmaf(vp[i], kLog2e, -lp2));
+          al += fminf(pv, qv);
+          S += (qv < pv) ? qv : 0.f;
+        }
+      }
+    }
+  }
+
+  __device__ __forceinline__ void unit_end(const Params& p, int, int slot, int) {
+    if (!row_ok) return;
+    float* base = p.part + static_cast<int64_t>(slot) * kPass2Fields * p.N + grow;
+    base[0 * p.N] = al;
+    base[1 * p.N] = S;
+    base[2 * p.N] = jp;
+    base[3 * p.N] = jq;
+  }
+};
+
+// Logits gradient of a weighted combination:
+//   dz_j = g [ q_j (a0 + a1 (m_j - S) + a2 (z_q,j - z_p,j) + a3 (a_j - T)) - beta p_j
+//              - w_ce [j = y] - w_am [j = y_am] ],   a_j = (log q_j - log M_j) / 2,
+// with a0 = w_ce + w_am + w_kl + w_lk lambda - w_rkl (L_q - L_p + RKL),
+//      a1 = -(w_tv + w_nla / alpha + w_lk (1 - lambda)),  a2 = w_rkl,  a3 = w_jsd,
+//      beta = w_kl + w_lk lambda:  the sum of the per-kind gradients of EpiDz.
+struct EpiDzCombo {
+  using Params = DzParams;
+  float lq, lq2, lp2, a0, a1, a2, a3, beta, S, T, wce, wam;
+  int32_t yce, yam;
+  bool row_ok;
+  int64_t lrow;
+
+  __device__ __forceinline__ void unit_begin(const Params& p, int row0, int row) {
+    lrow = static_cast<int64_t>(row0) + row;
+    row_ok = lrow < p.rows;
+    const int64_t n = p.row0 + lrow;
+    lq = lq2 = lp2 = a0 = a1 = a2 = a3 = beta = S = T = wce = wam = 0.f;
+    yce = yam = -1;
+    if (!row_ok) return;
+    const float* w = p.cw.w;
+    bool valid = true;
+    int32_t lab = -1;
+    if (p.labels) {
+      lab = p.labels[n];
+      valid = lab != p.ignore_index;
+      if (w[kCE] != 0.f && (lab < 0 || lab >= p.V)) valid = false;
+    }
+    const float g = row_grad(p, n, valid);
+    lq = p.stats[n];
+    const float lp = p.stats[p.N + n];
+    lq2 = lq * kLog2e;
+    lp2 = lp * kLog2e;
+    const float rkl = p.stats[3 * p.N + n];
+    const float al = p.stats[4 * p.N + n];
+    S = p.stats[5 * p.N + n];
+    T = p.stats[7 * p.N + n];
+    const float lam = (w[kLK] != 0.f) ? expf(-3.f * al) : 0.f;
+    a0 = g * (w[kCE] + w[kCEArgmax] + w[kKL] + w[kLK] * lam - w[kRKL] * (lq - lp + rkl));
+    a1 = -g * (w[kTV] + ((w[kNLA] != 0.f) ? w[kNLA] / fmaxf(al, 1e-30f) : 0.f) +
+               w[kLK] * (1.f - lam));
+    a2 = g * w[kRKL];
+    a3 = g * w[kJSD];
+    beta = g * (w[kKL] + w[kLK] * lam);
+    wce = g * w[kCE];
+    wam = g * w[kCEArgmax];
+    yce = (w[kCE] != 0.f) ? lab : -1;
+    yam = (w[kCEArgmax] != 0.f) ? __float_as_int(p.stats[8 * p.N + n]) : -1;
+  }
+
+  template <int TN>
+  __device__ __forceinline__ void tile(const Params& p, uint32_t tb, int, int64_t n0, int c0,
+                                       int c1, int) {
+    const float* w = p.cw.w;
+    // Uniform across the launch: which terms need the indicator and log M.
+    const bool need_m = w[kTV] != 0.f || w[kNLA] != 0.f || w[kLK] != 0.f;
+    const bool need_lm = w[kJSD] != 0.f;
+    __nv_bfloat16* out = p.dz + lrow * p.ldz + n0;
+#pragma unroll 1
+    for (int c = c0; c < c1; c += 32) {
+      float vq[32], vp[32];
+      tmem_ld32(tb + c, vq);
+      tmem_ld32(tb + TN + c, vp);
+      tmem_ld_wait();
+      const int64_t rce = static_cast<int64_t>(yce) - (n0 + c);
+      const int64_t ram = static_cast<int64_t>(yam) - (n0 + c);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float qv = exp2f(fmaf(vq[i], kLog2e, -lq2));
+        const float pv = exp2f(fmaf(vp[i], kLog2e, -lp2));
+        float t = fmaf(a2, vq[i] - vp[i], a0);
+        if (need_m) t = fmaf(a1, ((qv < pv) ? 1.f : 0.f) - S, t);
+        if (need_lm) {
+          const float ms = pv + qv;
+          if (ms > 0.f) {
+            const float lm = log2f(0.5f * ms) * kLn2;
+            t = fmaf(a3, 0.5f * ((vq[i] - lq) - lm) - T, t);
+          }
+        }
+        float dz = fmaf(qv, t, -beta * pv);
+        if (rce == i) dz -= wce;
+        if (ram == i) dz -= wam;
+        vq[i] = dz;
+      }
+      if (row_ok && n0 + c < p.V) store_bf16_row32(out + c, vq, n0 + c, p.V);
+    }
+  }
+
+  __device__ __forceinline__ void unit_end(const Params&, int, int, int) {}
+};
+
+// ----------------------------------------------------------------------------------------
 // Launchers: persistent 2-SM launches with clusters of two CTAs, at most as many clusters
 // as can be resident at once (so the static unit schedule never waits for a second wave).
 // ----------------------------------------------------------------------------------------
@@ -957,6 +1189,21 @@ cudaError_t launch_fwd_argmax(const CUtensorMap& tHq, const CUtensorMap& tHp,
 cudaError_t launch_jsd(const CUtensorMap& tHq, const CUtensorMap& tHp, const CUtensorMap& tW,
                        const GemmGeom& g, const FwdParams& p, const DevCtl& c, cudaStream_t s) {
   return launch_pair<256, 1, 2, 1, 2, false, false, 4, EpiJsd>(tHq, tHp, tW, g, p, c, s);
+}
+cudaError_t launch_fwd_union(const CUtensorMap& tHq, const CUtensorMap& tHp,
+                             const CUtensorMap& tW, const GemmGeom& g, const FwdParams& p,
+                             const DevCtl& c, cudaStream_t s) {
+  return launch_pair<256, 1, 2, 1, 2, false, false, 4, EpiFwdUnion>(tHq, tHp, tW, g, p, c, s);
+}
+cudaError_t launch_pass2_union(const CUtensorMap& tHq, const CUtensorMap& tHp,
+                               const CUtensorMap& tW, const GemmGeom& g, const FwdParams& p,
+                               const DevCtl& c, cudaStream_t s) {
+  return launch_pair<256, 1, 2, 1, 2, false, false, 4, EpiPass2Union>(tHq, tHp, tW, g, p, c, s);
+}
+cudaError_t launch_dz_combo(const CUtensorMap& tHq, const CUtensorMap& tHp,
+                            const CUtensorMap& tW, const GemmGeom& g, const DzParams& p,
+                            const DevCtl& c, cudaStream_t s) {
+  return launch_pair<256, 1, 2, 1, 2, false, false, 4, EpiDzCombo>(tHq, tHp, tW, g, p, c, s);
 }
 cudaError_t launch_alpha(const CUtensorMap& tHq, const CUtensorMap& tHp, const CUtensorMap& tW,
                          const GemmGeom& g, const FwdParams& p, const DevCtl& c,
@@ -1194,6 +1441,218 @@ cudaError_t launch_zero_f32(float* p, int64_t n, cudaStream_t s) {
   if (n <= 0) return cudaSuccess;
   const int sms = sm_count() > 0 ? sm_count() : 148;
   zero_f32_kernel<<<sms * 4, 256, 0, s>>>(p, n);
+  return cudaGetLastError();
+}
+
+
+// ----------------------------------------------------------------------------------------
+// Weighted combinations: per-row merge of the union partials into the statistics and the
+// per-term losses, the weighted total, and the fixed-order reductions.
+// ----------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(kCombineThreads)
+    combo_combine_kernel(int pass, ComboW cw, const float* __restrict__ part, int nch,
+                         const float* __restrict__ zy, const int32_t* __restrict__ labels,
+                         int32_t ignore_index, int64_t N, int64_t V, float* stats,
+                         float* term_tok, int* status) {
+  const int64_t n = static_cast<int64_t>(blockIdx.x) * kCombineThreads + threadIdx.x;
+  if (n >= N) return;
+  bool valid = true;
+  if (labels) {
+    const int32_t y = labels[n];
+    valid = y != ignore_index;
+    if (cw.w[kCE] != 0.f && valid && (y < 0 || y >= V)) {
+      if (pass == 1) atomicOr(status, kFlagLabelRange);
+      valid = false;
+    }
+  }
+  if (pass == 1) {
+    float Mq = -INFINITY, Mp = -INFINITY, best = -INFINITY, zq_best = 0.f;
+    int idx = -1;
+    for (int j = 0; j < nch; ++j) {
+      const float* b = part + (int64_t)j * kUnionFields * N + n;
+      Mq = fmaxf(Mq, b[0]);
+      Mp = fmaxf(Mp, b[2 * N]);
+      const float v = b[6 * N];
+      const int k = __float_as_int(b[7 * N]);
+      if (k >= 0 && (v > best || (v == best && k < idx))) {
+        best = v;
+        idx = k;
+        zq_best = b[8 * N];
+      }
+    }
+    float Sq = 0.f, Sp = 0.f, A = 0.f, B = 0.f;
+    for (int j = 0; j < nch; ++j) {
+      const float* b = part + (int64_t)j * kUnionFields * N + n;
+      const float rq = exp2f(b[0] - Mq);
+      const float rp = exp2f(b[2 * N] - Mp);
+      Sq += b[N] * rq;
+      B += b[5 * N] * rq;
+      Sp += b[3 * N] * rp;
+      A += b[4 * N] * rp;
+    }
+    const float Lq = (Mq + log2f(Sq)) * kLn2;
+    const float Lp = (Mp + log2f(Sp)) * kLn2;
+    const float kl = A / Sp - Lp + Lq;
+    const float rkl = B / Sq - Lq + Lp;
+    stats[n] = Lq;
+    stats[N + n] = Lp;
+    stats[2 * N + n] = kl;
+    stats[3 * N + n] = rkl;
+    stats[8 * N + n] = __int_as_float((valid && idx >= 0) ? idx : ignore_index);
+    for (int k = 0; k < kNumKinds; ++k) term_tok[k * N + n] = 0.f;
+    if (valid) {
+      if (cw.w[kCE] != 0.f) term_tok[kCE * N + n] = Lq - zy[n];
+      term_tok[kKL * N + n] = kl;
+      term_tok[kRKL * N + n] = rkl;
+      if (idx >= 0) term_tok[kCEArgmax * N + n] = Lq - zq_best;
+    }
+  } else {
+    float al = 0.f, S = 0.f, jp = 0.f, jq = 0.f;
+    for (int j = 0; j < nch; ++j) {
+      const float* b = part + (int64_t)j * kPass2Fields * N + n;
+      al += b[0];
+      S += b[N];
+      jp += b[2 * N];
+      jq += b[3 * N];
+    }
+    const float jsd = 0.5f * (jp + jq);
+    stats[4 * N + n] = al;
+    stats[5 * N + n] = S;
+    stats[6 * N + n] = jsd;
+    stats[7 * N + n] = 0.5f * jq;
+    if (valid) {
+      const float kl = stats[2 * N + n];
+      const float lam = expf(-3.f * al);
+      term_tok[kTV * N + n] = 1.f - al;
+      term_tok[kNLA * N + n] = -logf(fmaxf(al, 1e-30f));
+      term_tok[kLK * N + n] = lam * kl + (1.f - lam) * (1.f - al);
+      term_tok[kJSD * N + n] = jsd;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kCombineThreads)
+    combo_total_kernel(ComboW cw, const float* __restrict__ term_tok,
+                       const int32_t* __restrict__ labels, int32_t ignore_index, int64_t N,
+                       int64_t V, float* loss_tok, float* term_out, double* blk_sums,
+                       long long* blk_cnt) {
+  constexpr int kW = kCombineThreads / 32;
+  __shared__ double ss[kW][1 + kNumKinds];
+  __shared__ long long sc[kW];
+  const int64_t n = static_cast<int64_t>(blockIdx.x) * kCombineThreads + threadIdx.x;
+  double v[1 + kNumKinds];
+  for (int k = 0; k <= kNumKinds; ++k) v[k] = 0.0;
+  long long cnt = 0;
+  if (n < N) {
+    bool valid = true;
+    if (labels) {
+      const int32_t y = labels[n];
+      valid = y != ignore_index;
+      if (cw.w[kCE] != 0.f && valid && (y < 0 || y >= V)) valid = false;
+    }
+    float total = 0.f;
+    for (int k = 0; k < kNumKinds; ++k) {
+      const float t = valid ? term_tok[k * N + n] : 0.f;
+      if (cw.w[k] != 0.f) total = fmaf(cw.w[k], t, total);
+      if (term_out) term_out[k * N + n] = (cw.w[k] != 0.f) ? t : 0.f;
+      v[1 + k] = (cw.w[k] != 0.f) ? static_cast<double>(t) : 0.0;
+    }
+    if (loss_tok) loss_tok[n] = total;
+    v[0] = static_cast<double>(total);
+    cnt = valid ? 1 : 0;
+  }
+  for (int k = 0; k <= kNumKinds; ++k) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v[k] += __shfl_down_sync(0xffffffffu, v[k], o);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) cnt += __shfl_down_sync(0xffffffffu, cnt, o);
+  const int wi = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0) {
+    for (int k = 0; k <= kNumKinds; ++k) ss[wi][k] = v[k];
+    sc[wi] = cnt;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int k = 0; k <= kNumKinds; ++k) {
+      double t = 0.0;
+      for (int i = 0; i < kW; ++i) t += ss[i][k];
+      blk_sums[static_cast<int64_t>(blockIdx.x) * (1 + kNumKinds) + k] = t;
+    }
+    long long c = 0;
+    for (int i = 0; i < kW; ++i) c += sc[i];
+    blk_cnt[blockIdx.x] = c;
+  }
+}
+
+__global__ void __launch_bounds__(256)
+    combo_finalize_kernel(const double* blk_sums, const long long* blk_cnt, int nblk,
+                          double* loss_sum, double* term_sum, int64_t* n_valid,
+                          float* loss_mean) {
+  __shared__ double ss[8][1 + kNumKinds];
+  __shared__ long long sc[8];
+  double v[1 + kNumKinds];
+  for (int k = 0; k <= kNumKinds; ++k) v[k] = 0.0;
+  long long c = 0;
+  for (int i = threadIdx.x; i < nblk; i += blockDim.x) {
+    for (int k = 0; k <= kNumKinds; ++k) v[k] += blk_sums[static_cast<int64_t>(i) * (1 + kNumKinds) + k];
+    c += blk_cnt[i];
+  }
+  for (int k = 0; k <= kNumKinds; ++k) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v[k] += __shfl_down_sync(0xffffffffu, v[k], o);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) c += __shfl_down_sync(0xffffffffu, c, o);
+  const int wi = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0) {
+    for (int k = 0; k <= kNumKinds; ++k) ss[wi][k] = v[k];
+    sc[wi] = c;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double t[1 + kNumKinds];
+    long long k_valid = 0;
+    for (int k = 0; k <= kNumKinds; ++k) {
+      t[k] = 0.0;
+      for (int i = 0; i < static_cast<int>(blockDim.x >> 5); ++i) t[k] += ss[i][k];
+    }
+    for (int i = 0; i < static_cast<int>(blockDim.x >> 5); ++i) k_valid += sc[i];
+    *loss_sum = t[0];
+    if (term_sum)
+      for (int k = 0; k < kNumKinds; ++k) term_sum[k] = t[1 + k];
+    *n_valid = static_cast<int64_t>(k_valid);
+    if (loss_mean)
+      *loss_mean = k_valid > 0 ? static_cast<float>(t[0] / static_cast<double>(k_valid)) : 0.f;
+  }
+}
+
+cudaError_t launch_combo_combine(int pass, const ComboW& cw, const float* part, int nch,
+                                 const float* zy, const int32_t* labels, int32_t ignore_index,
+                                 int64_t N, int64_t V, float* stats, float* term_tok,
+                                 int* status, cudaStream_t s) {
+  const int blocks = static_cast<int>((N + kCombineThreads - 1) / kCombineThreads);
+  combo_combine_kernel<<<blocks, kCombineThreads, 0, s>>>(pass, cw, part, nch, zy, labels,
+                                                          ignore_index, N, V, stats, term_tok,
+                                                          status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combo_total(const ComboW& cw, const float* term_tok, const int32_t* labels,
+                               int32_t ignore_index, int64_t N, int64_t V, float* loss_tok,
+                               float* term_out, double* blk_sums, long long* blk_cnt,
+                               cudaStream_t s) {
+  const int blocks = static_cast<int>(std::max<int64_t>(1, (N + kCombineThreads - 1) / kCombineThreads));
+  combo_total_kernel<<<blocks, kCombineThreads, 0, s>>>(cw, term_tok, labels, ignore_index, N, V,
+                                                        loss_tok, term_out, blk_sums, blk_cnt);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combo_finalize(const double* blk_sums, const long long* blk_cnt, int nblk,
+                                  double* loss_sum, double* term_sum, int64_t* n_valid,
+                                  float* loss_mean, cudaStream_t s) {
+  combo_finalize_kernel<<<1, 256, 0, s>>>(blk_sums, blk_cnt, nblk, loss_sum, term_sum, n_valid,
+                                          loss_mean);
   return cudaGetLastError();
 }
 

@@ -124,6 +124,75 @@ def lm_head_loss_bwd(fwd: FwdResult, hidden, weight, labels=None, target_hidden=
     return dH, dW
 
 
+@dataclass
+class ComboResult:
+    weights: dict
+    loss_mean: torch.Tensor      # float32 [1], the weighted combination's mean
+    loss_sum: torch.Tensor       # float64 [1]
+    n_valid: torch.Tensor        # int64 [1]
+    loss_tok: torch.Tensor       # float32 [N], sum_k w_k loss_k
+    term_loss_tok: torch.Tensor  # float32 [SLM_NUM_KINDS, N], before weighting
+    term_loss_sum: torch.Tensor  # float64 [SLM_NUM_KINDS]
+    stats: torch.Tensor          # float32 [SLM_COMBO_STATS, N]
+    workspace: torch.Tensor
+
+    def term_means(self):
+        """{kind: mean loss of that term, before weighting} (the per-term log values)."""
+        nv = max(int(self.n_valid.item()), 1)
+        sums = self.term_loss_sum.cpu()
+        return {k: float(sums[_lib.KIND[k]]) / nv for k in self.weights}
+
+
+def lm_head_loss_combo_fwd(weights, hidden, weight, labels=None, target_hidden=None,
+                           ignore_index=IGNORE_INDEX, chunk_tokens=0) -> ComboResult:
+    """Forward of a weighted combination {kind: weight} through ``slm_combo_fwd``."""
+    for k in weights:
+        _kind_id(k)
+    N, d = hidden.shape
+    V = weight.shape[0]
+    dev = hidden.device
+    ws = torch.empty(max(_lib.slm_combo_workspace_bytes(N, d, V, chunk_tokens), 256),
+                     dtype=torch.uint8, device=dev)
+    r = ComboResult(dict(weights), torch.empty(1, device=dev),
+                    torch.empty(1, dtype=torch.float64, device=dev),
+                    torch.empty(1, dtype=torch.int64, device=dev), torch.empty(N, device=dev),
+                    torch.empty(_lib.SLM_NUM_KINDS, N, device=dev),
+                    torch.empty(_lib.SLM_NUM_KINDS, dtype=torch.float64, device=dev),
+                    torch.empty(_lib.SLM_COMBO_STATS, N, device=dev), ws)
+    st = _lib.slm_combo_fwd(weights, _ptr(hidden), _ptr(target_hidden), _ptr(weight),
+                            _ptr(labels), ignore_index, N, d, V, _ptr(r.loss_tok),
+                            _ptr(r.term_loss_tok), _ptr(r.loss_sum), _ptr(r.term_loss_sum),
+                            _ptr(r.n_valid), _ptr(r.loss_mean), _ptr(r.stats), _ptr(ws),
+                            ws.numel(), _stream())
+    _lib.check(st, "slm_combo_fwd")
+    return r
+
+
+def lm_head_loss_combo_bwd(fwd: ComboResult, hidden, weight, labels=None, target_hidden=None,
+                           ignore_index=IGNORE_INDEX, grad_tok=None, grad_scale=None,
+                           normalize=True, dH=None, dW=None, accumulate_dW=False,
+                           chunk_tokens=0):
+    """Backward of a weighted combination through ``slm_combo_bwd``."""
+    N, d = hidden.shape
+    V = weight.shape[0]
+    dev = hidden.device
+    if dH is None:
+        dH = torch.empty(N, d, dtype=torch.bfloat16, device=dev)
+    if dW is None:
+        dW = torch.empty(V, d, dtype=torch.float32, device=dev)
+    ws = fwd.workspace
+    need = _lib.slm_combo_workspace_bytes(N, d, V, chunk_tokens)
+    if ws.numel() < need:
+        ws = torch.empty(need, dtype=torch.uint8, device=dev)
+    st = _lib.slm_combo_bwd(fwd.weights, _ptr(hidden), _ptr(target_hidden), _ptr(weight),
+                            _ptr(labels), ignore_index, N, d, V, _ptr(grad_tok),
+                            _ptr(grad_scale), _ptr(fwd.n_valid) if normalize else None,
+                            _ptr(fwd.stats), _ptr(dH), _ptr(dW), 1 if accumulate_dW else 0,
+                            chunk_tokens, _ptr(ws), ws.numel(), _stream())
+    _lib.check(st, "slm_combo_bwd")
+    return dH, dW
+
+
 def device_status(fwd: FwdResult):
     """Synchronise and return the device status of the last call on this workspace."""
     return _lib.slm_device_status(_ptr(fwd.workspace), _stream())

@@ -124,3 +124,25 @@ def test_debug_hook_arguments(lib):
     assert _lib.slm_debug_set(2, 0) == 2     # SLM_ERR_SHAPE: unknown mode
     assert _lib.slm_debug_set(0, -1) == 2    # SLM_ERR_SHAPE: negative bound
     assert _lib.slm_debug_set(0, 0) == 0     # back to normal operation
+
+
+def _combo_fwd(weights, **kw):
+    args = dict(Hq=A, Hp=A, W=A, labels=A, ignore_index=-100, N=4, d=16, V=32, loss_tok=A,
+                term_loss_tok=None, loss_sum=A, term_loss_sum=None, n_valid=A, loss_mean=None,
+                stats=A, workspace=A, ws_bytes=1 << 30, stream=None)
+    args.update(kw)
+    return _lib.slm_combo_fwd(weights, *args.values())
+
+
+def test_combo_host_errors(lib):
+    assert _lib.slm_combo_workspace_bytes(4, 16, 32) > 0
+    assert _lib.slm_combo_workspace_bytes(4, 12, 32) == 0
+    assert _combo_fwd({}) == 4                          # no term: SLM_ERR_KIND
+    assert _combo_fwd({"kl_div": float("nan")}) == 4    # NaN weight
+    assert _combo_fwd({"kl_div": float("inf")}) == 4
+    assert _combo_fwd({"ce": 1.0}, labels=None) == 1    # CE term needs labels
+    assert _combo_fwd({"tv": 1.0}, Hp=None) == 1        # distribution term needs Hp
+    assert _combo_fwd({"tv": 1.0}, d=12) == 2
+    assert _combo_fwd({"tv": 1.0}, W=A + 8) == 3
+    assert _combo_fwd({"tv": 1.0}, ws_bytes=16) == 5
+    assert _combo_fwd({"tv": 1.0}, stats=None) == 1
