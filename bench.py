@@ -50,6 +50,9 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-sample-rows", type=int, default=0)
+    ap.add_argument("--fused", action="store_true",
+                    help="time the single-call forward+backward that keeps each chunk's "
+                         "logits instead of recomputing them")
     return ap.parse_args()
 
 
@@ -64,12 +67,28 @@ def gemm_passes(kind):
     return {"ce": 4, "kl_div": 6, "rkl": 6, "ce_argmax_p": 5}.get(kind, 8)
 
 
+def fused_gemm_passes(kind):
+    """Logit-sized GEMMs per token of the fused call (the chunk's logits are kept, not
+    recomputed): the forward pass(es) of the first pass only, then dH and dW."""
+    return {"ce": 3}.get(kind, 4)
+
+
 def fwd_gemm_passes(kind):
     """Logit-sized GEMMs (2NVd each) in the forward alone: one per operand (draft, and the
     target for every kind but CE), twice over for the two-pass kinds."""
     if kind == "ce":
         return 1
     return 4 if kind in ("tv", "nla", "lk_hybrid", "jsd") else 2
+
+
+def fused_launches_per_step(kind, N, chunk_tokens):
+    """Kernels of the fused call: count, then per chunk GEMM + combine (+ second pass +
+    combine) + logits-gradient + dH + dW, then finalize."""
+    C = min(chunk_tokens if chunk_tokens > 0 else 4096, N)
+    C = ((C + 255) // 256) * 256 if chunk_tokens > 0 else C
+    chunks = (N + C - 1) // C
+    per = 7 if kind in ("tv", "nla", "lk_hybrid", "jsd") else 5
+    return 2 + per * chunks
 
 
 def launches_per_step(kind, N, d, chunk_tokens):
@@ -222,7 +241,8 @@ def run_ours(args):
 
     from lm_head_loss_streaming_b200 import _lib, dp, synthetic
     from lm_head_loss_streaming_b200.loss import (FwdResult, lm_head_loss_bwd,
-                                                  lm_head_loss_fwd, workspace_bytes)
+                                                  lm_head_loss_fwd, lm_head_loss_fwd_bwd,
+                                                  workspace_bytes)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -241,8 +261,10 @@ def run_ours(args):
     d, V = inp.d, inp.V
     Hq, W, Hp, lab = inp.Hq, inp.W, inp.Hp, inp.labels
     k = _lib.KIND[kind]
-    ws = torch.empty(workspace_bytes(kind, N, d, V, args.chunk_tokens), dtype=torch.uint8,
-                     device=dev)
+    ws_bytes = workspace_bytes(kind, N, d, V, args.chunk_tokens)
+    if args.fused:
+        ws_bytes = max(ws_bytes, _lib.slm_fused_workspace_bytes(k, N, d, V, args.chunk_tokens))
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     nk = _lib.slm_stats_floats(k)
     res = FwdResult(k, torch.empty(1, device=dev), torch.empty(1, dtype=torch.float64, device=dev),
                     torch.empty(1, dtype=torch.int64, device=dev), torch.empty(N, device=dev),
@@ -268,7 +290,17 @@ def run_ours(args):
                                     chunk_tokens=args.chunk_tokens)
 
         def step(ev=None):
-            if world > 1:
+            if args.fused:
+                # One call: forward, logits kept per chunk, backward.  (The data-parallel
+                # exchange needs the global count before the backward, so --fused is 1 GPU.)
+                if ev is not None:
+                    ev[0].record(stream)
+                lm_head_loss_fwd_bwd(kind, Hq_, W_, lab_, Hp_, inp.ignore_index,
+                                     chunk_tokens=args.chunk_tokens, workspace=ws, out=res,
+                                     dH=dH, dW=dW)
+                if ev is not None:
+                    ev[1].record(stream)
+            elif world > 1:
                 # Data parallel over token rows: global valid count before the backward,
                 # dW and the loss sum summed after it (lm_head_loss_streaming_b200.dp).
                 dp.fwd_bwd(lambda: _fwd(ev), _bwd)
@@ -361,9 +393,13 @@ def run_ours(args):
                "ms_per_step": round(e_ms, 3)}
 
     peaks, peak_src = load_peaks()
-    flops_step = gemm_passes(kind) * 2.0 * N * V * d
+    passes = fused_gemm_passes(kind) if args.fused else gemm_passes(kind)
+    flops_step = passes * 2.0 * N * V * d
     base_flops = 8.0 * N * V * d
     fwd_flops = fwd_gemm_passes(kind) * 2.0 * N * V * d
+    if args.fused:
+        # The events bracket the whole fused call: report the step's GEMM flops over it.
+        fwd_flops = flops_step
     achieved = fwd_flops / (fwd_ms / 1e3) / 1e12
     peak = peaks["bf16_tflops_sustained"]
     traffic = traffic_for(args.workload, kind, "fwd_gemm")
@@ -381,6 +417,7 @@ def run_ours(args):
         "dtype": "bf16",
         "data": "synthetic (seeded; no weights or datasets)",
         "config": {"workload": args.workload, "kind": kind, "tokens_per_gpu": N, "d": d,
+                   "path": "fused (chunk logits kept)" if args.fused else "recompute",
                    "V": V, "global_batch_tokens": world * N, "parallelism": f"dp{world}",
                    "chunk_tokens": args.chunk_tokens or "auto",
                    "l2": "inputs larger than L2 (W alone is %.2f GB)" % (V * d * 2 / 1e9)},
@@ -388,11 +425,14 @@ def run_ours(args):
         "frac_bf16_peak": round(flops_step / (ms_step / 1e3) / 1e12 / peaks["bf16_tflops"], 4),
         "frac_bf16_peak_8NVd": round(base_flops / (ms_step / 1e3) / 1e12 / peaks["bf16_tflops"], 4),
         "peak_source": f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback",
-        "roofline": {"bound": "tensor", "kernel": "forward statistics GEMM",
+        "roofline": {"bound": "tensor",
+                     "kernel": ("fused call (all GEMMs + memory-bound logit kernels)"
+                                if args.fused else "forward statistics GEMM"),
                      "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic,
                      "fwd_ms": round(fwd_ms, 3), "peak_kind": "sustained bf16, " + peak_src},
-        "gpu_launches": launches_per_step(kind, N, d, args.chunk_tokens) * args.steps,
+        "gpu_launches": (fused_launches_per_step(kind, N, args.chunk_tokens) if args.fused
+                         else launches_per_step(kind, N, d, args.chunk_tokens)) * args.steps,
         "clocks": clocks,
         "e2e": e2e,
         "kernel_sha": kernel_source_hash(),

@@ -162,6 +162,31 @@ SLM_API int slm_loss_bwd(int kind, const void* Hq, const void* Hp, const void* W
  * word when it starts, so the status describes the most recent call. */
 SLM_API int slm_device_status(const void* workspace, void* stream);
 
+/* Fused forward + backward in one call ("Backward pass": for each token chunk, compute the
+ * logits, the loss and the gradients; the chunk's logits plus gradient buffer bounds the
+ * memory).  For each chunk of chunk_tokens rows (0 = automatic: 4096; rounded up to a
+ * multiple of 256), the forward GEMM keeps the chunk's fp32 logits (the draft's, and the
+ * target's for the distribution kinds) in the workspace, and the logits gradient (and the
+ * second pass of the alpha losses and JSD) read them back instead of recomputing them:
+ * 6NVd flops for CE instead of 8NVd, 8NVd for KL / RKL instead of 12NVd, 8NVd for the
+ * alpha losses and JSD instead of 16NVd, at the cost of about 10 bytes of memory traffic
+ * per logit and a workspace of chunk x V x (4 or 8 + 2) bytes.
+ * Outputs and conventions are those of slm_loss_fwd followed by slm_loss_bwd with
+ * n_valid = the forward's count: the upstream gradient of token n's loss is
+ *     valid_n * (grad_tok ? grad_tok[n] : 1) * (grad_scale ? *grad_scale : 1) / max(n_valid, 1).
+ * The workspace size comes from slm_fused_workspace_bytes. */
+SLM_API size_t slm_fused_workspace_bytes(int kind, int64_t N, int64_t d, int64_t V,
+                                         int64_t chunk_tokens);
+
+SLM_API int slm_loss_fwd_bwd(int kind, const void* Hq, const void* Hp, const void* W,
+                             const int32_t* labels, int32_t ignore_index,
+                             int64_t N, int64_t d, int64_t V,
+                             const float* grad_tok, const float* grad_scale,
+                             float* loss_tok, float* alpha_tok, double* loss_sum,
+                             int64_t* n_valid, float* loss_mean, float* stats,
+                             void* dHq, float* dW, int accumulate_dW, int64_t chunk_tokens,
+                             void* workspace, size_t ws_bytes, void* stream);
+
 /* ---------------------------------------------------------------------------------------
  * Weighted combinations ("Loss Functions", section "Weighted Combinations"): the loss is
  * sum_k w_k * loss_k over the kinds above, with the weights used as given (not

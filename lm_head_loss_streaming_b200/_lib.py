@@ -46,6 +46,9 @@ SIGNATURES = {
                             _P, _P, _P, _P, _P, _P, _INT, _I64, _P, _SZ, _P]),
     "slm_device_status": (_INT, [_P, _P]),
     "slm_debug_set": (_INT, [_INT, ctypes.c_longlong]),
+    "slm_fused_workspace_bytes": (_SZ, [_INT, _I64, _I64, _I64, _I64]),
+    "slm_loss_fwd_bwd": (_INT, [_INT, _P, _P, _P, _P, _I32, _I64, _I64, _I64, _P, _P,
+                                _P, _P, _P, _P, _P, _P, _P, _P, _INT, _I64, _P, _SZ, _P]),
     "slm_combo_workspace_bytes": (_SZ, [_I64, _I64, _I64, _I64]),
     "slm_combo_fwd": (_INT, [_P, _P, _P, _P, _P, _I32, _I64, _I64, _I64,
                              _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
@@ -175,3 +178,18 @@ def slm_combo_bwd(weights, Hq, Hp, W, labels, ignore_index, N, d, V, grad_tok, g
                                 int(N), int(d), int(V), grad_tok, grad_scale, n_valid, stats,
                                 dHq, dW, int(accumulate_dW), int(chunk_tokens), workspace,
                                 int(ws_bytes), stream)
+
+
+def slm_fused_workspace_bytes(kind, N, d, V, chunk_tokens=0):
+    return load().slm_fused_workspace_bytes(int(kind), int(N), int(d), int(V),
+                                            int(chunk_tokens))
+
+
+def slm_loss_fwd_bwd(kind, Hq, Hp, W, labels, ignore_index, N, d, V, grad_tok, grad_scale,
+                     loss_tok, alpha_tok, loss_sum, n_valid, loss_mean, stats, dHq, dW,
+                     accumulate_dW, chunk_tokens, workspace, ws_bytes, stream):
+    return load().slm_loss_fwd_bwd(int(kind), Hq, Hp, W, labels, int(ignore_index), int(N),
+                                   int(d), int(V), grad_tok, grad_scale, loss_tok, alpha_tok,
+                                   loss_sum, n_valid, loss_mean, stats, dHq, dW,
+                                   int(accumulate_dW), int(chunk_tokens), workspace,
+                                   int(ws_bytes), stream)

@@ -14,6 +14,7 @@
 //   backward  for each token chunk: GEMM recompute of the chunk's logits with the
 //             logits-gradient epilogue (bf16 chunk buffer) -> dH = dZ W -> dW (+)= dZ^T H.
 
+#include <stdint.h>
 #include <stdio.h>
 #include <string.h>
 
@@ -276,6 +277,44 @@ int combo_checks(const float* weights, ComboW* cw, bool* two_pass, const void* H
   return SLM_OK;
 }
 
+// Fused forward + backward: per chunk of C token rows, the forward GEMM stores the chunk's
+// fp32 logits (draft, and target for the dual kinds) and the logits gradient and the second
+// pass read them back.  C is a multiple of 256 (the row blocks of the loss reduction).
+int64_t fused_chunk(int64_t N, int64_t chunk_tokens) {
+  if (N <= 0) return 0;
+  int64_t c = chunk_tokens > 0 ? static_cast<int64_t>(align_up(static_cast<size_t>(chunk_tokens), 256))
+                               : 4096;
+  return std::min<int64_t>(c, N);
+}
+
+struct FusedLayout {
+  size_t status_off, red_off, nblk, part_off, zy_off, lq_off, lp_off, dz_off, ldl, ldz, total;
+};
+
+FusedLayout fused_layout(int kind, int64_t N, int64_t V, int64_t chunk_tokens) {
+  FusedLayout L{};
+  L.status_off = 0;
+  L.nblk = static_cast<size_t>(std::max<int64_t>(1, ceil_div(N, kCombineThreads)));
+  L.red_off = kAlign;
+  size_t off = align_up(L.red_off + L.nblk * (sizeof(double) + sizeof(long long)), kAlign);
+  const size_t C = static_cast<size_t>(fused_chunk(N, chunk_tokens));
+  const FwdSched f = fwd_sched(kind, V);
+  L.part_off = off;
+  off = align_up(off + static_cast<size_t>(f.slots) * f.fields * C * 4, kAlign);
+  L.zy_off = off;
+  off = align_up(off + C * 4, kAlign);
+  L.ldl = align_up(static_cast<size_t>(V), 4);
+  L.lq_off = off;
+  off = align_up(off + C * L.ldl * 4, kAlign);
+  L.lp_off = off;
+  if (dual_kind(kind) && kind != SLM_CE_ARGMAX_P) off = align_up(off + C * L.ldl * 4, kAlign);
+  L.ldz = align_up(static_cast<size_t>(V), 8);
+  L.dz_off = off;
+  off = align_up(off + C * L.ldz * 2, kAlign);
+  L.total = off;
+  return L;
+}
+
 #define SLM_TRY_CUDA(expr)                  \
   do {                                      \
     if ((expr) != cudaSuccess) return SLM_ERR_CUDA; \
@@ -344,7 +383,8 @@ int slm_loss_fwd(int kind, const void* Hq, const void* Hp, const void* W, const 
     CUtensorMap tHq, tHp, tW;
     if (!make_map(&tHq, Hq, d, N, d, kBK, kBM)) return SLM_ERR_CUDA;
     if (!make_map(&tW, W, d, V, d, kBK, 128)) return SLM_ERR_CUDA;
-    FwdParams p{labels, ignore_index, N, V, part, zy, stats, kind == SLM_JSD ? 1 : 0};
+    FwdParams p{labels, ignore_index, N, V, part, zy, stats, kind == SLM_JSD ? 1 : 0,
+                nullptr, nullptr, 0};
     if (!dual_kind(kind)) {
       SLM_TRY_CUDA(launch_fwd_ce(tHq, tW, g, p, ctl, s));
     } else {
@@ -443,6 +483,104 @@ int slm_loss_bwd(int kind, const void* Hq, const void* Hp, const void* W, const 
   return SLM_OK;
 }
 
+size_t slm_fused_workspace_bytes(int kind, int64_t N, int64_t d, int64_t V,
+                                 int64_t chunk_tokens) {
+  if (!valid_kind(kind) || N < 0 || d <= 0 || V <= 0 || (d % 8) != 0) return 0;
+  return fused_layout(kind, N, V, chunk_tokens).total;
+}
+
+int slm_loss_fwd_bwd(int kind, const void* Hq, const void* Hp, const void* W,
+                     const int32_t* labels, int32_t ignore_index, int64_t N, int64_t d,
+                     int64_t V, const float* grad_tok, const float* grad_scale, float* loss_tok,
+                     float* alpha_tok, double* loss_sum, int64_t* n_valid, float* loss_mean,
+                     float* stats, void* dHq, float* dW, int accumulate_dW,
+                     int64_t chunk_tokens, void* workspace, size_t ws_bytes, void* stream) {
+  // Shapes, pointers and alignment as for the two-call path; the workspace is checked below.
+  int st = common_checks(kind, Hq, Hp, W, labels, N, d, V, workspace, SIZE_MAX, 0, false);
+  if (st != SLM_OK) return st;
+  if (!loss_sum || !n_valid || !dW || (N > 0 && (!stats || !dHq))) return SLM_ERR_NULL;
+  if ((N > 0 && misaligned(dHq, 16)) || misaligned(dW, 16)) return SLM_ERR_ALIGN;
+  const FusedLayout L = fused_layout(kind, N, V, chunk_tokens);
+  if (ws_bytes < L.total) return SLM_ERR_WORKSPACE;
+  if ((st = check_device()) != SLM_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int* status = reinterpret_cast<int*>(ws + L.status_off);
+  double* blk_sum = reinterpret_cast<double*>(ws + L.red_off);
+  long long* blk_cnt = reinterpret_cast<long long*>(blk_sum + L.nblk);
+  float* part = reinterpret_cast<float*>(ws + L.part_off);
+  float* zy = reinterpret_cast<float*>(ws + L.zy_off);
+  float* lq = reinterpret_cast<float*>(ws + L.lq_off);
+  float* lp = reinterpret_cast<float*>(ws + L.lp_off);
+  __nv_bfloat16* dz = reinterpret_cast<__nv_bfloat16*>(ws + L.dz_off);
+  const int64_t ldl = static_cast<int64_t>(L.ldl);
+  const int64_t ldz = static_cast<int64_t>(L.ldz);
+  SLM_TRY_CUDA(cudaMemsetAsync(status, 0, sizeof(int), s));
+  const DevCtl ctl = make_ctl(status);
+  if (N == 0) {
+    SLM_TRY_CUDA(cudaMemsetAsync(blk_sum, 0, L.nblk * (sizeof(double) + sizeof(long long)), s));
+    SLM_TRY_CUDA(launch_finalize(blk_sum, blk_cnt, static_cast<int>(L.nblk), loss_sum, n_valid,
+                                 loss_mean, s));
+    if (!accumulate_dW) SLM_TRY_CUDA(launch_zero_f32(dW, V * d, s));
+    return SLM_OK;
+  }
+  // The mean's denominator is needed before the first chunk's gradient.
+  SLM_TRY_CUDA(launch_count_valid(labels, ignore_index, N, V, kind == SLM_CE ? 1 : 0, n_valid, s));
+  const int64_t C = fused_chunk(N, chunk_tokens);
+  const FwdSched f = fwd_sched(kind, V);
+  const bool argmax_kind = kind == SLM_CE_ARGMAX_P;
+  const int dz_kind = argmax_kind ? SLM_CE : kind;
+  const int32_t* dz_labels = argmax_kind ? reinterpret_cast<const int32_t*>(stats + N) : labels;
+  CUtensorMap tW, tW_mn;
+  if (!make_map(&tW, W, d, V, d, kBK, 128)) return SLM_ERR_CUDA;
+  if (!make_map(&tW_mn, W, d, V, d, 64, 64)) return SLM_ERR_CUDA;
+  for (int64_t c0 = 0; c0 < N; c0 += C) {
+    const int64_t rows = std::min<int64_t>(C, N - c0);
+    const __nv_bfloat16* hq = static_cast<const __nv_bfloat16*>(Hq) + c0 * d;
+    CUtensorMap tHq, tHp, tDz_k, tDz_mn, tH_mn;
+    if (!make_map(&tHq, hq, d, rows, d, kBK, kBM)) return SLM_ERR_CUDA;
+    // 1) Logits of the chunk: statistics in the epilogue, fp32 logits kept.
+    const GemmGeom g = geom(rows, V, d, f.bn, f.vc, kGroupPairs, kPairM);
+    FwdParams p{labels ? labels + c0 : nullptr, ignore_index, rows, V, part, zy, nullptr, 0,
+                lq, (dual_kind(kind) && !argmax_kind) ? lp : nullptr, ldl};
+    if (!dual_kind(kind)) {
+      SLM_TRY_CUDA(launch_fwd_ce(tHq, tW, g, p, ctl, s));
+    } else {
+      const __nv_bfloat16* hp = static_cast<const __nv_bfloat16*>(Hp) + c0 * d;
+      if (!make_map(&tHp, hp, d, rows, d, kBK, kBM)) return SLM_ERR_CUDA;
+      if (argmax_kind)
+        SLM_TRY_CUDA(launch_fwd_argmax(tHq, tHp, tW, g, p, ctl, s));
+      else
+        SLM_TRY_CUDA(launch_fwd_dual(tHq, tHp, tW, g, p, ctl, s));
+    }
+    SLM_TRY_CUDA(launch_combine(kind, 1, part, f.slots, zy, labels, ignore_index, rows, V,
+                                loss_tok, alpha_tok, stats, blk_sum, blk_cnt, status, s, c0, N));
+    // 2) Second pass of the alpha losses / JSD over the kept logits.
+    if (two_pass_kind(kind)) {
+      SLM_TRY_CUDA(launch_logits_pass2(kind, lq, lp, ldl, stats, c0, N, rows, V, part, s));
+      SLM_TRY_CUDA(launch_combine(kind, 2, part, 1, zy, labels, ignore_index, rows, V, loss_tok,
+                                  alpha_tok, stats, blk_sum, blk_cnt, status, s, c0, N));
+    }
+    // 3) Logits gradient of the chunk from the kept logits.
+    DzParams pz{dz_kind, dz_labels, ignore_index, c0, rows, N, V, stats, grad_tok, grad_scale,
+                n_valid, dz, ldz, ComboW{}};
+    SLM_TRY_CUDA(launch_logits_dz(pz, lq, lp, ldl, s));
+    // 4) dH[chunk] = dZ W and dW (+)= dZ^T H[chunk].
+    if (!make_map(&tDz_k, dz, V, rows, ldz, kBK, kBM)) return SLM_ERR_CUDA;
+    const GemmGeom gh = geom(rows, d, V, kTileDh, 1, 1, kPairM);
+    DhParams ph{static_cast<__nv_bfloat16*>(dHq), c0, rows, d};
+    SLM_TRY_CUDA(launch_dh(tDz_k, tW_mn, gh, ph, ctl, s));
+    if (!make_map(&tDz_mn, dz, V, rows, ldz, 64, 64)) return SLM_ERR_CUDA;
+    if (!make_map(&tH_mn, hq, d, rows, d, 64, 64)) return SLM_ERR_CUDA;
+    const GemmGeom gw = geom(V, d, rows, kTileDw, 1, 1, kPairM);
+    DwParams pw{dW, V, d, (accumulate_dW || c0 > 0) ? 1 : 0};
+    SLM_TRY_CUDA(launch_dw(tDz_mn, tH_mn, gw, pw, ctl, s));
+  }
+  SLM_TRY_CUDA(launch_finalize(blk_sum, blk_cnt, static_cast<int>(L.nblk), loss_sum, n_valid,
+                               loss_mean, s));
+  return SLM_OK;
+}
+
 size_t slm_combo_workspace_bytes(int64_t N, int64_t d, int64_t V, int64_t chunk_tokens) {
   if (N < 0 || d <= 0 || V <= 0 || (d % 8) != 0) return 0;
   return combo_layout(N, d, V, chunk_tokens).total;
@@ -481,7 +619,8 @@ int slm_combo_fwd(const float* weights, const void* Hq, const void* Hp, const vo
     if (!make_map(&tHq, Hq, d, N, d, kBK, kBM)) return SLM_ERR_CUDA;
     if (!make_map(&tHp, hp, d, N, d, kBK, kBM)) return SLM_ERR_CUDA;
     if (!make_map(&tW, W, d, V, d, kBK, 128)) return SLM_ERR_CUDA;
-    FwdParams p{labels, ignore_index, N, V, part, zy, stats, cw.w[SLM_JSD] != 0.f ? 1 : 0};
+    FwdParams p{labels, ignore_index, N, V, part, zy, stats, cw.w[SLM_JSD] != 0.f ? 1 : 0,
+                nullptr, nullptr, 0};
     SLM_TRY_CUDA(launch_fwd_union(tHq, tHp, tW, g, p, ctl, s));
     SLM_TRY_CUDA(launch_combo_combine(1, cw, part, f.slots, zy, labels, ignore_index, N, V,
                                       stats, tl, status, s));

@@ -71,6 +71,9 @@ struct FwdParams {
   float* zy;           // [N] label logit (CE)
   const float* stats;  // pass 2: L_q, L_p
   int with_jsd;        // combination pass 2: accumulate the JSD halves too
+  float* lq_out;       // fused path: store the fp32 draft logits here ([N][ldl]), or NULL
+  float* lp_out;       // fused path: store the fp32 target logits here, or NULL
+  int64_t ldl;         // leading dimension of the stored logits (V rounded up to 4)
 };
 
 // Logits-gradient tile (backward recompute + dZ epilogue).
@@ -125,6 +128,18 @@ cudaError_t launch_dh(const CUtensorMap& tDz, const CUtensorMap& tW, const GemmG
 cudaError_t launch_dw(const CUtensorMap& tDzT, const CUtensorMap& tH, const GemmGeom& g,
                       const DwParams& p, const DevCtl& c, cudaStream_t s);
 
+// Fused forward + backward over stored chunk logits.
+// Valid rows (label != ignore_index; for CE also in [0, V)) -> *n_valid.
+cudaError_t launch_count_valid(const int32_t* labels, int32_t ignore_index, int64_t N,
+                               int64_t V, int check_range, int64_t* n_valid, cudaStream_t s);
+// Second pass of the alpha losses / JSD from stored logits: one partial slot per row.
+cudaError_t launch_logits_pass2(int kind, const float* lq, const float* lp, int64_t ldl,
+                                const float* stats, int64_t row0, int64_t ldN, int64_t rows,
+                                int64_t V, float* part, cudaStream_t s);
+// Logits gradient of the rows [p.row0, p.row0 + p.rows) from stored logits.
+cudaError_t launch_logits_dz(const DzParams& p, const float* lq, const float* lp, int64_t ldl,
+                             cudaStream_t s);
+
 // Weighted combinations.
 cudaError_t launch_fwd_union(const CUtensorMap& tHq, const CUtensorMap& tHp,
                              const CUtensorMap& tW, const GemmGeom& g, const FwdParams& p,
@@ -152,10 +167,13 @@ cudaError_t launch_combo_finalize(const double* blk_sums, const long long* blk_c
                                   float* loss_mean, cudaStream_t s);
 
 // Row combines and the deterministic loss reduction.
+// N rows starting at row0 of a batch whose statistics have leading dimension ldN
+// (-1: ldN = N); partials and label logits are indexed by the row within the launch.
 cudaError_t launch_combine(int kind, int pass, const float* part, int nch, const float* zy,
                            const int32_t* labels, int32_t ignore_index, int64_t N, int64_t V,
                            float* loss_tok, float* alpha_tok, float* stats, double* blk_sum,
-                           long long* blk_cnt, int* status, cudaStream_t s);
+                           long long* blk_cnt, int* status, cudaStream_t s, int64_t row0 = 0,
+                           int64_t ldN = -1);
 cudaError_t launch_finalize(const double* blk_sum, const long long* blk_cnt, int nblk,
                             double* loss_sum, int64_t* n_valid, float* loss_mean,
                             cudaStream_t s);

@@ -359,6 +359,17 @@ __device__ __forceinline__ void mask_tail(float (&v)[32], int64_t col0, int64_t 
     if (col0 + i >= V) v[i] = -INFINITY;
 }
 
+// Fused path: store 32 fp32 logits of one row (columns >= V land in the row padding; the
+// leading dimension is V rounded up to 4, so every float4 that starts below V fits).
+__device__ __forceinline__ void store_f32_row32(float* dst, const float (&v)[32], int64_t col0,
+                                                int64_t V) {
+#pragma unroll
+  for (int k = 0; k < 8; ++k)
+    if (col0 + 4 * k < V)
+      reinterpret_cast<float4*>(dst)[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2],
+                                                      v[4 * k + 3]);
+}
+
 // CE forward: per row, online max m (log2 units) and s = sum 2^(z log2e - m) over the
 // warpgroup's columns of the unit's vocabulary run, plus the label logit z_y when the
 // label falls there.
@@ -389,6 +400,7 @@ struct EpiFwdCE {
       tmem_ld32(tb + c, v);
       tmem_ld_wait();
       if (n0 + c + 32 > p.V) mask_tail(v, n0 + c, p.V);
+      if (p.lq_out && row_ok) store_f32_row32(p.lq_out + grow * p.ldl + n0 + c, v, n0 + c, p.V);
       if (static_cast<uint64_t>(rel - c) < 32u) {
         const int o = static_cast<int>(rel - c);
 #pragma unroll
@@ -482,13 +494,19 @@ struct EpiFwdDual {
       tmem_ld32(tb + c, vq);
       tmem_ld32(tb + TN + c, vp);
       tmem_ld_wait();
-      if (n0 + c + 32 > p.V) {
+      const bool tail = n0 + c + 32 > p.V;
+      if (tail) {
         mask_tail(vq, n0 + c, p.V);
         mask_tail(vp, n0 + c, p.V);
-        chunk<true>(vq, vp);
-      } else {
-        chunk<false>(vq, vp);
       }
+      if (p.lq_out && row_ok) {
+        store_f32_row32(p.lq_out + grow * p.ldl + n0 + c, vq, n0 + c, p.V);
+        store_f32_row32(p.lp_out + grow * p.ldl + n0 + c, vp, n0 + c, p.V);
+      }
+      if (tail)
+        chunk<true>(vq, vp);
+      else
+        chunk<false>(vq, vp);
     }
   }
 
@@ -536,6 +554,7 @@ struct EpiFwdArgmax {
         mask_tail(vq, n0 + c, p.V);
         mask_tail(vp, n0 + c, p.V);
       }
+      if (p.lq_out && row_ok) store_f32_row32(p.lq_out + grow * p.ldl + n0 + c, vq, n0 + c, p.V);
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
         if (vp[i] > pmax) {
@@ -769,18 +788,12 @@ struct EpiDz {
     }
   }
 
-  template <int TN>
-  __device__ __forceinline__ void tile(const Params& p, uint32_t tb, int, int64_t n0, int c0,
-                                       int c1, int) {
-    __nv_bfloat16* out = p.dz + lrow * p.ldz + n0;
-#pragma unroll 1
-    for (int c = c0; c < c1; c += 32) {
-      float vq[32];
-      tmem_ld32(tb + c, vq);
-      if (DUAL) {
-        float vp[32];
-        tmem_ld32(tb + TN + c, vp);
-        tmem_ld_wait();
+  // vq (draft logits of columns [col0, col0 + 32)) becomes dz; vp holds the target logits
+  // of the same columns (unused for CE).
+  __device__ __forceinline__ void apply(float (&vq)[32], const float (&vp)[32],
+                                        int64_t col0) const {
+    if (DUAL) {
+      {
         if (mode == 0) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
@@ -808,15 +821,28 @@ struct EpiDz {
             vq[i] = dz;
           }
         }
-      } else {
-        tmem_ld_wait();
-        const int64_t rel = static_cast<int64_t>(lab) - (n0 + c);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float qv = exp2f(fmaf(vq[i], kLog2e, -lq2));
-          vq[i] = g * (qv - (rel == i ? 1.f : 0.f));
-        }
       }
+    } else {
+      const int64_t rel = static_cast<int64_t>(lab) - col0;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float qv = exp2f(fmaf(vq[i], kLog2e, -lq2));
+        vq[i] = g * (qv - (rel == i ? 1.f : 0.f));
+      }
+    }
+  }
+
+  template <int TN>
+  __device__ __forceinline__ void tile(const Params& p, uint32_t tb, int, int64_t n0, int c0,
+                                       int c1, int) {
+    __nv_bfloat16* out = p.dz + lrow * p.ldz + n0;
+#pragma unroll 1
+    for (int c = c0; c < c1; c += 32) {
+      float vq[32], vp[32];
+      tmem_ld32(tb + c, vq);
+      if (DUAL) tmem_ld32(tb + TN + c, vp);
+      tmem_ld_wait();
+      apply(vq, vp, n0 + c);
       if (row_ok && n0 + c < p.V) store_bf16_row32(out + c, vq, n0 + c, p.V);
     }
   }
@@ -1264,15 +1290,18 @@ __global__ void __launch_bounds__(kCombineThreads)
                    const float* __restrict__ zy, const int32_t* __restrict__ labels,
                    int32_t ignore_index, int64_t N, int64_t V, float* loss_tok,
                    float* alpha_tok, float* stats, double* blk_sum, long long* blk_cnt,
-                   int* status) {
+                   int* status, int64_t row0, int64_t ldN) {
+  // n: row within this launch (partials and label logits are indexed by it);
+  // gn = row0 + n: the row of the whole batch (labels, statistics, per-token outputs).
   const int64_t n = static_cast<int64_t>(blockIdx.x) * kCombineThreads + threadIdx.x;
+  const int64_t gn = row0 + n;
   double lsum = 0.0;
   long long cnt = 0;
   if (n < N) {
     bool valid = true;
     int32_t y = 0;
     if (labels) {
-      y = labels[n];
+      y = labels[gn];
       valid = y != ignore_index;
       if (kind == kCE && valid && (y < 0 || y >= V)) {
         atomicOr(status, kFlagLabelRange);
@@ -1287,7 +1316,7 @@ __global__ void __launch_bounds__(kCombineThreads)
       for (int j = 0; j < nch; ++j)
         S += part[(2 * (int64_t)j + 1) * N + n] * exp2f(part[(2 * (int64_t)j) * N + n] - M);
       const float L = (M + log2f(S)) * kLn2;
-      stats[n] = L;
+      stats[gn] = L;
       loss = valid ? (L - zy[n]) : 0.f;
     } else if (kind == kCEArgmax) {
       // Log-sum-exp of the draft; the target's argmax over all slots (the largest value,
@@ -1312,8 +1341,8 @@ __global__ void __launch_bounds__(kCombineThreads)
       }
       const float Lq = (Mq + log2f(Sq)) * kLn2;
       if (idx < 0) valid = false;
-      stats[n] = Lq;
-      stats[N + n] = __int_as_float(valid ? idx : ignore_index);
+      stats[gn] = Lq;
+      stats[ldN + gn] = __int_as_float(valid ? idx : ignore_index);
       loss = valid ? (Lq - zq_best) : 0.f;
     } else if (pass == 1) {
       float Mq = -INFINITY, Mp = -INFINITY;
@@ -1337,9 +1366,9 @@ __global__ void __launch_bounds__(kCombineThreads)
       // KL(p||q) = sum p (z_p - z_q) - L_p + L_q;  KL(q||p) = sum q (z_q - z_p) - L_q + L_p.
       const float kl = A / Sp - Lp + Lq;
       const float rkl = B / Sq - Lq + Lp;
-      stats[n] = Lq;
-      stats[N + n] = Lp;
-      stats[2 * N + n] = (kind == kRKL) ? rkl : kl;
+      stats[gn] = Lq;
+      stats[ldN + gn] = Lp;
+      stats[2 * ldN + gn] = (kind == kRKL) ? rkl : kl;
       loss = valid ? ((kind == kRKL) ? rkl : kl) : 0.f;
     } else if (kind == kJSD) {
       float jp = 0.f, jq = 0.f;
@@ -1348,8 +1377,8 @@ __global__ void __launch_bounds__(kCombineThreads)
         jq += part[(2 * (int64_t)j + 1) * N + n];
       }
       const float jsd = 0.5f * (jp + jq);
-      stats[3 * N + n] = jsd;
-      stats[4 * N + n] = 0.5f * jq;
+      stats[3 * ldN + gn] = jsd;
+      stats[4 * ldN + gn] = 0.5f * jq;
       loss = valid ? jsd : 0.f;
     } else {
       float al = 0.f, S = 0.f;
@@ -1357,10 +1386,10 @@ __global__ void __launch_bounds__(kCombineThreads)
         al += part[(2 * (int64_t)j) * N + n];
         S += part[(2 * (int64_t)j + 1) * N + n];
       }
-      stats[3 * N + n] = al;
-      stats[4 * N + n] = S;
-      if (alpha_tok) alpha_tok[n] = al;
-      const float kl = stats[2 * N + n];
+      stats[3 * ldN + gn] = al;
+      stats[4 * ldN + gn] = S;
+      if (alpha_tok) alpha_tok[gn] = al;
+      const float kl = stats[2 * ldN + gn];
       float l;
       if (kind == kTV) {
         l = 1.f - al;
@@ -1372,11 +1401,11 @@ __global__ void __launch_bounds__(kCombineThreads)
       }
       loss = valid ? l : 0.f;
     }
-    if (loss_tok) loss_tok[n] = loss;
+    if (loss_tok) loss_tok[gn] = loss;
     lsum = static_cast<double>(loss);
     cnt = valid ? 1 : 0;
   }
-  block_reduce_store(lsum, cnt, blk_sum, blk_cnt);
+  block_reduce_store(lsum, cnt, blk_sum + row0 / kCombineThreads, blk_cnt + row0 / kCombineThreads);
 }
 
 __global__ void __launch_bounds__(1024)
@@ -1422,11 +1451,13 @@ __global__ void zero_f32_kernel(float* p, int64_t n) {
 cudaError_t launch_combine(int kind, int pass, const float* part, int nch, const float* zy,
                            const int32_t* labels, int32_t ignore_index, int64_t N, int64_t V,
                            float* loss_tok, float* alpha_tok, float* stats, double* blk_sum,
-                           long long* blk_cnt, int* status, cudaStream_t s) {
+                           long long* blk_cnt, int* status, cudaStream_t s, int64_t row0,
+                           int64_t ldN) {
+  if (ldN < 0) ldN = N;
   const int blocks = static_cast<int>((N + kCombineThreads - 1) / kCombineThreads);
   combine_kernel<<<blocks, kCombineThreads, 0, s>>>(kind, pass, part, nch, zy, labels,
                                                     ignore_index, N, V, loss_tok, alpha_tok,
-                                                    stats, blk_sum, blk_cnt, status);
+                                                    stats, blk_sum, blk_cnt, status, row0, ldN);
   return cudaGetLastError();
 }
 
@@ -1653,6 +1684,160 @@ cudaError_t launch_combo_finalize(const double* blk_sums, const long long* blk_c
                                   float* loss_mean, cudaStream_t s) {
   combo_finalize_kernel<<<1, 256, 0, s>>>(blk_sums, blk_cnt, nblk, loss_sum, term_sum, n_valid,
                                           loss_mean);
+  return cudaGetLastError();
+}
+
+
+// ----------------------------------------------------------------------------------------
+// Fused forward + backward ("Backward pass": per token chunk, the logits, the loss and the
+// gradients; the chunk's logits are kept, as on the page, instead of recomputed): kernels
+// that read the chunk's stored fp32 logits.  Memory-bound, one CTA per row, float4 loads.
+// ----------------------------------------------------------------------------------------
+__device__ __forceinline__ void block_sum2(float& a, float& b) {
+  __shared__ float sa[32], sb[32];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    a += __shfl_down_sync(0xffffffffu, a, o);
+    b += __shfl_down_sync(0xffffffffu, b, o);
+  }
+  const int w = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0) {
+    sa[w] = a;
+    sb[w] = b;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float ta = 0.f, tb = 0.f;
+    for (int i = 0; i < static_cast<int>(blockDim.x >> 5); ++i) {
+      ta += sa[i];
+      tb += sb[i];
+    }
+    a = ta;
+    b = tb;
+  }
+}
+
+__global__ void __launch_bounds__(1024)
+    count_valid_kernel(const int32_t* __restrict__ labels, int32_t ignore_index, int64_t N,
+                       int64_t V, int check_range, int64_t* n_valid) {
+  __shared__ long long sc[32];
+  long long c = 0;
+  for (int64_t i = threadIdx.x; i < N; i += blockDim.x) {
+    bool valid = true;
+    if (labels) {
+      const int32_t y = labels[i];
+      valid = y != ignore_index && (!check_range || (y >= 0 && y < V));
+    }
+    c += valid ? 1 : 0;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) c += __shfl_down_sync(0xffffffffu, c, o);
+  if ((threadIdx.x & 31) == 0) sc[threadIdx.x >> 5] = c;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    long long t = 0;
+    for (int i = 0; i < static_cast<int>(blockDim.x >> 5); ++i) t += sc[i];
+    *n_valid = static_cast<int64_t>(t);
+  }
+}
+
+// alpha = sum min(p, q) and S = sum_{q<p} q, or the JSD halves jp, jq, of one row.
+__global__ void __launch_bounds__(256)
+    logits_pass2_kernel(int kind, const float* __restrict__ lq, const float* __restrict__ lp,
+                        int64_t ldl, const float* __restrict__ stats, int64_t row0, int64_t ldN,
+                        int64_t rows, int64_t V, float* part) {
+  const int64_t r = blockIdx.x;
+  if (r >= rows) return;
+  const int64_t gn = row0 + r;
+  const float Lq = stats[gn], Lp = stats[ldN + gn];
+  const float lq2 = Lq * kLog2e, lp2 = Lp * kLog2e;
+  const float* rq = lq + r * ldl;
+  const float* rp = lp + r * ldl;
+  float a = 0.f, b = 0.f;
+  for (int64_t c = static_cast<int64_t>(threadIdx.x) * 4; c < V; c += 4 * blockDim.x) {
+    const float4 q4 = *reinterpret_cast<const float4*>(rq + c);
+    const float4 p4 = *reinterpret_cast<const float4*>(rp + c);
+    const float zq[4] = {q4.x, q4.y, q4.z, q4.w};
+    const float zp[4] = {p4.x, p4.y, p4.z, p4.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (c + j >= V) break;
+      const float qv = exp2f(fmaf(zq[j], kLog2e, -lq2));
+      const float pv = exp2f(fmaf(zp[j], kLog2e, -lp2));
+      if (kind == kJSD) {
+        const float ms = pv + qv;
+        if (ms > 0.f) {
+          const float lm = log2f(0.5f * ms) * kLn2;
+          a = fmaf(pv, (zp[j] - Lp) - lm, a);
+          b = fmaf(qv, (zq[j] - Lq) - lm, b);
+        }
+      } else {
+        a += fminf(pv, qv);
+        b += (qv < pv) ? qv : 0.f;
+      }
+    }
+  }
+  block_sum2(a, b);
+  if (threadIdx.x == 0) {
+    part[r] = a;
+    part[rows + r] = b;
+  }
+}
+
+template <bool DUAL>
+__global__ void __launch_bounds__(256)
+    logits_dz_kernel(const DzParams p, const float* __restrict__ lq,
+                     const float* __restrict__ lp, int64_t ldl) {
+  const int64_t r = blockIdx.x;
+  EpiDz<DUAL> e;
+  e.unit_begin(p, 0, static_cast<int>(r));
+  if (!e.row_ok) return;
+  const float* rq = lq + r * ldl;
+  const float* rp = DUAL ? lp + r * ldl : lq;
+  __nv_bfloat16* out = p.dz + r * p.ldz;
+  for (int64_t c = static_cast<int64_t>(threadIdx.x) * 32; c < p.V; c += 32 * blockDim.x) {
+    float vq[32], vp[32];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      if (c + 4 * k < p.V) {
+        const float4 a = *reinterpret_cast<const float4*>(rq + c + 4 * k);
+        vq[4 * k] = a.x, vq[4 * k + 1] = a.y, vq[4 * k + 2] = a.z, vq[4 * k + 3] = a.w;
+        if (DUAL) {
+          const float4 b = *reinterpret_cast<const float4*>(rp + c + 4 * k);
+          vp[4 * k] = b.x, vp[4 * k + 1] = b.y, vp[4 * k + 2] = b.z, vp[4 * k + 3] = b.w;
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) vq[4 * k + j] = vp[4 * k + j] = -INFINITY;
+      }
+    }
+    e.apply(vq, vp, c);
+    store_bf16_row32(out + c, vq, c, p.V);
+  }
+}
+
+cudaError_t launch_count_valid(const int32_t* labels, int32_t ignore_index, int64_t N,
+                               int64_t V, int check_range, int64_t* n_valid, cudaStream_t s) {
+  count_valid_kernel<<<1, 1024, 0, s>>>(labels, ignore_index, N, V, check_range, n_valid);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_logits_pass2(int kind, const float* lq, const float* lp, int64_t ldl,
+                                const float* stats, int64_t row0, int64_t ldN, int64_t rows,
+                                int64_t V, float* part, cudaStream_t s) {
+  if (rows <= 0) return cudaSuccess;
+  logits_pass2_kernel<<<static_cast<unsigned>(rows), 256, 0, s>>>(kind, lq, lp, ldl, stats, row0,
+                                                                  ldN, rows, V, part);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_logits_dz(const DzParams& p, const float* lq, const float* lp, int64_t ldl,
+                             cudaStream_t s) {
+  if (p.rows <= 0) return cudaSuccess;
+  if (p.kind == kCE)
+    logits_dz_kernel<false><<<static_cast<unsigned>(p.rows), 256, 0, s>>>(p, lq, lp, ldl);
+  else
+    logits_dz_kernel<true><<<static_cast<unsigned>(p.rows), 256, 0, s>>>(p, lq, lp, ldl);
   return cudaGetLastError();
 }
 

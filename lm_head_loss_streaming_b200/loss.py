@@ -193,6 +193,46 @@ def lm_head_loss_combo_bwd(fwd: ComboResult, hidden, weight, labels=None, target
     return dH, dW
 
 
+def lm_head_loss_fwd_bwd(kind, hidden, weight, labels=None, target_hidden=None,
+                        ignore_index=IGNORE_INDEX, grad_tok=None, grad_scale=None,
+                        chunk_tokens=0, workspace=None, out=None, dH=None, dW=None,
+                        accumulate_dW=False):
+    """Forward and backward in one call through ``slm_loss_fwd_bwd`` (the chunk's logits are
+    kept instead of recomputed).  Returns (FwdResult, dH, dW); the gradient is that of the
+    mean loss, scaled by grad_tok / grad_scale when given."""
+    k = _kind_id(kind)
+    _check_inputs(k, hidden, weight, labels, target_hidden)
+    N, d = hidden.shape
+    V = weight.shape[0]
+    dev = hidden.device
+    need = max(_lib.slm_fused_workspace_bytes(k, N, d, V, chunk_tokens), 256)
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    if out is None:
+        out = FwdResult(
+            k, torch.empty(1, dtype=torch.float32, device=dev),
+            torch.empty(1, dtype=torch.float64, device=dev),
+            torch.empty(1, dtype=torch.int64, device=dev),
+            torch.empty(N, dtype=torch.float32, device=dev),
+            torch.empty(N, dtype=torch.float32, device=dev) if k in _lib.ALPHA_KINDS else None,
+            torch.empty(_lib.slm_stats_floats(k), N, dtype=torch.float32, device=dev),
+            workspace)
+    else:
+        out.workspace = workspace
+    if dH is None:
+        dH = torch.empty(N, d, dtype=torch.bfloat16, device=dev)
+    if dW is None:
+        dW = torch.empty(V, d, dtype=torch.float32, device=dev)
+    st = _lib.slm_loss_fwd_bwd(k, _ptr(hidden), _ptr(target_hidden), _ptr(weight),
+                               _ptr(labels), ignore_index, N, d, V, _ptr(grad_tok),
+                               _ptr(grad_scale), _ptr(out.loss_tok), _ptr(out.alpha_tok),
+                               _ptr(out.loss_sum), _ptr(out.n_valid), _ptr(out.loss_mean),
+                               _ptr(out.stats), _ptr(dH), _ptr(dW), 1 if accumulate_dW else 0,
+                               chunk_tokens, _ptr(workspace), workspace.numel(), _stream())
+    _lib.check(st, "slm_loss_fwd_bwd")
+    return out, dH, dW
+
+
 def device_status(fwd: FwdResult):
     """Synchronise and return the device status of the last call on this workspace."""
     return _lib.slm_device_status(_ptr(fwd.workspace), _stream())

@@ -23,12 +23,12 @@ def _np64(t):
 
 
 def gpu_fwd_bwd(inp, kind=None, chunk_tokens=0, grad_tok=None, normalize=True,
-                accumulate_dW=None):
-    """Forward and backward through the C ABI on cuda:0.  Returns numpy results plus the
-    device status after each call."""
+                accumulate_dW=None, fused=False):
+    """Forward and backward through the C ABI on cuda:0 (two calls, or the fused single
+    call).  Returns numpy results plus the device status after each call."""
     from lm_head_loss_streaming_b200 import _lib
     from lm_head_loss_streaming_b200.loss import (device_status, lm_head_loss_bwd,
-                                                  lm_head_loss_fwd)
+                                                  lm_head_loss_fwd, lm_head_loss_fwd_bwd)
 
     kind = kind or inp.kind
     dev = torch.device("cuda", 0)
@@ -36,19 +36,26 @@ def gpu_fwd_bwd(inp, kind=None, chunk_tokens=0, grad_tok=None, normalize=True,
     W = inp.W.to(dev)
     Hp = inp.Hp.to(dev) if (kind != "ce" and inp.Hp is not None) else None
     labels = inp.labels.to(dev) if inp.labels is not None else None
-    fwd = lm_head_loss_fwd(kind, Hq, W, labels, Hp, inp.ignore_index,
-                           chunk_tokens=chunk_tokens)
-    st_fwd = device_status(fwd)
     gt = None
     if grad_tok is not None:
         gt = torch.as_tensor(grad_tok, dtype=torch.float32).to(dev).contiguous()
     dW = None
     if accumulate_dW is not None:
         dW = torch.as_tensor(accumulate_dW, dtype=torch.float32).to(dev).contiguous()
-    dH, dW = lm_head_loss_bwd(fwd, Hq, W, labels, Hp, inp.ignore_index, grad_tok=gt,
-                              normalize=normalize, chunk_tokens=chunk_tokens, dW=dW,
-                              accumulate_dW=accumulate_dW is not None)
-    st_bwd = device_status(fwd)
+    if fused:
+        assert normalize, "the fused call always divides by the valid count"
+        fwd, dH, dW = lm_head_loss_fwd_bwd(kind, Hq, W, labels, Hp, inp.ignore_index,
+                                           grad_tok=gt, chunk_tokens=chunk_tokens, dW=dW,
+                                           accumulate_dW=accumulate_dW is not None)
+        st_fwd = st_bwd = device_status(fwd)
+    else:
+        fwd = lm_head_loss_fwd(kind, Hq, W, labels, Hp, inp.ignore_index,
+                               chunk_tokens=chunk_tokens)
+        st_fwd = device_status(fwd)
+        dH, dW = lm_head_loss_bwd(fwd, Hq, W, labels, Hp, inp.ignore_index, grad_tok=gt,
+                                  normalize=normalize, chunk_tokens=chunk_tokens, dW=dW,
+                                  accumulate_dW=accumulate_dW is not None)
+        st_bwd = device_status(fwd)
     torch.cuda.synchronize()
     out = dict(
         loss_tok=_np64(fwd.loss_tok), loss_mean=float(fwd.loss_mean.item()),

@@ -17,11 +17,11 @@ pytestmark = pytest.mark.gpu
 KINDS = ["ce", "kl_div", "tv", "nla", "lk_hybrid", "rkl", "jsd", "ce_argmax_p"]
 
 
-def _compare_argmax(inp, chunk_tokens=0, what=""):
+def _compare_argmax(inp, chunk_tokens=0, what="", fused=False):
     """CE against argmax p: the targets are an argmax decided in fp32 on the GPU.  Check
     they are valid argmaxes of the float64 target logits, then compare the loss and the
     gradients with the oracle's hard-label CE on the GPU's targets."""
-    g = gpu_fwd_bwd(inp, "ce_argmax_p", chunk_tokens=chunk_tokens)
+    g = gpu_fwd_bwd(inp, "ce_argmax_p", chunk_tokens=chunk_tokens, fused=fused)
     assert g["st_fwd"] == 0 and g["st_bwd"] == 0, (g["st_fwd"], g["st_bwd"])
     y = g["stats32"][1].view(np.int32)
     assert argmax_targets_valid(inp, y) <= 0.01, what
@@ -34,10 +34,10 @@ def _compare_argmax(inp, chunk_tokens=0, what=""):
     return g, r
 
 
-def _compare(inp, kind, chunk_tokens=0, what=""):
+def _compare(inp, kind, chunk_tokens=0, what="", fused=False):
     if kind == "ce_argmax_p":
-        return _compare_argmax(inp, chunk_tokens, what)
-    g = gpu_fwd_bwd(inp, kind, chunk_tokens=chunk_tokens)
+        return _compare_argmax(inp, chunk_tokens, what, fused)
+    g = gpu_fwd_bwd(inp, kind, chunk_tokens=chunk_tokens, fused=fused)
     r = oracle_fwd_bwd(inp, kind)
     assert g["st_fwd"] == 0 and g["st_bwd"] == 0, (g["st_fwd"], g["st_bwd"])
     assert g["n_valid"] == r["n_valid"]
