@@ -113,6 +113,16 @@ struct PairCfg {
   static_assert(kSmem <= 232448, "shared memory per CTA");
 };
 
+// Bytes of shared staging per epilogue warp an epilogue asks for (kStageBytesPerWarp).
+template <class E, class = void>
+struct EpiStageBytes {
+  static constexpr int value = 0;
+};
+template <class E>
+struct EpiStageBytes<E, decltype(void(E::kStageBytesPerWarp))> {
+  static constexpr int value = E::kStageBytesPerWarp;
+};
+
 template <int BNI, int NSUB, int NUM_A, int NBUF, int NWG, bool A_MN, bool B_MN, int STAGES,
           class Epi>
 __global__ void __launch_bounds__(64 + 128 * NWG, 1)
@@ -300,6 +310,12 @@ __global__ void __launch_bounds__(64 + 128 * NWG, 1)
     const uint32_t tempty_leader0 = mapa_shared(smem_u32(&pc->tempty[0]), 0);
     const uint32_t tempty_leader1 = mapa_shared(smem_u32(&pc->tempty[1]), 0);
     Epi epi;
+    if constexpr (EpiStageBytes<Epi>::value > 0) {
+      // Per-warp staging buffers live after the control block.
+      uint8_t* st = reinterpret_cast<uint8_t*>(
+          (reinterpret_cast<uintptr_t>(pc + 1) + 127) & ~static_cast<uintptr_t>(127));
+      epi.stage = reinterpret_cast<float*>(st + (warp - 2) * EpiStageBytes<Epi>::value);
+    }
     uint32_t t = 0;
     bool ok = true;
     for (int u = pair; ok && u < g.num_units; u += npairs) {
@@ -359,15 +375,30 @@ __device__ __forceinline__ void mask_tail(float (&v)[32], int64_t col0, int64_t 
     if (col0 + i >= V) v[i] = -INFINITY;
 }
 
-// Fused path: store 32 fp32 logits of one row (columns >= V land in the row padding; the
-// leading dimension is V rounded up to 4, so every float4 that starts below V fits).
-__device__ __forceinline__ void store_f32_row32(float* dst, const float (&v)[32], int64_t col0,
-                                                int64_t V) {
+// Fused path: store the warp's 32 rows x 32 columns of fp32 logits (each lane holds its
+// row's 32 values).  The block goes through the warp's 4 KB staging buffer with the 16-byte
+// chunk index XOR-swizzled by the row (conflict-free writes and reads), so that each global
+// store instruction writes four full 128-byte row segments instead of 32 scattered pieces.
+// Columns >= V land in the row padding (the leading dimension is V rounded up to 4, so every
+// float4 that starts below V fits).  Warp-collective.
+__device__ __forceinline__ void store_block32_f32(float* stage, const float (&v)[32],
+                                                  float* gdst, int64_t ldl, int nrows,
+                                                  int64_t col0, int64_t V) {
+  const int lane = threadIdx.x & 31;
+  float4* srow = reinterpret_cast<float4*>(stage + lane * 32);
 #pragma unroll
   for (int k = 0; k < 8; ++k)
-    if (col0 + 4 * k < V)
-      reinterpret_cast<float4*>(dst)[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2],
-                                                      v[4 * k + 3]);
+    srow[k ^ (lane & 7)] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+  __syncwarp();
+  const int k = lane & 7;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int r = i * 4 + (lane >> 3);
+    const float4 x = reinterpret_cast<const float4*>(stage + r * 32)[k ^ (r & 7)];
+    if (r < nrows && col0 + 4 * k < V)
+      *reinterpret_cast<float4*>(gdst + static_cast<int64_t>(r) * ldl + 4 * k) = x;
+  }
+  __syncwarp();
 }
 
 // CE forward: per row, online max m (log2 units) and s = sum 2^(z log2e - m) over the
@@ -375,6 +406,8 @@ __device__ __forceinline__ void store_f32_row32(float* dst, const float (&v)[32]
 // label falls there.
 struct EpiFwdCE {
   using Params = FwdParams;
+  static constexpr int kStageBytesPerWarp = 4096;
+  float* stage;  // this warp's staging buffer (fused path stores)
   float m, s, zyv;
   int32_t lab;
   bool has_zy, row_ok;
@@ -400,7 +433,7 @@ struct EpiFwdCE {
       tmem_ld32(tb + c, v);
       tmem_ld_wait();
       if (n0 + c + 32 > p.V) mask_tail(v, n0 + c, p.V);
-      if (p.lq_out && row_ok) store_f32_row32(p.lq_out + grow * p.ldl + n0 + c, v, n0 + c, p.V);
+      if (p.lq_out) store_rows(p, p.lq_out, v, n0 + c);
       if (static_cast<uint64_t>(rel - c) < 32u) {
         const int o = static_cast<int>(rel - c);
 #pragma unroll
@@ -425,6 +458,9 @@ struct EpiFwdCE {
     }
   }
 
+  __device__ __forceinline__ void store_rows(const Params& p, float* buf, const float (&v)[32],
+                                             int64_t col0) const;
+
   __device__ __forceinline__ void unit_end(const Params& p, int, int slot, int) {
     if (!row_ok) return;
     p.part[(static_cast<int64_t>(slot) * 2 + 0) * p.N + grow] = m;
@@ -433,12 +469,31 @@ struct EpiFwdCE {
   }
 };
 
+// The rows of a warp are consecutive: lane 0 holds row grow - lane.  Store the warp's
+// 32 x 32 block of one logits buffer at columns [col0, col0 + 32).
+template <class E>
+__device__ __forceinline__ void epi_store_rows(const E& e, const FwdParams& p, float* buf,
+                                               const float (&v)[32], int64_t col0) {
+  const int lane = threadIdx.x & 31;
+  const int64_t r0 = e.grow - lane;
+  const int64_t left = p.N - r0;
+  const int nrows = left < 32 ? static_cast<int>(left) : 32;
+  store_block32_f32(e.stage, v, buf + r0 * p.ldl + col0, p.ldl, nrows, col0, p.V);
+}
+
+__device__ __forceinline__ void EpiFwdCE::store_rows(const Params& p, float* buf,
+                                                     const float (&v)[32], int64_t col0) const {
+  epi_store_rows(*this, p, buf, v, col0);
+}
+
 // KL / RKL forward (and the first pass of the alpha losses and of JSD): per row and for
 // both the draft (q, accumulator 0) and the target (p, accumulator 1): online max and sum
 // of exp; plus A = sum_v 2^(z_p log2e - m_p) (z_p - z_q), rescaled whenever m_p grows, and
 // B = sum_v 2^(z_q log2e - m_q) (z_q - z_p), rescaled whenever m_q grows.
 struct EpiFwdDual {
   using Params = FwdParams;
+  static constexpr int kStageBytesPerWarp = 4096;
+  float* stage;  // this warp's staging buffer (fused path stores)
   float mq, sq, mp, sp, A, B;
   bool row_ok;
   int64_t grow;
@@ -499,9 +554,9 @@ struct EpiFwdDual {
         mask_tail(vq, n0 + c, p.V);
         mask_tail(vp, n0 + c, p.V);
       }
-      if (p.lq_out && row_ok) {
-        store_f32_row32(p.lq_out + grow * p.ldl + n0 + c, vq, n0 + c, p.V);
-        store_f32_row32(p.lp_out + grow * p.ldl + n0 + c, vp, n0 + c, p.V);
+      if (p.lq_out) {
+        epi_store_rows(*this, p, p.lq_out, vq, n0 + c);
+        epi_store_rows(*this, p, p.lp_out, vp, n0 + c);
       }
       if (tail)
         chunk<true>(vq, vp);
@@ -528,6 +583,8 @@ struct EpiFwdDual {
 // replaces), with the draft logit at that column.
 struct EpiFwdArgmax {
   using Params = FwdParams;
+  static constexpr int kStageBytesPerWarp = 4096;
+  float* stage;  // this warp's staging buffer (fused path stores)
   float mq, sq, pmax, zqa;
   int pidx;
   bool row_ok;
@@ -554,7 +611,7 @@ struct EpiFwdArgmax {
         mask_tail(vq, n0 + c, p.V);
         mask_tail(vp, n0 + c, p.V);
       }
-      if (p.lq_out && row_ok) store_f32_row32(p.lq_out + grow * p.ldl + n0 + c, vq, n0 + c, p.V);
+      if (p.lq_out) epi_store_rows(*this, p, p.lq_out, vq, n0 + c);
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
         if (vp[i] > pmax) {
@@ -1162,9 +1219,12 @@ static cudaError_t launch_pair(const CUtensorMap& a0, const CUtensorMap& a1,
                                const CUtensorMap& b, const GemmGeom& g,
                                const typename Epi::Params& p, const DevCtl& c, cudaStream_t s) {
   using Cfg = PairCfg<BNI, NSUB, NUM_A, NBUF, NWG, A_MN, B_MN, STAGES>;
+  constexpr size_t kStage = EpiStageBytes<Epi>::value;
+  constexpr size_t kSmem = Cfg::kSmem + (kStage ? 128 + kStage * 4 * NWG : 0);
+  static_assert(kSmem <= 232448, "shared memory per CTA");
   auto kern = gemm_pair_kernel<BNI, NSUB, NUM_A, NBUF, NWG, A_MN, B_MN, STAGES, Epi>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(Cfg::kSmem));
+                                       static_cast<int>(kSmem));
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
@@ -1173,7 +1233,7 @@ static cudaError_t launch_pair(const CUtensorMap& a0, const CUtensorMap& a1,
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.blockDim = dim3(Cfg::kThreads, 1, 1);
-  cfg.dynamicSmemBytes = Cfg::kSmem;
+  cfg.dynamicSmemBytes = kSmem;
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
