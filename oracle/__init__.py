@@ -20,6 +20,8 @@ from .slm_oracle import (  # noqa: F401
     loss_and_grads,
     combo_forward,
     combo_backward,
+    align_labels,
+    flatness,
     logits_bytes,
     chunk_buffer_bytes,
 )

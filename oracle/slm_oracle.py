@@ -21,6 +21,8 @@ Sources, cited by page title and section:
        chunk buffer arithmetic chunk x vocab x dtype x 2.
      - Gradient-accumulation and streaming normalisation equations: normalise by the
        number of valid, non-masked tokens, never by the number of chunks.
+[FT] "Flatter Tokens are More Valuable for Speculative Draft Model Training" (summary):
+     flatness of a token = cosine similarity of the target distribution to uniform.
 [LF] "Loss Functions" (speculators user guide), table "Available Losses": p is the
      target distribution, q the draft distribution, alpha = sum_v min(p_v, q_v);
      kl_div = forward KL target->draft, rkl = reverse KL, jsd = Jensen-Shannon,
@@ -352,3 +354,44 @@ def combo_backward(weights, Hq, W, labels=None, Hp=None, grad_tok=None, ignore_i
         dH += float(w) * h
         dW += float(w) * g
     return dH, dW
+
+
+# ----------------------------------------------------------------------------------------
+# Draft-head helpers either side of the path.
+# [SD] "Correctness: alignment before chunking": hidden states, targets and masks are
+# aligned for the objective first (for draft heads the target shift depends on the head),
+# masks applied, and only then split into chunks.
+# [FT] "Flatter Tokens are More Valuable for Speculative Draft Model Training": a token's
+# flatness is the cosine similarity of the target distribution to the uniform one.
+# ----------------------------------------------------------------------------------------
+def align_labels(tokens, shift, loss_mask=None, seq_ids=None, ignore_index=-100):
+    """Labels for a head that predicts the token ``shift`` positions ahead.
+
+    tokens [B, S] int; loss_mask [B, S] (nonzero = the token may be a target) or None;
+    seq_ids [B, S] (packed sequences: position t may only target a token of the same
+    sequence) or None.  Returns int64 [B, S]: tokens[b, t + shift] where t + shift < S, the
+    target position is unmasked and in the same sequence; ignore_index elsewhere.
+    Written as a plain loop over positions."""
+    tok = np.asarray(tokens)
+    B, S = tok.shape
+    out = np.full((B, S), ignore_index, dtype=np.int64)
+    for b in range(B):
+        for t in range(S):
+            u = t + shift
+            if u >= S:
+                continue
+            if loss_mask is not None and not np.asarray(loss_mask)[b, u]:
+                continue
+            if seq_ids is not None and np.asarray(seq_ids)[b, u] != np.asarray(seq_ids)[b, t]:
+                continue
+            out[b, t] = tok[b, u]
+    return out
+
+
+def flatness(zp):
+    """Cosine similarity of softmax(zp) (per row) to the uniform distribution:
+    <p, u> / (||p|| ||u||) with u = 1/V, which equals 1 / (sqrt(V) ||p||_2)."""
+    p = np.exp(log_softmax(zp))
+    V = p.shape[1]
+    u = np.full(V, 1.0 / V)
+    return (p @ u) / (np.linalg.norm(p, axis=1) * np.linalg.norm(u))

@@ -439,3 +439,49 @@ def test_combination_against_torch_autograd():
         for k in weights:
             assert np.allclose(out["terms"][k]["loss_tok"],
                                orc.forward(k, Hq, W, y, Hp)["loss_tok"], atol=0)
+
+
+# --------------------------------------------------------------------------------------
+# Draft-head helpers: alignment before chunking, and flatness.
+# --------------------------------------------------------------------------------------
+def test_align_labels_worked_examples():
+    tok = np.array([[10, 11, 12, 13, 14, 15]])
+    # Standard next-token targets (shift 1): the last position has none.
+    assert orc.align_labels(tok, 1).tolist() == [[11, 12, 13, 14, 15, -100]]
+    # A draft head two tokens ahead.
+    assert orc.align_labels(tok, 2).tolist() == [[12, 13, 14, 15, -100, -100]]
+    # Packed sequences [10 11 12 | 13 14 15]: targets never cross the boundary.
+    seq = np.array([[0, 0, 0, 1, 1, 1]])
+    assert orc.align_labels(tok, 1, seq_ids=seq).tolist() == [[11, 12, -100, 14, 15, -100]]
+    assert orc.align_labels(tok, 2, seq_ids=seq).tolist() == [[12, -100, -100, 15, -100, -100]]
+    # A loss mask on the target positions (e.g. only the answer tokens count).
+    mask = np.array([[0, 0, 1, 1, 0, 1]])
+    assert orc.align_labels(tok, 1, loss_mask=mask).tolist() == [[-100, 12, 13, -100, 15, -100]]
+
+
+def test_align_then_chunk_equals_dense():
+    # Aligning before chunking keeps the streaming loss equal to the dense one ([SD]).
+    rng = np.random.default_rng(70)
+    B, S, d, V = 3, 17, 8, 29
+    tok = rng.integers(0, V, (B, S))
+    seq = np.cumsum(rng.random((B, S)) < 0.2, axis=1)
+    lab = orc.align_labels(tok, 2, seq_ids=seq).reshape(-1)
+    H = rng.standard_normal((B * S, d))
+    W = 0.5 * rng.standard_normal((V, d))
+    dense = F.cross_entropy(torch.tensor(H @ W.T), torch.tensor(lab), ignore_index=-100)
+    for cs in (1, 5, 51):
+        assert abs(orc.forward("ce", H, W, lab, chunk_size=cs)["loss"] - dense.item()) < 1e-12
+
+
+def test_flatness_closed_forms_and_scipy():
+    from scipy.spatial.distance import cosine
+    V = 37
+    assert np.allclose(orc.flatness(np.zeros((2, V))), 1.0)           # uniform p
+    z = np.zeros((1, V)); z[0, 5] = 800.0                               # one-hot p
+    assert np.allclose(orc.flatness(z), 1.0 / math.sqrt(V))
+    rng = np.random.default_rng(71)
+    z = rng.standard_normal((4, V)) * 2
+    p = np.exp(orc.log_softmax(z))
+    ref = [1.0 - cosine(p[i], np.full(V, 1.0 / V)) for i in range(4)]
+    assert np.allclose(orc.flatness(z), ref, atol=1e-12)
+    assert np.allclose(orc.flatness(z), 1.0 / (math.sqrt(V) * np.linalg.norm(p, axis=1)))
