@@ -29,8 +29,15 @@ namespace slm {
 namespace {
 
 constexpr size_t kAlign = 256;
-constexpr int kPairM = 2 * kBM;   // M rows of one 2-SM tile
-constexpr int kGroupPairs = 8;    // pair M tiles per raster group (2048 token rows)
+#ifndef SLM_GROUP_PAIRS
+#define SLM_GROUP_PAIRS 8
+#endif
+#ifndef SLM_MAX_RUNS
+#define SLM_MAX_RUNS 32
+#endif
+constexpr int kPairM = 2 * kBM;                // M rows of one 2-SM tile
+constexpr int kGroupPairs = SLM_GROUP_PAIRS;   // pair M tiles per raster group
+constexpr int kMaxRuns = SLM_MAX_RUNS;         // vocabulary runs per row, at most
 constexpr long long kTimeoutCycles = 4000000000LL;  // ~2 s at the B200's boost clock
 
 // Test hooks set through slm_debug_set (process-wide, read at every launch).
@@ -52,7 +59,7 @@ bool two_pass_kind(int k) {
   return k == SLM_TV || k == SLM_NLA || k == SLM_LK_HYBRID || k == SLM_JSD;
 }
 
-// Forward vocabulary schedule: tiles of `bn` columns, grouped into at most 32 runs per row
+// Forward vocabulary schedule: tiles of `bn` columns, grouped into at most kMaxRuns runs per row
 // (so the per-row partials stay O(N)), each run at least 2048 columns long.  Each run
 // leaves kFwdPartsPerRun partial slots per row (one per epilogue warpgroup).
 struct FwdSched {
@@ -63,8 +70,8 @@ FwdSched fwd_sched(int kind, int64_t V) {
   FwdSched f;
   f.bn = dual_kind(kind) ? kTileDual : kTileCE;
   f.num_n = static_cast<int>(ceil_div(V, f.bn));
-  const int min_vc = 2048 / f.bn;
-  f.vc = std::max<int>(min_vc, static_cast<int>(ceil_div(f.num_n, 32)));
+  const int min_vc = std::max(1, 2048 / f.bn);
+  f.vc = std::max<int>(min_vc, static_cast<int>(ceil_div(f.num_n, kMaxRuns)));
   f.vc = std::min(f.vc, f.num_n);
   f.units_n = static_cast<int>(ceil_div(f.num_n, f.vc));
   f.slots = f.units_n * kFwdPartsPerRun;
