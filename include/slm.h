@@ -226,6 +226,36 @@ SLM_API int slm_combo_bwd(const float* weights, const void* Hq, const void* Hp, 
                           int accumulate_dW, int64_t chunk_tokens, void* workspace,
                           size_t ws_bytes, void* stream);
 
+/* ---------------------------------------------------------------------------------------
+ * Draft-head helpers either side of the path.
+ * ------------------------------------------------------------------------------------- */
+/* Target alignment before chunking ("Training speculative decoders: ...", section
+ * "Correctness: alignment before chunking": hidden states, targets and masks are aligned
+ * for the objective first, masks applied, and only then split into chunks; each draft head
+ * may predict a different future token, so the target shift depends on the head).
+ *   tokens     int32 [B, S] token ids (device).
+ *   loss_mask  uint8 [B, S] or NULL: 0 = this position may not be a target.
+ *   seq_ids    int32 [B, S] or NULL: packed-sequence id of each position; a target never
+ *              crosses into another sequence.
+ *   shift      >= 0: the head predicts the token `shift` positions ahead (1 = next token).
+ *   labels     int32 [B, S] out: tokens[b, t + shift] where t + shift < S and the target is
+ *              unmasked and in the same sequence, else ignore_index.
+ * Integer work, exact.  Returns SLM_ERR_SHAPE for negative sizes or shift. */
+SLM_API int slm_align_labels(const int32_t* tokens, const uint8_t* loss_mask,
+                             const int32_t* seq_ids, int64_t B, int64_t S, int32_t shift,
+                             int32_t ignore_index, int32_t* labels, void* stream);
+
+/* Per-token flatness of the target distribution p = softmax(H_p W^T) ("Flatter Tokens are
+ * More Valuable for Speculative Draft Model Training": the cosine similarity of the target
+ * distribution to the uniform one), which equals 1 / (sqrt(V) ||p||_2): 1 for a uniform p,
+ * 1/sqrt(V) for a one-hot p.  One vocabulary-tiled GEMM pass over H_p with an online
+ * sum of e^(2 (z - m)) in the epilogue; the logits are never stored.
+ *   Hp    bf16 [N, d];  W bf16 [V, d];  flat  float [N] out.
+ *   workspace  at least slm_flatness_workspace_bytes(N, d, V) bytes. */
+SLM_API size_t slm_flatness_workspace_bytes(int64_t N, int64_t d, int64_t V);
+SLM_API int slm_target_flatness(const void* Hp, const void* W, int64_t N, int64_t d, int64_t V,
+                                float* flat, void* workspace, size_t ws_bytes, void* stream);
+
 /* Test hook for the device-side failure path (not for production use).  fault_mode 1 makes
  * every following launch withhold one internal pipeline release, so that a bounded wait in
  * the kernel runs out: the kernel then records SLM_ERR_TIMEOUT in the workspace status word,

@@ -50,6 +50,9 @@ SIGNATURES = {
     "slm_loss_fwd_bwd": (_INT, [_INT, _P, _P, _P, _P, _I32, _I64, _I64, _I64, _P, _P,
                                 _P, _P, _P, _P, _P, _P, _P, _P, _INT, _I64, _P, _SZ, _P]),
     "slm_combo_workspace_bytes": (_SZ, [_I64, _I64, _I64, _I64]),
+    "slm_align_labels": (_INT, [_P, _P, _P, _I64, _I64, _I32, _I32, _P, _P]),
+    "slm_flatness_workspace_bytes": (_SZ, [_I64, _I64, _I64]),
+    "slm_target_flatness": (_INT, [_P, _P, _I64, _I64, _I64, _P, _P, _SZ, _P]),
     "slm_combo_fwd": (_INT, [_P, _P, _P, _P, _P, _I32, _I64, _I64, _I64,
                              _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "slm_combo_bwd": (_INT, [_P, _P, _P, _P, _P, _I32, _I64, _I64, _I64,
@@ -193,3 +196,17 @@ def slm_loss_fwd_bwd(kind, Hq, Hp, W, labels, ignore_index, N, d, V, grad_tok, g
                                    loss_sum, n_valid, loss_mean, stats, dHq, dW,
                                    int(accumulate_dW), int(chunk_tokens), workspace,
                                    int(ws_bytes), stream)
+
+
+def slm_align_labels(tokens, loss_mask, seq_ids, B, S, shift, ignore_index, labels, stream):
+    return load().slm_align_labels(tokens, loss_mask, seq_ids, int(B), int(S), int(shift),
+                                   int(ignore_index), labels, stream)
+
+
+def slm_flatness_workspace_bytes(N, d, V):
+    return load().slm_flatness_workspace_bytes(int(N), int(d), int(V))
+
+
+def slm_target_flatness(Hp, W, N, d, V, flat, workspace, ws_bytes, stream):
+    return load().slm_target_flatness(Hp, W, int(N), int(d), int(V), flat, workspace,
+                                      int(ws_bytes), stream)

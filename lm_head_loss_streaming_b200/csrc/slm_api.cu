@@ -490,6 +490,55 @@ int slm_loss_bwd(int kind, const void* Hq, const void* Hp, const void* W, const 
   return SLM_OK;
 }
 
+int slm_align_labels(const int32_t* tokens, const uint8_t* loss_mask, const int32_t* seq_ids,
+                     int64_t B, int64_t S, int32_t shift, int32_t ignore_index,
+                     int32_t* labels, void* stream) {
+  if (B < 0 || S < 0 || shift < 0 || B * S >= (int64_t(1) << 40)) return SLM_ERR_SHAPE;
+  if (B * S == 0) return SLM_OK;
+  if (!tokens || !labels) return SLM_ERR_NULL;
+  int st = check_device();
+  if (st != SLM_OK) return st;
+  SLM_TRY_CUDA(launch_align_labels(tokens, loss_mask, seq_ids, B, S, shift, ignore_index, labels,
+                                   static_cast<cudaStream_t>(stream)));
+  return SLM_OK;
+}
+
+size_t slm_flatness_workspace_bytes(int64_t N, int64_t d, int64_t V) {
+  if (N < 0 || d <= 0 || V <= 0 || (d % 8) != 0) return 0;
+  const FwdSched f = fwd_sched(SLM_CE, V);
+  return kAlign + align_up(static_cast<size_t>(f.slots) * kFlatFields *
+                               static_cast<size_t>(std::max<int64_t>(N, 1)) * 4,
+                           kAlign);
+}
+
+int slm_target_flatness(const void* Hp, const void* W, int64_t N, int64_t d, int64_t V,
+                        float* flat, void* workspace, size_t ws_bytes, void* stream) {
+  if (N < 0 || d <= 0 || V <= 0 || (d % 8) != 0) return SLM_ERR_SHAPE;
+  if (N >= (int64_t(1) << 31) || V >= (int64_t(1) << 31)) return SLM_ERR_SHAPE;
+  if (N == 0) return SLM_OK;
+  if (!Hp || !W || !flat || !workspace) return SLM_ERR_NULL;
+  if (misaligned(Hp, 16) || misaligned(W, 16)) return SLM_ERR_ALIGN;
+  if (misaligned(workspace, kAlign) || ws_bytes < slm_flatness_workspace_bytes(N, d, V))
+    return SLM_ERR_WORKSPACE;
+  int st = check_device();
+  if (st != SLM_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int* status = reinterpret_cast<int*>(ws);
+  float* part = reinterpret_cast<float*>(ws + kAlign);
+  SLM_TRY_CUDA(cudaMemsetAsync(status, 0, sizeof(int), s));
+  const DevCtl ctl = make_ctl(status);
+  const FwdSched f = fwd_sched(SLM_CE, V);
+  const GemmGeom g = geom(N, V, d, f.bn, f.vc, kGroupPairs, kPairM);
+  CUtensorMap tHp, tW;
+  if (!make_map(&tHp, Hp, d, N, d, kBK, kBM)) return SLM_ERR_CUDA;
+  if (!make_map(&tW, W, d, V, d, kBK, 128)) return SLM_ERR_CUDA;
+  FwdParams p{nullptr, 0, N, V, part, nullptr, nullptr, 0, nullptr, nullptr, 0};
+  SLM_TRY_CUDA(launch_fwd_flat(tHp, tW, g, p, ctl, s));
+  SLM_TRY_CUDA(launch_flat_combine(part, f.slots, N, V, flat, s));
+  return SLM_OK;
+}
+
 size_t slm_fused_workspace_bytes(int kind, int64_t N, int64_t d, int64_t V,
                                  int64_t chunk_tokens) {
   if (!valid_kind(kind) || N < 0 || d <= 0 || V <= 0 || (d % 8) != 0) return 0;

@@ -140,6 +140,16 @@ cudaError_t launch_logits_pass2(int kind, const float* lq, const float* lp, int6
 cudaError_t launch_logits_dz(const DzParams& p, const float* lq, const float* lp, int64_t ldl,
                              cudaStream_t s);
 
+// Draft-head helpers.
+constexpr int kFlatFields = 3;  // m, s, s2 = sum 2^(2 (z log2e - m))
+cudaError_t launch_align_labels(const int32_t* tokens, const uint8_t* loss_mask,
+                                const int32_t* seq_ids, int64_t B, int64_t S, int32_t shift,
+                                int32_t ignore_index, int32_t* labels, cudaStream_t s);
+cudaError_t launch_fwd_flat(const CUtensorMap& tHp, const CUtensorMap& tW, const GemmGeom& g,
+                            const FwdParams& p, const DevCtl& c, cudaStream_t s);
+cudaError_t launch_flat_combine(const float* part, int nch, int64_t N, int64_t V,
+                                float* flat, cudaStream_t s);
+
 // Weighted combinations.
 cudaError_t launch_fwd_union(const CUtensorMap& tHq, const CUtensorMap& tHp,
                              const CUtensorMap& tW, const GemmGeom& g, const FwdParams& p,

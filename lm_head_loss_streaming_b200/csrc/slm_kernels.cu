@@ -965,6 +965,60 @@ struct EpiDw {
 };
 
 // ----------------------------------------------------------------------------------------
+// Target flatness ("Flatter Tokens are More Valuable for Speculative Draft Model
+// Training"): cos(p, uniform) = 1 / (sqrt(V) ||p||_2).  Per row and vocabulary slot the
+// online max m, s = sum 2^(z log2e - m) and s2 = sum 2^(2 (z log2e - m)).
+// ----------------------------------------------------------------------------------------
+struct EpiFlat {
+  using Params = FwdParams;
+  float m, s, s2;
+  bool row_ok;
+  int64_t grow;
+
+  __device__ __forceinline__ void unit_begin(const Params& p, int row0, int row) {
+    m = -INFINITY;
+    s = s2 = 0.f;
+    grow = static_cast<int64_t>(row0) + row;
+    row_ok = grow < p.N;
+  }
+
+  template <int TN>
+  __device__ __forceinline__ void tile(const Params& p, uint32_t tb, int, int64_t n0, int c0,
+                                       int c1, int) {
+#pragma unroll 1
+    for (int c = c0; c < c1; c += 32) {
+      float v[32];
+      tmem_ld32(tb + c, v);
+      tmem_ld_wait();
+      if (n0 + c + 32 > p.V) mask_tail(v, n0 + c, p.V);
+      const float mx = max32(v) * kLog2e;
+      if (mx > m) {
+        const float r = exp2f(m - mx);
+        s *= r;
+        s2 *= r * r;
+        m = mx;
+      }
+      if (m != -INFINITY) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float e = exp2f(fmaf(v[i], kLog2e, -m));
+          s += e;
+          s2 = fmaf(e, e, s2);
+        }
+      }
+    }
+  }
+
+  __device__ __forceinline__ void unit_end(const Params& p, int, int slot, int) {
+    if (!row_ok) return;
+    float* base = p.part + static_cast<int64_t>(slot) * kFlatFields * p.N + grow;
+    base[0] = m;
+    base[p.N] = s;
+    base[2 * p.N] = s2;
+  }
+};
+
+// ----------------------------------------------------------------------------------------
 // Weighted combinations ("Loss Functions", "Weighted Combinations"): every term shares one
 // logit pass.  Pass 1 gathers the union of the one-pass statistics; pass 2 (only when a
 // term needs the final log-sum-exps) the union of alpha, S and the JSD halves; the
@@ -1275,6 +1329,10 @@ cudaError_t launch_fwd_argmax(const CUtensorMap& tHq, const CUtensorMap& tHp,
 cudaError_t launch_jsd(const CUtensorMap& tHq, const CUtensorMap& tHp, const CUtensorMap& tW,
                        const GemmGeom& g, const FwdParams& p, const DevCtl& c, cudaStream_t s) {
   return launch_pair<256, 1, 2, 1, 2, false, false, 4, EpiJsd>(tHq, tHp, tW, g, p, c, s);
+}
+cudaError_t launch_fwd_flat(const CUtensorMap& tHp, const CUtensorMap& tW, const GemmGeom& g,
+                            const FwdParams& p, const DevCtl& c, cudaStream_t s) {
+  return launch_pair<256, 2, 1, 1, 2, false, false, 4, EpiFlat>(tHp, tHp, tW, g, p, c, s);
 }
 cudaError_t launch_fwd_union(const CUtensorMap& tHq, const CUtensorMap& tHp,
                              const CUtensorMap& tW, const GemmGeom& g, const FwdParams& p,
@@ -1898,6 +1956,67 @@ cudaError_t launch_logits_dz(const DzParams& p, const float* lq, const float* lp
     logits_dz_kernel<false><<<static_cast<unsigned>(p.rows), 256, 0, s>>>(p, lq, lp, ldl);
   else
     logits_dz_kernel<true><<<static_cast<unsigned>(p.rows), 256, 0, s>>>(p, lq, lp, ldl);
+  return cudaGetLastError();
+}
+
+
+// ----------------------------------------------------------------------------------------
+// Alignment before chunking ("Correctness: alignment before chunking"): the label of
+// position t for a head that predicts `shift` tokens ahead is tokens[t + shift], unless the
+// target lies past the sequence, in another packed sequence, or under the loss mask.
+// ----------------------------------------------------------------------------------------
+__global__ void align_labels_kernel(const int32_t* __restrict__ tokens,
+                                    const uint8_t* __restrict__ loss_mask,
+                                    const int32_t* __restrict__ seq_ids, int64_t B, int64_t S,
+                                    int32_t shift, int32_t ignore_index, int32_t* labels) {
+  const int64_t n = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (n >= B * S) return;
+  const int64_t b = n / S;
+  const int64_t t = n - b * S;
+  const int64_t u = t + shift;
+  int32_t y = ignore_index;
+  if (u < S) {
+    const int64_t nu = b * S + u;
+    const bool masked = loss_mask && loss_mask[nu] == 0;
+    const bool crosses = seq_ids && seq_ids[nu] != seq_ids[n];
+    if (!masked && !crosses) y = tokens[nu];
+  }
+  labels[n] = y;
+}
+
+__global__ void __launch_bounds__(kCombineThreads)
+    flat_combine_kernel(const float* __restrict__ part, int nch, int64_t N, int64_t V,
+                        float* flat) {
+  const int64_t n = static_cast<int64_t>(blockIdx.x) * kCombineThreads + threadIdx.x;
+  if (n >= N) return;
+  float M = -INFINITY;
+  for (int j = 0; j < nch; ++j) M = fmaxf(M, part[(int64_t)j * kFlatFields * N + n]);
+  float S = 0.f, S2 = 0.f;
+  for (int j = 0; j < nch; ++j) {
+    const float* b = part + (int64_t)j * kFlatFields * N + n;
+    const float r = exp2f(b[0] - M);
+    S += b[N] * r;
+    S2 += b[2 * N] * (r * r);
+  }
+  // ||p||_2 = sqrt(S2) / S, so cos(p, uniform) = S / (sqrt(V) sqrt(S2)).
+  flat[n] = S / (sqrtf(static_cast<float>(V)) * sqrtf(S2));
+}
+
+cudaError_t launch_align_labels(const int32_t* tokens, const uint8_t* loss_mask,
+                                const int32_t* seq_ids, int64_t B, int64_t S, int32_t shift,
+                                int32_t ignore_index, int32_t* labels, cudaStream_t s) {
+  const int64_t n = B * S;
+  if (n <= 0) return cudaSuccess;
+  align_labels_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(
+      tokens, loss_mask, seq_ids, B, S, shift, ignore_index, labels);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_flat_combine(const float* part, int nch, int64_t N, int64_t V, float* flat,
+                                cudaStream_t s) {
+  if (N <= 0) return cudaSuccess;
+  flat_combine_kernel<<<static_cast<unsigned>((N + kCombineThreads - 1) / kCombineThreads),
+                        kCombineThreads, 0, s>>>(part, nch, N, V, flat);
   return cudaGetLastError();
 }
 

@@ -233,6 +233,39 @@ def lm_head_loss_fwd_bwd(kind, hidden, weight, labels=None, target_hidden=None,
     return out, dH, dW
 
 
+def align_labels(tokens, shift, loss_mask=None, seq_ids=None, ignore_index=IGNORE_INDEX):
+    """Labels of a draft head that predicts ``shift`` tokens ahead, aligned before chunking
+    (through ``slm_align_labels``).  tokens int32 [B, S] (CUDA); loss_mask bool/uint8 [B, S]
+    or None; seq_ids int32 [B, S] or None.  Returns int32 [B * S]."""
+    if tokens.dtype != torch.int32 or not tokens.is_cuda or tokens.dim() != 2:
+        raise ValueError("tokens must be a 2-D int32 CUDA tensor")
+    B, S = tokens.shape
+    tokens = tokens.contiguous()
+    mask = None if loss_mask is None else loss_mask.to(torch.uint8).contiguous()
+    seq = None if seq_ids is None else seq_ids.to(torch.int32).contiguous()
+    out = torch.empty(B * S, dtype=torch.int32, device=tokens.device)
+    st = _lib.slm_align_labels(_ptr(tokens), _ptr(mask), _ptr(seq), B, S, shift, ignore_index,
+                               _ptr(out), _stream())
+    _lib.check(st, "slm_align_labels")
+    return out
+
+
+def target_flatness(target_hidden, weight):
+    """Per-token flatness cos(p, uniform) of p = softmax(target_hidden weight^T) through
+    ``slm_target_flatness``.  Returns float32 [N]."""
+    _check_inputs(_lib.SLM_KL, target_hidden, weight, None, target_hidden)
+    N, d = target_hidden.shape
+    V = weight.shape[0]
+    dev = target_hidden.device
+    ws = torch.empty(max(_lib.slm_flatness_workspace_bytes(N, d, V), 256), dtype=torch.uint8,
+                     device=dev)
+    out = torch.empty(N, dtype=torch.float32, device=dev)
+    st = _lib.slm_target_flatness(_ptr(target_hidden), _ptr(weight), N, d, V, _ptr(out),
+                                  _ptr(ws), ws.numel(), _stream())
+    _lib.check(st, "slm_target_flatness")
+    return out
+
+
 def device_status(fwd: FwdResult):
     """Synchronise and return the device status of the last call on this workspace."""
     return _lib.slm_device_status(_ptr(fwd.workspace), _stream())

@@ -146,3 +146,14 @@ def test_combo_host_errors(lib):
     assert _combo_fwd({"tv": 1.0}, W=A + 8) == 3
     assert _combo_fwd({"tv": 1.0}, ws_bytes=16) == 5
     assert _combo_fwd({"tv": 1.0}, stats=None) == 1
+
+
+def test_helper_host_errors(lib):
+    assert _lib.slm_align_labels(A, None, None, 2, 3, -1, -100, A, None) == 2   # shift < 0
+    assert _lib.slm_align_labels(A, None, None, -1, 3, 1, -100, A, None) == 2
+    assert _lib.slm_align_labels(None, None, None, 0, 3, 1, -100, None, None) == 0  # empty
+    assert _lib.slm_align_labels(None, None, None, 2, 3, 1, -100, A, None) == 1
+    assert _lib.slm_flatness_workspace_bytes(4, 12, 10) == 0
+    assert _lib.slm_target_flatness(A, A, 4, 12, 10, A, A, 1 << 30, None) == 2
+    assert _lib.slm_target_flatness(None, A, 4, 16, 10, A, A, 1 << 30, None) == 1
+    assert _lib.slm_target_flatness(A, A, 4, 16, 10, A, A, 16, None) == 5
