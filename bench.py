@@ -50,6 +50,8 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-sample-rows", type=int, default=0)
+    ap.add_argument("--no-fused-line", action="store_true",
+                    help="skip timing the fused single call beside the default path")
     ap.add_argument("--fused", action="store_true",
                     help="time the single-call forward+backward that keeps each chunk's "
                          "logits instead of recomputing them")
@@ -345,6 +347,34 @@ def run_ours(args):
     ms_step = total_ms / args.steps
     tokens_per_s = world * N / (ms_step / 1e3)
 
+    # The fused single call (each chunk's logits kept instead of recomputed), timed the same
+    # way on the same inputs, for reference beside the default path.
+    fused_info = None
+    if not args.fused and world == 1 and not args.no_fused_line:
+        fws = torch.empty(_lib.slm_fused_workspace_bytes(k, N, d, V, args.chunk_tokens),
+                          dtype=torch.uint8, device=dev)
+
+        def fused_step():
+            lm_head_loss_fwd_bwd(kind, Hq, W, lab, Hp, inp.ignore_index,
+                                 chunk_tokens=args.chunk_tokens, workspace=fws, out=res,
+                                 dH=dH, dW=dW)
+
+        for _ in range(max(1, args.warmup)):
+            fused_step()
+        torch.cuda.synchronize()
+        fa, fb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        fa.record(stream)
+        for _ in range(args.steps):
+            fused_step()
+        fb.record(stream)
+        torch.cuda.synchronize()
+        f_ms = fa.elapsed_time(fb) / args.steps
+        fused_info = {"ms_per_step": round(f_ms, 3), "value": round(N / (f_ms / 1e3), 1),
+                      "unit": "tokens/s",
+                      "tflops": round(fused_gemm_passes(kind) * 2.0 * N * V * d / (f_ms / 1e3) / 1e12, 1),
+                      "flops_per_token": f"{fused_gemm_passes(kind) * 2}*V*d"}
+        del fws
+
     # End to end through the public API with host buffers: each step copies the inputs
     # from pinned host memory and reads the loss back.
     e2e = None
@@ -435,6 +465,7 @@ def run_ours(args):
                          else launches_per_step(kind, N, d, args.chunk_tokens)) * args.steps,
         "clocks": clocks,
         "e2e": e2e,
+        "fused": fused_info,
         "kernel_sha": kernel_source_hash(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
