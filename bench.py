@@ -275,6 +275,10 @@ def run_ours(args):
     dH = torch.empty(N, d, dtype=torch.bfloat16, device=dev)
     dW = torch.empty(V, d, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
+    # Peak memory of a step: inputs, outputs and workspace (the library allocates nothing),
+    # measured after the synthetic draws' temporaries are gone.
+    torch.cuda.synchronize()
+    torch.cuda.reset_peak_memory_stats(dev)
 
     def make_step(Hq_, W_, lab_, Hp_):
         def _fwd(ev=None):
@@ -346,6 +350,16 @@ def run_ours(args):
         total_ms = float(tt.item())
     ms_step = total_ms / args.steps
     tokens_per_s = world * N / (ms_step / 1e3)
+    gib = float(1 << 30)
+    dual = Hp is not None and kind != "ce"
+    memory = {
+        "peak_allocated_gib": round(torch.cuda.max_memory_allocated(dev) / gib, 3),
+        "workspace_gib": round(ws_bytes / gib, 3),
+        "inputs_gib": round(sum(t.numel() * t.element_size()
+                                for t in (Hq, W, Hp, lab) if t is not None) / gib, 3),
+        "grads_gib": round((dH.numel() * 2 + dW.numel() * 4) / gib, 3),
+        "fp32_logits_avoided_gib": round(N * V * 4 * (2 if dual else 1) / gib, 2),
+    }
 
     # The fused single call (each chunk's logits kept instead of recomputed), timed the same
     # way on the same inputs, for reference beside the default path.
@@ -372,7 +386,8 @@ def run_ours(args):
         fused_info = {"ms_per_step": round(f_ms, 3), "value": round(N / (f_ms / 1e3), 1),
                       "unit": "tokens/s",
                       "tflops": round(fused_gemm_passes(kind) * 2.0 * N * V * d / (f_ms / 1e3) / 1e12, 1),
-                      "flops_per_token": f"{fused_gemm_passes(kind) * 2}*V*d"}
+                      "flops_per_token": f"{fused_gemm_passes(kind) * 2}*V*d",
+                      "workspace_gib": round(fws.numel() / float(1 << 30), 3)}
         del fws
 
     # End to end through the public API with host buffers: each step copies the inputs
@@ -464,6 +479,7 @@ def run_ours(args):
         "gpu_launches": (fused_launches_per_step(kind, N, args.chunk_tokens) if args.fused
                          else launches_per_step(kind, N, d, args.chunk_tokens)) * args.steps,
         "clocks": clocks,
+        "memory": memory,
         "e2e": e2e,
         "fused": fused_info,
         "kernel_sha": kernel_source_hash(),

@@ -69,6 +69,27 @@ def test_workspace_holds_chunk_buffer(lib):
     assert _lib.slm_workspace_bytes(_lib.SLM_CE, 0, 8, 10) > 0
 
 
+@pytest.mark.parametrize("kind", range(8))
+def test_workspace_is_linear_in_tokens_and_bounded_by_dw(lib, kind):
+    """Memory stays O(N d + V d): the backward's chunk buffer is capped by the size of the
+    fp32 dW (chunk = min(N, 2d) rows of bf16 logit gradients), and everything else grows
+    by a fixed number of bytes per token (the forward's per-row partial statistics).  The
+    fused call's buffer holds a fixed number of chunk rows, whatever N and d are."""
+    V = 128256
+    for d in (256, 2048, 4096, 16384):
+        for N in (256, 8192, 65536, 1 << 20):
+            ws = _lib.slm_workspace_bytes(kind, N, d, V, 0)
+            assert 0 < ws <= 4 * V * d + 1536 * N + (1 << 20), (d, N, ws)
+            assert ws < N * V * 4 or N <= 2 * d   # never the whole batch's fp32 logits
+            fws = _lib.slm_fused_workspace_bytes(kind, N, d, V, 0)
+            # fp32 q and p logits plus bf16 dZ for 4096 rows, and the chunk's partials.
+            assert 0 < fws <= 10 * 4096 * V + 64 * N + (16 << 20), (d, N, fws)
+    # Doubling the batch past the chunk size adds only per-token bytes.
+    a = _lib.slm_workspace_bytes(kind, 1 << 16, 4096, V, 0)
+    b = _lib.slm_workspace_bytes(kind, 1 << 17, 4096, V, 0)
+    assert 0 <= b - a <= 1536 * (1 << 16)
+
+
 A = 1 << 20  # a 256-byte aligned fake address; never dereferenced on these paths
 
 
