@@ -35,6 +35,21 @@ constexpr size_t kAlign = 256;
 #ifndef SLM_MAX_RUNS
 #define SLM_MAX_RUNS 32
 #endif
+// Loose lockstep of the GEMMs' CTA pairs (K blocks per progress step, steps of slack; 0 K
+// blocks = off): V for the GEMMs over the vocabulary (forward, logits gradient, second
+// pass), B for the dH and dW GEMMs.
+#ifndef SLM_SYNC_KB_V
+#define SLM_SYNC_KB_V 16
+#endif
+#ifndef SLM_SYNC_SLACK_V
+#define SLM_SYNC_SLACK_V 2
+#endif
+#ifndef SLM_SYNC_KB_B
+#define SLM_SYNC_KB_B 0
+#endif
+#ifndef SLM_SYNC_SLACK_B
+#define SLM_SYNC_SLACK_B 2
+#endif
 constexpr int kPairM = 2 * kBM;                // M rows of one 2-SM tile
 constexpr int kGroupPairs = SLM_GROUP_PAIRS;   // pair M tiles per raster group
 constexpr int kMaxRuns = SLM_MAX_RUNS;         // vocabulary runs per row, at most
@@ -174,8 +189,11 @@ bool make_map(CUtensorMap* m, const void* base, int64_t inner, int64_t outer, in
 bool misaligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) != 0; }
 
 // Tile schedule of a GEMM with M tiles of `bm` rows (256: a 2-SM CTA pair).
-GemmGeom geom(int64_t M, int64_t Nn, int64_t K, int bn, int vc, int group_m, int bm) {
-  GemmGeom g;
+GemmGeom geom(int64_t M, int64_t Nn, int64_t K, int bn, int vc, int group_m, int bm,
+              int sync_kb, int slack) {
+  GemmGeom g{};
+  g.sync_kb = sync_kb;
+  g.slack = slack;
   g.num_m = static_cast<int>(ceil_div(M, bm));
   g.num_n = static_cast<int>(ceil_div(Nn, bn));
   g.k_blocks = static_cast<int>(ceil_div(K, kBK));
@@ -386,7 +404,8 @@ int slm_loss_fwd(int kind, const void* Hq, const void* Hp, const void* W, const 
 
   if (N > 0) {
     const FwdSched f = fwd_sched(kind, V);
-    const GemmGeom g = geom(N, V, d, f.bn, f.vc, kGroupPairs, kPairM);
+    const GemmGeom g = geom(N, V, d, f.bn, f.vc, kGroupPairs, kPairM,
+                             SLM_SYNC_KB_V, SLM_SYNC_SLACK_V);
     CUtensorMap tHq, tHp, tW;
     if (!make_map(&tHq, Hq, d, N, d, kBK, kBM)) return SLM_ERR_CUDA;
     if (!make_map(&tW, W, d, V, d, kBK, 128)) return SLM_ERR_CUDA;
@@ -464,7 +483,8 @@ int slm_loss_bwd(int kind, const void* Hq, const void* Hp, const void* W, const 
     // 1) Recompute the chunk's logits and write its logits gradient dZ [rows, V] (bf16).
     CUtensorMap tHq, tHp;
     if (!make_map(&tHq, hq, d, rows, d, kBK, kBM)) return SLM_ERR_CUDA;
-    const GemmGeom gz = geom(rows, V, d, f.bn, f.vc, kGroupPairs, kPairM);
+    const GemmGeom gz = geom(rows, V, d, f.bn, f.vc, kGroupPairs, kPairM,
+                             SLM_SYNC_KB_V, SLM_SYNC_SLACK_V);
     DzParams pz{dz_kind, dz_labels, ignore_index, c0, rows, N, V, stats, grad_tok, grad_scale,
                 n_valid, dz, ldz, ComboW{}};
     if (!dual_kind(dz_kind)) {
@@ -477,13 +497,15 @@ int slm_loss_bwd(int kind, const void* Hq, const void* Hp, const void* W, const 
     // 2) dH[chunk] = dZ W   (M = rows, N = d, K = V; W read MN-major).
     CUtensorMap tDz_k, tDz_mn, tH_mn;
     if (!make_map(&tDz_k, dz, V, rows, ldz, kBK, kBM)) return SLM_ERR_CUDA;
-    const GemmGeom gh = geom(rows, d, V, kTileDh, 1, 1, kPairM);
+    const GemmGeom gh = geom(rows, d, V, kTileDh, 1, 1, kPairM,
+                              SLM_SYNC_KB_B, SLM_SYNC_SLACK_B);
     DhParams ph{static_cast<__nv_bfloat16*>(dHq), c0, rows, d};
     SLM_TRY_CUDA(launch_dh(tDz_k, tW_mn, gh, ph, ctl, s));
     // 3) dW (+)= dZ^T H[chunk]   (M = V, N = d, K = rows; both operands MN-major).
     if (!make_map(&tDz_mn, dz, V, rows, ldz, 64, 64)) return SLM_ERR_CUDA;
     if (!make_map(&tH_mn, hq, d, rows, d, 64, 64)) return SLM_ERR_CUDA;
-    const GemmGeom gw = geom(V, d, rows, kTileDw, 1, 1, kPairM);
+    const GemmGeom gw = geom(V, d, rows, kTileDw, 1, 1, kPairM,
+                              SLM_SYNC_KB_B, SLM_SYNC_SLACK_B);
     DwParams pw{dW, V, d, (accumulate_dW || c0 > 0) ? 1 : 0};
     SLM_TRY_CUDA(launch_dw(tDz_mn, tH_mn, gw, pw, ctl, s));
   }
@@ -529,7 +551,8 @@ int slm_target_flatness(const void* Hp, const void* W, int64_t N, int64_t d, int
   SLM_TRY_CUDA(cudaMemsetAsync(status, 0, sizeof(int), s));
   const DevCtl ctl = make_ctl(status);
   const FwdSched f = fwd_sched(SLM_CE, V);
-  const GemmGeom g = geom(N, V, d, f.bn, f.vc, kGroupPairs, kPairM);
+  const GemmGeom g = geom(N, V, d, f.bn, f.vc, kGroupPairs, kPairM,
+                             SLM_SYNC_KB_V, SLM_SYNC_SLACK_V);
   CUtensorMap tHp, tW;
   if (!make_map(&tHp, Hp, d, N, d, kBK, kBM)) return SLM_ERR_CUDA;
   if (!make_map(&tW, W, d, V, d, kBK, 128)) return SLM_ERR_CUDA;
@@ -596,7 +619,8 @@ int slm_loss_fwd_bwd(int kind, const void* Hq, const void* Hp, const void* W,
     CUtensorMap tHq, tHp, tDz_k, tDz_mn, tH_mn;
     if (!make_map(&tHq, hq, d, rows, d, kBK, kBM)) return SLM_ERR_CUDA;
     // 1) Logits of the chunk: statistics in the epilogue, fp32 logits kept.
-    const GemmGeom g = geom(rows, V, d, f.bn, f.vc, kGroupPairs, kPairM);
+    const GemmGeom g = geom(rows, V, d, f.bn, f.vc, kGroupPairs, kPairM,
+                             SLM_SYNC_KB_V, SLM_SYNC_SLACK_V);
     FwdParams p{labels ? labels + c0 : nullptr, ignore_index, rows, V, part, zy, nullptr, 0,
                 lq, (dual_kind(kind) && !argmax_kind) ? lp : nullptr, ldl};
     if (!dual_kind(kind)) {
@@ -623,12 +647,14 @@ int slm_loss_fwd_bwd(int kind, const void* Hq, const void* Hp, const void* W,
     SLM_TRY_CUDA(launch_logits_dz(pz, lq, lp, ldl, s));
     // 4) dH[chunk] = dZ W and dW (+)= dZ^T H[chunk].
     if (!make_map(&tDz_k, dz, V, rows, ldz, kBK, kBM)) return SLM_ERR_CUDA;
-    const GemmGeom gh = geom(rows, d, V, kTileDh, 1, 1, kPairM);
+    const GemmGeom gh = geom(rows, d, V, kTileDh, 1, 1, kPairM,
+                              SLM_SYNC_KB_B, SLM_SYNC_SLACK_B);
     DhParams ph{static_cast<__nv_bfloat16*>(dHq), c0, rows, d};
     SLM_TRY_CUDA(launch_dh(tDz_k, tW_mn, gh, ph, ctl, s));
     if (!make_map(&tDz_mn, dz, V, rows, ldz, 64, 64)) return SLM_ERR_CUDA;
     if (!make_map(&tH_mn, hq, d, rows, d, 64, 64)) return SLM_ERR_CUDA;
-    const GemmGeom gw = geom(V, d, rows, kTileDw, 1, 1, kPairM);
+    const GemmGeom gw = geom(V, d, rows, kTileDw, 1, 1, kPairM,
+                              SLM_SYNC_KB_B, SLM_SYNC_SLACK_B);
     DwParams pw{dW, V, d, (accumulate_dW || c0 > 0) ? 1 : 0};
     SLM_TRY_CUDA(launch_dw(tDz_mn, tH_mn, gw, pw, ctl, s));
   }
@@ -667,7 +693,8 @@ int slm_combo_fwd(const float* weights, const void* Hq, const void* Hp, const vo
   const DevCtl ctl = make_ctl(status);
   if (N > 0) {
     const FwdSched f = fwd_sched(SLM_KL, V);
-    const GemmGeom g = geom(N, V, d, f.bn, f.vc, kGroupPairs, kPairM);
+    const GemmGeom g = geom(N, V, d, f.bn, f.vc, kGroupPairs, kPairM,
+                             SLM_SYNC_KB_V, SLM_SYNC_SLACK_V);
     // A CE-only combination has no target: the draft stands in for it (its statistics are
     // computed and unused).
     const void* hp = Hp ? Hp : Hq;
@@ -731,17 +758,20 @@ int slm_combo_bwd(const float* weights, const void* Hq, const void* Hp, const vo
     CUtensorMap tHq, tHp, tDz_k, tDz_mn, tH_mn;
     if (!make_map(&tHq, hq, d, rows, d, kBK, kBM)) return SLM_ERR_CUDA;
     if (!make_map(&tHp, hp, d, rows, d, kBK, kBM)) return SLM_ERR_CUDA;
-    const GemmGeom gz = geom(rows, V, d, f.bn, f.vc, kGroupPairs, kPairM);
+    const GemmGeom gz = geom(rows, V, d, f.bn, f.vc, kGroupPairs, kPairM,
+                             SLM_SYNC_KB_V, SLM_SYNC_SLACK_V);
     DzParams pz{-1, labels, ignore_index, c0, rows, N, V, stats, grad_tok, grad_scale,
                 n_valid, dz, ldz, cw};
     SLM_TRY_CUDA(launch_dz_combo(tHq, tHp, tW_k, gz, pz, ctl, s));
     if (!make_map(&tDz_k, dz, V, rows, ldz, kBK, kBM)) return SLM_ERR_CUDA;
-    const GemmGeom gh = geom(rows, d, V, kTileDh, 1, 1, kPairM);
+    const GemmGeom gh = geom(rows, d, V, kTileDh, 1, 1, kPairM,
+                              SLM_SYNC_KB_B, SLM_SYNC_SLACK_B);
     DhParams ph{static_cast<__nv_bfloat16*>(dHq), c0, rows, d};
     SLM_TRY_CUDA(launch_dh(tDz_k, tW_mn, gh, ph, ctl, s));
     if (!make_map(&tDz_mn, dz, V, rows, ldz, 64, 64)) return SLM_ERR_CUDA;
     if (!make_map(&tH_mn, hq, d, rows, d, 64, 64)) return SLM_ERR_CUDA;
-    const GemmGeom gw = geom(V, d, rows, kTileDw, 1, 1, kPairM);
+    const GemmGeom gw = geom(V, d, rows, kTileDw, 1, 1, kPairM,
+                              SLM_SYNC_KB_B, SLM_SYNC_SLACK_B);
     DwParams pw{dW, V, d, (accumulate_dW || c0 > 0) ? 1 : 0};
     SLM_TRY_CUDA(launch_dw(tDz_mn, tH_mn, gw, pw, ctl, s));
   }

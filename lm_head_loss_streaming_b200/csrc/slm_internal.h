@@ -54,6 +54,12 @@ struct GemmGeom {
   int group_m;    // M tiles per raster group
   int units_n;    // ceil(num_n / vc)
   int num_units;  // num_m * units_n
+  // Loose lockstep of the pairs (set at launch): every sync_kb K blocks a pair publishes its
+  // progress under this launch's tag `epoch` and waits, briefly and boundedly, until no
+  // started pair is more than `slack` such steps behind it.  epoch 0 = off.
+  uint32_t epoch;
+  int sync_kb;
+  int slack;
 };
 
 struct DevCtl {

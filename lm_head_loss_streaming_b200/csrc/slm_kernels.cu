@@ -33,6 +33,7 @@
 #include <math.h>
 
 #include <algorithm>
+#include <atomic>
 
 #include "slm_internal.h"
 #include "sm100.cuh"
@@ -66,13 +67,76 @@ __device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, volati
   return __all_sync(0xffffffffu, done);
 }
 
+// Work unit u -> (pair M tile mt, vocabulary run j).  Units are handed to the pairs round
+// robin, so the pairs that start together share B tiles only while their units have the
+// same length.  The runs of vc tiles come first, in raster groups of group_m M tiles with M
+// fastest (the pairs running the same run j at once read the same W tiles); the short last
+// run of every row (when vc does not divide num_n) is deferred to the end of the schedule,
+// where its small units also even out the pairs' finishing times.
 __device__ __forceinline__ void unit_coords(const GemmGeom& g, int u, int& mt, int& j) {
-  const int per_group = g.group_m * g.units_n;
+  const int full_runs = (g.num_n % g.vc) != 0 ? g.units_n - 1 : g.units_n;
+  const int n_full = g.num_m * full_runs;
+  if (u >= n_full) {
+    mt = u - n_full;
+    j = full_runs;
+    return;
+  }
+  const int per_group = g.group_m * full_runs;
   const int grp = u / per_group;
   const int r = u - grp * per_group;
   const int gm = min(g.group_m, g.num_m - grp * g.group_m);
   j = r / gm;
   mt = grp * g.group_m + (r - j * gm);
+}
+
+// Loose lockstep of the pairs.  Pairs that read the same W tiles at nearly the same time
+// share them in L2; left alone they drift apart by more than a tile's L2 residency, and W
+// is then fetched from DRAM once per pair.  The leader CTA's producer of every pair records
+// its progress (K blocks issued, in steps of g.sync_kb) under the launch's tag and lets no
+// pair run more than g.slack steps ahead of the slowest started pair.
+constexpr int kMaxSyncPairs = 128;
+constexpr long long kSyncSpinCycles = 1LL << 21;
+__device__ unsigned long long g_pair_progress[kMaxSyncPairs];
+
+__device__ __forceinline__ void st_relaxed_u64(unsigned long long* p, unsigned long long v) {
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+__device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Records that this pair begins progress step `step` (from 1) and waits until every started
+// pair of this launch has begun step `step - slack`.  Pairs with no record under this
+// launch's tag (not resident yet) and finished pairs (step 0xffffffff) hold nobody back.
+// The wait only shapes performance: after kSyncSpinCycles it gives up, marks this pair as
+// finished for the others and returns false, and the caller stops synchronising.
+// Warp-collective.
+__device__ __forceinline__ bool lockstep(const GemmGeom& g, int pair, int npairs,
+                                         uint32_t step) {
+  const int lane = threadIdx.x & 31;
+  const unsigned long long tag = static_cast<unsigned long long>(g.epoch) << 32;
+  if (lane == 0) st_relaxed_u64(&g_pair_progress[pair], tag | step);
+  __syncwarp();
+  if (step <= static_cast<uint32_t>(g.slack)) return true;
+  const uint32_t need = step - static_cast<uint32_t>(g.slack);
+  const long long t0 = clock64();
+  while (true) {
+    uint32_t mn = 0xffffffffu;
+    for (int i = lane; i < npairs; i += 32) {
+      const unsigned long long v = ld_relaxed_u64(&g_pair_progress[i]);
+      if ((v >> 32) == g.epoch) mn = min(mn, static_cast<uint32_t>(v));
+    }
+    mn = __reduce_min_sync(0xffffffffu, mn);
+    if (mn >= need) return true;
+    if (__any_sync(0xffffffffu, clock64() - t0 > kSyncSpinCycles)) {
+      if (lane == 0) st_relaxed_u64(&g_pair_progress[pair], tag | 0xffffffffull);
+      __syncwarp();
+      return false;
+    }
+    __nanosleep(128);
+  }
 }
 
 // ----------------------------------------------------------------------------------------
@@ -183,6 +247,9 @@ __global__ void __launch_bounds__(64 + 128 * NWG, 1)
     // ------------------------------ TMA producer (both CTAs) ------------------------------
     uint32_t it = 0;
     bool ok = true;
+    const bool sync_pub = g.epoch != 0 && leader && pair < kMaxSyncPairs && npairs <= kMaxSyncPairs;
+    bool sync_on = sync_pub;
+    uint32_t sync_step = 0;
     for (int u = pair; ok && u < g.num_units; u += npairs) {
       int mt, j;
       unit_coords(g, u, mt, j);
@@ -190,6 +257,8 @@ __global__ void __launch_bounds__(64 + 128 * NWG, 1)
       const int n_end = min((j + 1) * g.vc, g.num_n);
       for (int nt = j * g.vc; ok && nt < n_end; ++nt) {
         for (int kb = 0; kb < g.k_blocks; ++kb, ++it) {
+          if (sync_on && it % static_cast<uint32_t>(g.sync_kb) == 0)
+            sync_on = lockstep(g, pair, npairs, ++sync_step);
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
           if (!wait_warp(&pc->empty[s], ph ^ 1u, abort, ctl)) {
@@ -228,6 +297,9 @@ __global__ void __launch_bounds__(64 + 128 * NWG, 1)
         }
       }
     }
+    if (sync_pub && lane == 0)
+      st_relaxed_u64(&g_pair_progress[pair],
+                     (static_cast<unsigned long long>(g.epoch) << 32) | 0xffffffffull);
     if (!ok) {
       if (leader) {
         // The full barriers count both CTAs' copies: waiting on them lets the pair's
@@ -1303,7 +1375,16 @@ static cudaError_t launch_pair(const CUtensorMap& a0, const CUtensorMap& a1,
   }
   const int pairs = std::max(1, std::min(g.num_units, max_clusters[dev]));
   cfg.gridDim = dim3(2 * pairs, 1, 1);
-  return cudaLaunchKernelEx(&cfg, kern, a0, a1, b, g, p, c);
+  GemmGeom gg = g;
+  gg.epoch = 0;
+  if (g.sync_kb > 0 && g.slack >= 0 && pairs > 1 && pairs <= kMaxSyncPairs) {
+    // A fresh tag per launch: records left by earlier launches are ignored.
+    static std::atomic<uint32_t> next_epoch{1};
+    uint32_t e = next_epoch.fetch_add(1);
+    if (e == 0) e = next_epoch.fetch_add(1);
+    gg.epoch = e;
+  }
+  return cudaLaunchKernelEx(&cfg, kern, a0, a1, b, gg, p, c);
 }
 
 // Forward statistics and logits gradient: A = hidden states (K-major), B = W (K-major).
