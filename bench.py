@@ -31,9 +31,12 @@ if ROOT not in sys.path:
 METRIC = "LM-head+loss fwd+bwd tokens/s (d=4096,V=128256); % of BF16 tensor peak"
 DEFAULT_WORKLOAD = "llama8b_kl"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# The kernels and the host code that picks their tiles, schedule and launch shape: DRAM
+# counters taken with other sources do not describe this build.
 KERNEL_SOURCES = ["lm_head_loss_streaming_b200/csrc/slm_kernels.cu",
                   "lm_head_loss_streaming_b200/csrc/sm100.cuh",
-                  "lm_head_loss_streaming_b200/csrc/slm_internal.h"]
+                  "lm_head_loss_streaming_b200/csrc/slm_internal.h",
+                  "lm_head_loss_streaming_b200/csrc/slm_api.cu"]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.txt")
 
 
