@@ -58,6 +58,11 @@ def parse_args():
     ap.add_argument("--fused", action="store_true",
                     help="time the single-call forward+backward that keeps each chunk's "
                          "logits instead of recomputing them")
+    ap.add_argument("--no-overlap", action="store_true",
+                    help="N > 1: sum dW across ranks after the backward instead of "
+                         "overlapping the sum with the last chunk's dH GEMM")
+    ap.add_argument("--reserve-sms", type=int, default=8,
+                    help="N > 1: SMs the last dH GEMM leaves to the dW reduction")
     return ap.parse_args()
 
 
@@ -295,8 +300,16 @@ def run_ours(args):
 
         def _bwd(r, n_valid_global):
             r.n_valid.copy_(n_valid_global)
-            return lm_head_loss_bwd(r, Hq_, W_, lab_, Hp_, inp.ignore_index, dH=dH, dW=dW,
-                                    chunk_tokens=args.chunk_tokens)
+            if args.no_overlap:
+                return lm_head_loss_bwd(r, Hq_, W_, lab_, Hp_, inp.ignore_index, dH=dH, dW=dW,
+                                        chunk_tokens=args.chunk_tokens)
+            # dW is summed across ranks on a side stream while the last chunk's dH GEMM
+            # runs (lm_head_loss_streaming_b200.dp).
+            ready = torch.cuda.Event()
+            gh, gw = lm_head_loss_bwd(r, Hq_, W_, lab_, Hp_, inp.ignore_index, dH=dH, dW=dW,
+                                      chunk_tokens=args.chunk_tokens, dw_ready=ready,
+                                      reserve_sms=args.reserve_sms)
+            return gh, gw, ready
 
         def step(ev=None):
             if args.fused:
@@ -312,7 +325,8 @@ def run_ours(args):
             elif world > 1:
                 # Data parallel over token rows: global valid count before the backward,
                 # dW and the loss sum summed after it (lm_head_loss_streaming_b200.dp).
-                dp.fwd_bwd(lambda: _fwd(ev), _bwd)
+                dp.fwd_bwd(lambda: _fwd(ev), _bwd,
+                           comm_stream=None if args.no_overlap else dp.comm_stream_for(dev))
             else:
                 r = _fwd(ev)
                 lm_head_loss_bwd(r, Hq_, W_, lab_, Hp_, inp.ignore_index, dH=dH, dW=dW,
@@ -468,6 +482,9 @@ def run_ours(args):
                    "path": "fused (chunk logits kept)" if args.fused else "recompute",
                    "V": V, "global_batch_tokens": world * N, "parallelism": f"dp{world}",
                    "chunk_tokens": args.chunk_tokens or "auto",
+                   "dw_exchange": (None if world == 1 else
+                                   "after the backward" if args.no_overlap else
+                                   "overlapped with the last chunk's dH GEMM"),
                    "l2": "inputs larger than L2 (W alone is %.2f GB)" % (V * d * 2 / 1e9)},
         "tflops": round(flops_step / (ms_step / 1e3) / 1e12, 1),
         "frac_bf16_peak": round(flops_step / (ms_step / 1e3) / 1e12 / peaks["bf16_tflops"], 4),

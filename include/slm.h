@@ -156,6 +156,28 @@ SLM_API int slm_loss_bwd(int kind, const void* Hq, const void* Hp, const void* W
                  const float* stats, void* dHq, float* dW, int accumulate_dW,
                  int64_t chunk_tokens, void* workspace, size_t ws_bytes, void* stream);
 
+/* slm_loss_bwd for data-parallel training, where dW is summed across ranks after the
+ * backward ("Training speculative decoders: removing the logits and attention
+ * bottlenecks", "Streaming Cross Entropy": the streaming loss is orthogonal to data
+ * parallelism).  Same arguments, same results, bit for bit, plus:
+ *   dw_ready_event  a cudaEvent_t created by the caller, or NULL.  It is recorded on
+ *                   `stream` as soon as dW is final, before the last chunk's dH GEMM, so a
+ *                   reduction of dW on another stream can wait on it and overlap that GEMM.
+ *                   The caller owns the event; it is recorded once per call.
+ *   reserve_sms     SMs (0..128) that the last chunk's dH GEMM leaves idle, so that the
+ *                   reduction's kernels find free SMs while it runs; rounded up to whole
+ *                   2-SM pairs.  0 = use them all.
+ * To make this possible, the last chunk runs its dW GEMM before its dH GEMM.
+ * Returns SLM_ERR_SHAPE for reserve_sms outside 0..128 and otherwise what slm_loss_bwd
+ * returns. */
+SLM_API int slm_loss_bwd_overlap(int kind, const void* Hq, const void* Hp, const void* W,
+                 const int32_t* labels, int32_t ignore_index,
+                 int64_t N, int64_t d, int64_t V,
+                 const float* grad_tok, const float* grad_scale, const int64_t* n_valid,
+                 const float* stats, void* dHq, float* dW, int accumulate_dW,
+                 int64_t chunk_tokens, void* workspace, size_t ws_bytes, void* stream,
+                 void* dw_ready_event, int reserve_sms);
+
 /* Synchronises `stream`, then returns and clears the device status word of `workspace`:
  * SLM_OK, SLM_ERR_LABEL_RANGE or SLM_ERR_TIMEOUT (the first found), or SLM_ERR_CUDA if
  * the stream reported an error.  Every slm_loss_fwd / slm_loss_bwd call also clears the

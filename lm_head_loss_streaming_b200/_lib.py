@@ -44,6 +44,9 @@ SIGNATURES = {
                             _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "slm_loss_bwd": (_INT, [_INT, _P, _P, _P, _P, _I32, _I64, _I64, _I64,
                             _P, _P, _P, _P, _P, _P, _INT, _I64, _P, _SZ, _P]),
+    "slm_loss_bwd_overlap": (_INT, [_INT, _P, _P, _P, _P, _I32, _I64, _I64, _I64,
+                                    _P, _P, _P, _P, _P, _P, _INT, _I64, _P, _SZ, _P,
+                                    _P, _INT]),
     "slm_device_status": (_INT, [_P, _P]),
     "slm_debug_set": (_INT, [_INT, ctypes.c_longlong]),
     "slm_fused_workspace_bytes": (_SZ, [_INT, _I64, _I64, _I64, _I64]),
@@ -131,6 +134,16 @@ def slm_loss_bwd(kind, Hq, Hp, W, labels, ignore_index, N, d, V, grad_tok, grad_
                                int(d), int(V), grad_tok, grad_scale, n_valid, stats, dHq, dW,
                                int(accumulate_dW), int(chunk_tokens), workspace,
                                int(ws_bytes), stream)
+
+
+def slm_loss_bwd_overlap(kind, Hq, Hp, W, labels, ignore_index, N, d, V, grad_tok,
+                         grad_scale, n_valid, stats, dHq, dW, accumulate_dW, chunk_tokens,
+                         workspace, ws_bytes, stream, dw_ready_event, reserve_sms):
+    return load().slm_loss_bwd_overlap(int(kind), Hq, Hp, W, labels, int(ignore_index),
+                                       int(N), int(d), int(V), grad_tok, grad_scale, n_valid,
+                                       stats, dHq, dW, int(accumulate_dW), int(chunk_tokens),
+                                       workspace, int(ws_bytes), stream, dw_ready_event,
+                                       int(reserve_sms))
 
 
 def slm_device_status(workspace, stream):

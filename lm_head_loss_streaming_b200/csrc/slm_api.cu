@@ -51,6 +51,7 @@ constexpr size_t kAlign = 256;
 #define SLM_SYNC_SLACK_B 2
 #endif
 constexpr int kPairM = 2 * kBM;                // M rows of one 2-SM tile
+constexpr int kMaxReserveSms = 128;            // slm_loss_bwd_overlap's reserve_sms, at most
 constexpr int kGroupPairs = SLM_GROUP_PAIRS;   // pair M tiles per raster group
 constexpr int kMaxRuns = SLM_MAX_RUNS;         // vocabulary runs per row, at most
 constexpr long long kTimeoutCycles = 4000000000LL;  // ~2 s at the B200's boost clock
@@ -440,11 +441,15 @@ int slm_loss_fwd(int kind, const void* Hq, const void* Hp, const void* W, const 
   return SLM_OK;
 }
 
-int slm_loss_bwd(int kind, const void* Hq, const void* Hp, const void* W, const int32_t* labels,
-                 int32_t ignore_index, int64_t N, int64_t d, int64_t V, const float* grad_tok,
-                 const float* grad_scale, const int64_t* n_valid, const float* stats, void* dHq,
-                 float* dW, int accumulate_dW, int64_t chunk_tokens, void* workspace,
-                 size_t ws_bytes, void* stream) {
+// The backward of slm_loss_bwd and slm_loss_bwd_overlap.  With `overlap`, the last chunk
+// runs its dW GEMM before its dH GEMM, records `dw_ready` (if given) between the two, and
+// launches that dH GEMM on `reserve_pairs` fewer CTA pairs.
+static int loss_bwd(int kind, const void* Hq, const void* Hp, const void* W,
+                    const int32_t* labels, int32_t ignore_index, int64_t N, int64_t d, int64_t V,
+                    const float* grad_tok, const float* grad_scale, const int64_t* n_valid,
+                    const float* stats, void* dHq, float* dW, int accumulate_dW,
+                    int64_t chunk_tokens, void* workspace, size_t ws_bytes, void* stream,
+                    bool overlap, cudaEvent_t dw_ready, int reserve_pairs) {
   int st = common_checks(kind, Hq, Hp, W, labels, N, d, V, workspace, ws_bytes, chunk_tokens,
                          true);
   if (st != SLM_OK) return st;
@@ -461,6 +466,7 @@ int slm_loss_bwd(int kind, const void* Hq, const void* Hp, const void* W, const 
 
   if (N == 0) {
     if (!accumulate_dW) SLM_TRY_CUDA(launch_zero_f32(dW, V * d, s));
+    if (dw_ready) SLM_TRY_CUDA(cudaEventRecord(dw_ready, s));
     return SLM_OK;
   }
   const int64_t C = default_chunk(N, d, chunk_tokens);
@@ -497,19 +503,49 @@ int slm_loss_bwd(int kind, const void* Hq, const void* Hp, const void* W, const 
     // 2) dH[chunk] = dZ W   (M = rows, N = d, K = V; W read MN-major).
     CUtensorMap tDz_k, tDz_mn, tH_mn;
     if (!make_map(&tDz_k, dz, V, rows, ldz, kBK, kBM)) return SLM_ERR_CUDA;
-    const GemmGeom gh = geom(rows, d, V, kTileDh, 1, 1, kPairM,
-                              SLM_SYNC_KB_B, SLM_SYNC_SLACK_B);
+    GemmGeom gh = geom(rows, d, V, kTileDh, 1, 1, kPairM, SLM_SYNC_KB_B, SLM_SYNC_SLACK_B);
     DhParams ph{static_cast<__nv_bfloat16*>(dHq), c0, rows, d};
-    SLM_TRY_CUDA(launch_dh(tDz_k, tW_mn, gh, ph, ctl, s));
     // 3) dW (+)= dZ^T H[chunk]   (M = V, N = d, K = rows; both operands MN-major).
     if (!make_map(&tDz_mn, dz, V, rows, ldz, 64, 64)) return SLM_ERR_CUDA;
     if (!make_map(&tH_mn, hq, d, rows, d, 64, 64)) return SLM_ERR_CUDA;
     const GemmGeom gw = geom(V, d, rows, kTileDw, 1, 1, kPairM,
                               SLM_SYNC_KB_B, SLM_SYNC_SLACK_B);
     DwParams pw{dW, V, d, (accumulate_dW || c0 > 0) ? 1 : 0};
-    SLM_TRY_CUDA(launch_dw(tDz_mn, tH_mn, gw, pw, ctl, s));
+    if (overlap && c0 + rows >= N) {
+      // Last chunk: dW is final once its GEMM is done; the dH GEMM that follows leaves
+      // SMs free for the caller's reduction of dW.
+      SLM_TRY_CUDA(launch_dw(tDz_mn, tH_mn, gw, pw, ctl, s));
+      if (dw_ready) SLM_TRY_CUDA(cudaEventRecord(dw_ready, s));
+      gh.reserve_pairs = reserve_pairs;
+      SLM_TRY_CUDA(launch_dh(tDz_k, tW_mn, gh, ph, ctl, s));
+    } else {
+      SLM_TRY_CUDA(launch_dh(tDz_k, tW_mn, gh, ph, ctl, s));
+      SLM_TRY_CUDA(launch_dw(tDz_mn, tH_mn, gw, pw, ctl, s));
+    }
   }
   return SLM_OK;
+}
+
+int slm_loss_bwd(int kind, const void* Hq, const void* Hp, const void* W, const int32_t* labels,
+                 int32_t ignore_index, int64_t N, int64_t d, int64_t V, const float* grad_tok,
+                 const float* grad_scale, const int64_t* n_valid, const float* stats, void* dHq,
+                 float* dW, int accumulate_dW, int64_t chunk_tokens, void* workspace,
+                 size_t ws_bytes, void* stream) {
+  return loss_bwd(kind, Hq, Hp, W, labels, ignore_index, N, d, V, grad_tok, grad_scale,
+                  n_valid, stats, dHq, dW, accumulate_dW, chunk_tokens, workspace, ws_bytes,
+                  stream, false, nullptr, 0);
+}
+
+int slm_loss_bwd_overlap(int kind, const void* Hq, const void* Hp, const void* W,
+                         const int32_t* labels, int32_t ignore_index, int64_t N, int64_t d,
+                         int64_t V, const float* grad_tok, const float* grad_scale,
+                         const int64_t* n_valid, const float* stats, void* dHq, float* dW,
+                         int accumulate_dW, int64_t chunk_tokens, void* workspace,
+                         size_t ws_bytes, void* stream, void* dw_ready_event, int reserve_sms) {
+  if (reserve_sms < 0 || reserve_sms > kMaxReserveSms) return SLM_ERR_SHAPE;
+  return loss_bwd(kind, Hq, Hp, W, labels, ignore_index, N, d, V, grad_tok, grad_scale,
+                  n_valid, stats, dHq, dW, accumulate_dW, chunk_tokens, workspace, ws_bytes,
+                  stream, true, static_cast<cudaEvent_t>(dw_ready_event), (reserve_sms + 1) / 2);
 }
 
 int slm_align_labels(const int32_t* tokens, const uint8_t* loss_mask, const int32_t* seq_ids,

@@ -60,6 +60,8 @@ struct GemmGeom {
   uint32_t epoch;
   int sync_kb;
   int slack;
+  // CTA pairs to leave idle (so that a collective on another stream finds free SMs).
+  int reserve_pairs;
 };
 
 struct DevCtl {

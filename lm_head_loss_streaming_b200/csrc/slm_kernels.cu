@@ -1373,7 +1373,8 @@ static cudaError_t launch_pair(const CUtensorMap& a0, const CUtensorMap& a1,
     if ((e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg)) != cudaSuccess) return e;
     max_clusters[dev] = n > 0 ? n : 1;
   }
-  const int pairs = std::max(1, std::min(g.num_units, max_clusters[dev]));
+  const int cap = std::max(1, max_clusters[dev] - std::max(0, g.reserve_pairs));
+  const int pairs = std::max(1, std::min(g.num_units, cap));
   cfg.gridDim = dim3(2 * pairs, 1, 1);
   GemmGeom gg = g;
   gg.epoch = 0;

@@ -99,9 +99,15 @@ def lm_head_loss_fwd(kind, hidden, weight, labels=None, target_hidden=None,
 
 def lm_head_loss_bwd(fwd: FwdResult, hidden, weight, labels=None, target_hidden=None,
                      ignore_index=IGNORE_INDEX, grad_tok=None, grad_scale=None,
-                     normalize=True, dH=None, dW=None, accumulate_dW=False, chunk_tokens=0):
+                     normalize=True, dH=None, dW=None, accumulate_dW=False, chunk_tokens=0,
+                     dw_ready=None, reserve_sms=0):
     """Backward through ``slm_loss_bwd``.  With ``normalize`` the upstream gradient is
     divided by the forward's valid-row count (gradient of the mean loss).
+
+    ``dw_ready`` (a ``torch.cuda.Event``) or ``reserve_sms`` > 0 selects
+    ``slm_loss_bwd_overlap``: the event is recorded on the current stream as soon as dW is
+    final, before the last chunk's dH GEMM, which then leaves ``reserve_sms`` SMs idle, so
+    that a reduction of dW on another stream can overlap it.  The results are the same.
     Returns (dH bf16 [N, d], dW fp32 [V, d])."""
     k = fwd.kind
     N, d = hidden.shape
@@ -115,12 +121,20 @@ def lm_head_loss_bwd(fwd: FwdResult, hidden, weight, labels=None, target_hidden=
     ws = fwd.workspace
     if ws.numel() < ws_need:
         ws = torch.empty(ws_need, dtype=torch.uint8, device=dev)
-    st = _lib.slm_loss_bwd(k, _ptr(hidden), _ptr(target_hidden), _ptr(weight), _ptr(labels),
-                           ignore_index, N, d, V, _ptr(grad_tok), _ptr(grad_scale),
-                           _ptr(fwd.n_valid) if normalize else None, _ptr(fwd.stats),
-                           _ptr(dH), _ptr(dW), 1 if accumulate_dW else 0, chunk_tokens,
-                           _ptr(ws), ws.numel(), _stream())
-    _lib.check(st, "slm_loss_bwd")
+    args = (k, _ptr(hidden), _ptr(target_hidden), _ptr(weight), _ptr(labels), ignore_index,
+            N, d, V, _ptr(grad_tok), _ptr(grad_scale),
+            _ptr(fwd.n_valid) if normalize else None, _ptr(fwd.stats), _ptr(dH), _ptr(dW),
+            1 if accumulate_dW else 0, chunk_tokens, _ptr(ws), ws.numel(), _stream())
+    if dw_ready is None and not reserve_sms:
+        _lib.check(_lib.slm_loss_bwd(*args), "slm_loss_bwd")
+        return dH, dW
+    handle = None
+    if dw_ready is not None:
+        # torch creates the CUDA event on its first record; the library records it again
+        # at the point where dW is final.
+        dw_ready.record(torch.cuda.current_stream())
+        handle = dw_ready.cuda_event
+    _lib.check(_lib.slm_loss_bwd_overlap(*args, handle, reserve_sms), "slm_loss_bwd_overlap")
     return dH, dW
 
 

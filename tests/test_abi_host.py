@@ -178,3 +178,19 @@ def test_helper_host_errors(lib):
     assert _lib.slm_target_flatness(A, A, 4, 12, 10, A, A, 1 << 30, None) == 2
     assert _lib.slm_target_flatness(None, A, 4, 16, 10, A, A, 1 << 30, None) == 1
     assert _lib.slm_target_flatness(A, A, 4, 16, 10, A, A, 16, None) == 5
+
+
+def test_overlap_backward_host_errors(lib):
+    def bwd_ov(reserve, **kw):
+        args = dict(kind=0, Hq=A, Hp=None, W=A, labels=A, ignore_index=-100, N=4, d=16, V=32,
+                    grad_tok=None, grad_scale=None, n_valid=None, stats=A, dHq=A, dW=A,
+                    accumulate_dW=0, chunk_tokens=0, workspace=A, ws_bytes=1 << 30,
+                    stream=None, event=None)
+        args.update(kw)
+        return _lib.slm_loss_bwd_overlap(*args.values(), reserve)
+    assert bwd_ov(-1) == 2                   # SLM_ERR_SHAPE: reserve_sms out of range
+    assert bwd_ov(129) == 2
+    assert bwd_ov(8, kind=8) == 4            # then the backward's own checks
+    assert bwd_ov(8, d=12) == 2
+    assert bwd_ov(8, dW=None) == 1
+    assert bwd_ov(8, ws_bytes=16) == 5

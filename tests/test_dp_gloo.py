@@ -64,6 +64,10 @@ def _worker(rank, world, port, kind, outdir, mode):
             valid = (lab != inp.ignore_index).numpy()
             g = np.where(valid, 1.0 / max(int(n_valid_global.item()), 1), 0.0)
             dH, dW = oracle.backward(kind, Hq, W, lab, Hp, g, inp.ignore_index)
+            if mode == "ready3":
+                # The overlapped form's result: (dH, dW, ready); without an event or a
+                # side stream the exchange runs in line.
+                return torch.from_numpy(dH), torch.from_numpy(dW), None
             return torch.from_numpy(dH), torch.from_numpy(dW)
 
         try:
@@ -81,11 +85,12 @@ def _worker(rank, world, port, kind, outdir, mode):
             pass
 
 
-@pytest.mark.parametrize("kind", ["ce", "kl_div", "lk_hybrid"])
-def test_two_rank_data_parallel_matches_whole_batch(kind):
+@pytest.mark.parametrize("kind,mode", [("ce", "ok"), ("kl_div", "ok"), ("lk_hybrid", "ok"),
+                                       ("kl_div", "ready3")])
+def test_two_rank_data_parallel_matches_whole_batch(kind, mode):
     import oracle
     with tempfile.TemporaryDirectory() as d:
-        mp.start_processes(_worker, args=(2, _free_port(), kind, d, "ok"), nprocs=2,
+        mp.start_processes(_worker, args=(2, _free_port(), kind, d, mode), nprocs=2,
                            join=True, start_method="spawn")
         inp = _inputs(kind)
         Hp = None if kind == "ce" else inp.Hp
