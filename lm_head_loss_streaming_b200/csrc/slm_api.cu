@@ -24,36 +24,13 @@
 
 #include "../../include/slm.h"
 #include "slm_internal.h"
+#include "slm_schedule.h"
 
 namespace slm {
 namespace {
 
 constexpr size_t kAlign = 256;
-#ifndef SLM_GROUP_PAIRS
-#define SLM_GROUP_PAIRS 8
-#endif
-#ifndef SLM_MAX_RUNS
-#define SLM_MAX_RUNS 32
-#endif
-// Loose lockstep of the GEMMs' CTA pairs (K blocks per progress step, steps of slack; 0 K
-// blocks = off): V for the GEMMs over the vocabulary (forward, logits gradient, second
-// pass), B for the dH and dW GEMMs.
-#ifndef SLM_SYNC_KB_V
-#define SLM_SYNC_KB_V 16
-#endif
-#ifndef SLM_SYNC_SLACK_V
-#define SLM_SYNC_SLACK_V 2
-#endif
-#ifndef SLM_SYNC_KB_B
-#define SLM_SYNC_KB_B 0
-#endif
-#ifndef SLM_SYNC_SLACK_B
-#define SLM_SYNC_SLACK_B 2
-#endif
-constexpr int kPairM = 2 * kBM;                // M rows of one 2-SM tile
-constexpr int kMaxReserveSms = 128;            // slm_loss_bwd_overlap's reserve_sms, at most
-constexpr int kGroupPairs = SLM_GROUP_PAIRS;   // pair M tiles per raster group
-constexpr int kMaxRuns = SLM_MAX_RUNS;         // vocabulary runs per row, at most
+constexpr int kMaxReserveSms = 128;  // slm_loss_bwd_overlap's reserve_sms, at most
 constexpr long long kTimeoutCycles = 4000000000LL;  // ~2 s at the B200's boost clock
 
 // Test hooks set through slm_debug_set (process-wide, read at every launch).
@@ -65,34 +42,11 @@ DevCtl make_ctl(int* status) {
 }
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
-int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 bool valid_kind(int k) { return k >= SLM_CE && k <= SLM_CE_ARGMAX_P; }
-// Kinds whose forward reads the target logits z_p (all but hard-label CE).
-bool dual_kind(int k) { return k != SLM_CE; }
 // Kinds whose loss needs the final log-sum-exps: a second pass over the vocabulary.
 bool two_pass_kind(int k) {
   return k == SLM_TV || k == SLM_NLA || k == SLM_LK_HYBRID || k == SLM_JSD;
-}
-
-// Forward vocabulary schedule: tiles of `bn` columns, grouped into at most kMaxRuns runs per row
-// (so the per-row partials stay O(N)), each run at least 2048 columns long.  Each run
-// leaves kFwdPartsPerRun partial slots per row (one per epilogue warpgroup).
-struct FwdSched {
-  int bn, num_n, vc, units_n, slots, fields;
-};
-
-FwdSched fwd_sched(int kind, int64_t V) {
-  FwdSched f;
-  f.bn = dual_kind(kind) ? kTileDual : kTileCE;
-  f.num_n = static_cast<int>(ceil_div(V, f.bn));
-  const int min_vc = std::max(1, 2048 / f.bn);
-  f.vc = std::max<int>(min_vc, static_cast<int>(ceil_div(f.num_n, kMaxRuns)));
-  f.vc = std::min(f.vc, f.num_n);
-  f.units_n = static_cast<int>(ceil_div(f.num_n, f.vc));
-  f.slots = f.units_n * kFwdPartsPerRun;
-  f.fields = kind == SLM_CE ? kCEFields : (kind == SLM_CE_ARGMAX_P ? kArgmaxFields : kDualFields);
-  return f;
 }
 
 int64_t default_chunk(int64_t N, int64_t d, int64_t chunk_tokens) {
@@ -188,22 +142,6 @@ bool make_map(CUtensorMap* m, const void* base, int64_t inner, int64_t outer, in
 }
 
 bool misaligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) != 0; }
-
-// Tile schedule of a GEMM with M tiles of `bm` rows (256: a 2-SM CTA pair).
-GemmGeom geom(int64_t M, int64_t Nn, int64_t K, int bn, int vc, int group_m, int bm,
-              int sync_kb, int slack) {
-  GemmGeom g{};
-  g.sync_kb = sync_kb;
-  g.slack = slack;
-  g.num_m = static_cast<int>(ceil_div(M, bm));
-  g.num_n = static_cast<int>(ceil_div(Nn, bn));
-  g.k_blocks = static_cast<int>(ceil_div(K, kBK));
-  g.vc = std::max(1, std::min(vc, g.num_n));
-  g.group_m = std::max(1, std::min(group_m, g.num_m));
-  g.units_n = static_cast<int>(ceil_div(g.num_n, g.vc));
-  g.num_units = g.num_m * g.units_n;
-  return g;
-}
 
 // `backward` selects which pass's workspace needs are checked.
 int common_checks(int kind, const void* Hq, const void* Hp, const void* W, const int32_t* labels,
