@@ -282,7 +282,9 @@ SLM_API int slm_target_flatness(const void* Hp, const void* W, int64_t N, int64_
  * every following launch withhold one internal pipeline release, so that a bounded wait in
  * the kernel runs out: the kernel then records SLM_ERR_TIMEOUT in the workspace status word,
  * lets its own copies and MMAs finish, frees its tensor memory and returns; results of that
- * call are undefined.  fault_mode 0 restores normal operation.  timeout_cycles bounds every
+ * call are undefined.  fault_mode 2 makes the GEMMs' CTA pairs give up their loose
+ * lockstep at the first wait (it only shapes performance: results must not change).
+ * fault_mode 0 restores normal operation.  timeout_cycles bounds every
  * pipeline wait in SM clock cycles (0 = the default of 4e9, about 2 s).  Process-wide;
  * takes effect at the next launch.  Returns SLM_ERR_SHAPE for an invalid mode or bound. */
 SLM_API int slm_debug_set(int fault_mode, long long timeout_cycles);

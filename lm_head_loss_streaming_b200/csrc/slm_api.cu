@@ -753,7 +753,7 @@ int slm_combo_bwd(const float* weights, const void* Hq, const void* Hp, const vo
 }
 
 int slm_debug_set(int fault_mode, long long timeout_cycles) {
-  if (fault_mode < 0 || fault_mode > 1 || timeout_cycles < 0) return SLM_ERR_SHAPE;
+  if (fault_mode < 0 || fault_mode > 2 || timeout_cycles < 0) return SLM_ERR_SHAPE;
   g_fault.store(fault_mode);
   g_timeout.store(timeout_cycles > 0 ? timeout_cycles : kTimeoutCycles);
   return SLM_OK;

@@ -67,7 +67,8 @@ struct GemmGeom {
 struct DevCtl {
   int* status;               // device status word (in the workspace)
   long long timeout_cycles;  // bound of every pipeline wait
-  int fault;                 // test hook: 1 = the epilogue withholds its first accumulator release
+  int fault;                 // test hook: 1 = the epilogue withholds its first accumulator
+                             // release; 2 = the pairs' lockstep waits give up at once
 };
 
 // Forward statistics (pass 1) and the alpha pass (pass 2).

@@ -114,7 +114,9 @@ __device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long
 // finished for the others and returns false, and the caller stops synchronising.
 // Warp-collective.
 __device__ __forceinline__ bool lockstep(const GemmGeom& g, int pair, int npairs,
-                                         uint32_t step) {
+                                         uint32_t step, const DevCtl& ctl) {
+  // Test hook (fault == 2): give up at the first wait, as a pair held back too long would.
+  const long long spin = ctl.fault == 2 ? 0 : kSyncSpinCycles;
   const int lane = threadIdx.x & 31;
   const unsigned long long tag = static_cast<unsigned long long>(g.epoch) << 32;
   if (lane == 0) st_relaxed_u64(&g_pair_progress[pair], tag | step);
@@ -130,7 +132,7 @@ __device__ __forceinline__ bool lockstep(const GemmGeom& g, int pair, int npairs
     }
     mn = __reduce_min_sync(0xffffffffu, mn);
     if (mn >= need) return true;
-    if (__any_sync(0xffffffffu, clock64() - t0 > kSyncSpinCycles)) {
+    if (__any_sync(0xffffffffu, clock64() - t0 >= spin)) {
       if (lane == 0) st_relaxed_u64(&g_pair_progress[pair], tag | 0xffffffffull);
       __syncwarp();
       return false;
@@ -258,7 +260,7 @@ __global__ void __launch_bounds__(64 + 128 * NWG, 1)
       for (int nt = j * g.vc; ok && nt < n_end; ++nt) {
         for (int kb = 0; kb < g.k_blocks; ++kb, ++it) {
           if (sync_on && it % static_cast<uint32_t>(g.sync_kb) == 0)
-            sync_on = lockstep(g, pair, npairs, ++sync_step);
+            sync_on = lockstep(g, pair, npairs, ++sync_step, ctl);
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
           if (!wait_warp(&pc->empty[s], ph ^ 1u, abort, ctl)) {
@@ -1349,9 +1351,19 @@ static cudaError_t launch_pair(const CUtensorMap& a0, const CUtensorMap& a1,
   constexpr size_t kSmem = Cfg::kSmem + (kStage ? 128 + kStage * 4 * NWG : 0);
   static_assert(kSmem <= 232448, "shared memory per CTA");
   auto kern = gemm_pair_kernel<BNI, NSUB, NUM_A, NBUF, NWG, A_MN, B_MN, STAGES, Epi>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(kSmem));
-  if (e != cudaSuccess) return e;
+  cudaError_t e = cudaSuccess;
+  int dev = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  // Per device, once: the shared-memory opt-in and the number of co-resident pairs.  Later
+  // launches make no such calls, so that they can be captured into a CUDA graph.
+  static bool smem_set[64] = {false};
+  if (!smem_set[dev]) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kSmem));
+    if (e != cudaSuccess) return e;
+    smem_set[dev] = true;
+  }
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -1364,9 +1376,6 @@ static cudaError_t launch_pair(const CUtensorMap& a0, const CUtensorMap& a1,
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   static int max_clusters[64] = {0};
-  int dev = 0;
-  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (max_clusters[dev] == 0) {
     int n = 0;
     cfg.gridDim = dim3(2 * 512, 1, 1);

@@ -142,7 +142,9 @@ def test_bwd_output_pointer_errors(lib):
 
 
 def test_debug_hook_arguments(lib):
-    assert _lib.slm_debug_set(2, 0) == 2     # SLM_ERR_SHAPE: unknown mode
+    assert _lib.slm_debug_set(3, 0) == 2     # SLM_ERR_SHAPE: unknown mode
+    assert _lib.slm_debug_set(2, 0) == 0     # lockstep gives up at once
+    assert _lib.slm_debug_set(-1, 0) == 2
     assert _lib.slm_debug_set(0, -1) == 2    # SLM_ERR_SHAPE: negative bound
     assert _lib.slm_debug_set(0, 0) == 0     # back to normal operation
 
