@@ -494,14 +494,7 @@ def run_ours(args):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded; no weights or datasets)",
-        "config": {"workload": args.workload, "kind": kind, "tokens_per_gpu": N, "d": d,
-                   "path": "fused (chunk logits kept)" if args.fused else "recompute",
-                   "V": V, "global_batch_tokens": world * N, "parallelism": f"dp{world}",
-                   "chunk_tokens": args.chunk_tokens or "auto",
-                   "dw_exchange": (None if world == 1 else
-                                   "after the backward" if args.no_overlap else
-                                   "overlapped with the last chunk's dH GEMM"),
-                   "l2": "inputs larger than L2 (W alone is %.2f GB)" % (V * d * 2 / 1e9)},
+        "config": arm_config(args, kind, N, d, V, world),
         "tflops": round(flops_step / (ms_step / 1e3) / 1e12, 1),
         "frac_bf16_peak": round(flops_step / (ms_step / 1e3) / 1e12 / peaks["bf16_tflops"], 4),
         "frac_bf16_peak_8NVd": round(base_flops / (ms_step / 1e3) / 1e12 / peaks["bf16_tflops"], 4),
@@ -529,6 +522,18 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+def arm_config(args, kind, N, d, V, world):
+    """The workload description both arms print (the reference arm times a sample of it)."""
+    return {"workload": args.workload, "kind": kind, "tokens_per_gpu": N, "d": d,
+            "path": "fused (chunk logits kept)" if args.fused else "recompute",
+            "V": V, "global_batch_tokens": world * N, "parallelism": f"dp{world}",
+            "chunk_tokens": args.chunk_tokens or "auto",
+            "dw_exchange": (None if world == 1 else
+                            "after the backward" if args.no_overlap else
+                            "overlapped with the last chunk's dH GEMM"),
+            "l2": "inputs larger than L2 (W alone is %.2f GB)" % (V * d * 2 / 1e9)}
+
+
 def run_reference(args):
     """The oracle as it stands, on host cores, on a bounded sample of the same workload."""
     rank = int(os.environ.get("RANK", "0"))
@@ -547,8 +552,8 @@ def run_reference(args):
         "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(t * 1e3, 1), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": args.workload, "kind": kind, "tokens_per_step": rows,
-                   "d": cfg["d"], "V": cfg["V"]},
+        "config": arm_config(args, kind, args.tokens or cfg["N"], cfg["d"], cfg["V"],
+                             int(os.environ.get("WORLD_SIZE", "1"))),
         "cpu_baseline": {"value": round(tps, 3), "unit": "tokens/s", "cores": cores,
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": round(tps, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
