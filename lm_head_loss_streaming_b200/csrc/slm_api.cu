@@ -357,7 +357,7 @@ int slm_loss_fwd(int kind, const void* Hq, const void* Hp, const void* W, const 
       if (kind == SLM_CE_ARGMAX_P)
         SLM_TRY_CUDA(launch_fwd_argmax(tHq, tHp, tW, g, p, ctl, s));
       else
-        SLM_TRY_CUDA(launch_fwd_dual(tHq, tHp, tW, g, p, ctl, s));
+        SLM_TRY_CUDA(launch_fwd_dual(tHq, tHp, tW, g, p, ctl, kind == SLM_RKL, s));
     }
     SLM_TRY_CUDA(launch_combine(kind, 1, part, f.slots, zy, labels, ignore_index, N, V,
                                 loss_tok, alpha_tok, stats, blk_sum, blk_cnt, status, s));
@@ -605,7 +605,7 @@ int slm_loss_fwd_bwd(int kind, const void* Hq, const void* Hp, const void* W,
       if (argmax_kind)
         SLM_TRY_CUDA(launch_fwd_argmax(tHq, tHp, tW, g, p, ctl, s));
       else
-        SLM_TRY_CUDA(launch_fwd_dual(tHq, tHp, tW, g, p, ctl, s));
+        SLM_TRY_CUDA(launch_fwd_dual(tHq, tHp, tW, g, p, ctl, kind == SLM_RKL, s));
     }
     SLM_TRY_CUDA(launch_combine(kind, 1, part, f.slots, zy, labels, ignore_index, rows, V,
                                 loss_tok, alpha_tok, stats, blk_sum, blk_cnt, status, s, c0, N));

@@ -116,9 +116,9 @@ struct DwParams {
 int sm_count();
 cudaError_t launch_fwd_ce(const CUtensorMap& tH, const CUtensorMap& tW, const GemmGeom& g,
                           const FwdParams& p, const DevCtl& c, cudaStream_t s);
-cudaError_t launch_fwd_dual(const CUtensorMap& tHq, const CUtensorMap& tHp,
-                            const CUtensorMap& tW, const GemmGeom& g, const FwdParams& p,
-                            const DevCtl& c, cudaStream_t s);
+cudaError_t launch_fwd_dual(const CUtensorMap& tHq, const CUtensorMap& tHp, const CUtensorMap& tW,
+                            const GemmGeom& g, const FwdParams& p, const DevCtl& c, bool rkl,
+                            cudaStream_t s);
 cudaError_t launch_fwd_argmax(const CUtensorMap& tHq, const CUtensorMap& tHp,
                               const CUtensorMap& tW, const GemmGeom& g, const FwdParams& p,
                               const DevCtl& c, cudaStream_t s);

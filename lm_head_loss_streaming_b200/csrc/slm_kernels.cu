@@ -564,7 +564,9 @@ __device__ __forceinline__ void EpiFwdCE::store_rows(const Params& p, float* buf
 // both the draft (q, accumulator 0) and the target (p, accumulator 1): online max and sum
 // of exp; plus A = sum_v 2^(z_p log2e - m_p) (z_p - z_q), rescaled whenever m_p grows, and
 // B = sum_v 2^(z_q log2e - m_q) (z_q - z_p), rescaled whenever m_q grows.
-struct EpiFwdDual {
+// ACC selects the divergence accumulators: 1 = forward KL (A), 2 = reverse KL (B), 3 = both.
+template <int ACC>
+struct EpiFwdDualT {
   using Params = FwdParams;
   static constexpr int kStageBytesPerWarp = 4096;
   float* stage;  // this warp's staging buffer (fused path stores)
@@ -586,13 +588,13 @@ struct EpiFwdDual {
     if (xq > mq) {
       const float r = exp2f(mq - xq);
       sq *= r;
-      B *= r;
+      if (ACC & 2) B *= r;
       mq = xq;
     }
     if (xp > mp) {
       const float r = exp2f(mp - xp);
       sp *= r;
-      A *= r;
+      if (ACC & 1) A *= r;
       mp = xp;
     }
     if (mq == -INFINITY || mp == -INFINITY) return;
@@ -604,12 +606,12 @@ struct EpiFwdDual {
       sp += e;
       if (TAIL) {
         // Masked columns are -inf in both: their weights are 0 and their difference NaN.
-        if (e > 0.f) A = fmaf(e, vp[i] - vq[i], A);
-        if (eq > 0.f) B = fmaf(eq, vq[i] - vp[i], B);
+        if ((ACC & 1) && e > 0.f) A = fmaf(e, vp[i] - vq[i], A);
+        if ((ACC & 2) && eq > 0.f) B = fmaf(eq, vq[i] - vp[i], B);
       } else {
         const float dpq = vp[i] - vq[i];
-        A = fmaf(e, dpq, A);
-        B = fmaf(-eq, dpq, B);
+        if (ACC & 1) A = fmaf(e, dpq, A);
+        if (ACC & 2) B = fmaf(-eq, dpq, B);
       }
     }
   }
@@ -650,6 +652,8 @@ struct EpiFwdDual {
     base[5 * p.N] = B;
   }
 };
+
+using EpiFwdDual = EpiFwdDualT<3>;
 
 // CE against argmax p (forward): online max / sum of exp of the draft logits, and the
 // target's running argmax over the slot's columns (the first, i.e. lowest, column wins
@@ -894,7 +898,7 @@ struct EpiDz {
       lp = p.stats[p.N + n];
       lp2 = lp * kLog2e;
       if (p.kind == kKL) {
-        ck = g;
+        ck = g;  // mode 0: dz = g (q - p)
       } else if (p.kind == kRKL) {
         mode = 1;
         ck = g;
@@ -904,6 +908,7 @@ struct EpiDz {
         ck = g;
         S = p.stats[4 * p.N + n];  // T
       } else {
+        mode = 3;
         const float al = p.stats[3 * p.N + n];
         S = p.stats[4 * p.N + n];
         if (p.kind == kTV) {
@@ -926,6 +931,13 @@ struct EpiDz {
     if (DUAL) {
       {
         if (mode == 0) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float qv = exp2f(fmaf(vq[i], kLog2e, -lq2));
+            const float pv = exp2f(fmaf(vp[i], kLog2e, -lp2));
+            vq[i] = ck * (qv - pv);
+          }
+        } else if (mode == 3) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             const float qv = exp2f(fmaf(vq[i], kLog2e, -lq2));
@@ -1408,9 +1420,13 @@ cudaError_t launch_fwd_ce(const CUtensorMap& tH, const CUtensorMap& tW, const Ge
   return launch_pair<256, 2, 1, 1, 2, false, false, 4, EpiFwdCE>(tH, tH, tW, g, p, c, s);
 }
 cudaError_t launch_fwd_dual(const CUtensorMap& tHq, const CUtensorMap& tHp, const CUtensorMap& tW,
-                            const GemmGeom& g, const FwdParams& p, const DevCtl& c,
+                            const GemmGeom& g, const FwdParams& p, const DevCtl& c, bool rkl,
                             cudaStream_t s) {
-  return launch_pair<256, 1, 2, 1, 2, false, false, 4, EpiFwdDual>(tHq, tHp, tW, g, p, c, s);
+  // Reverse KL needs only the accumulator B, every other kind only A.
+  if (rkl)
+    return launch_pair<256, 1, 2, 1, 2, false, false, 4, EpiFwdDualT<2>>(tHq, tHp, tW, g, p, c,
+                                                                         s);
+  return launch_pair<256, 1, 2, 1, 2, false, false, 4, EpiFwdDualT<1>>(tHq, tHp, tW, g, p, c, s);
 }
 cudaError_t launch_fwd_argmax(const CUtensorMap& tHq, const CUtensorMap& tHp,
                               const CUtensorMap& tW, const GemmGeom& g, const FwdParams& p,
