@@ -431,6 +431,8 @@ static int loss_bwd(int kind, const void* Hq, const void* Hp, const void* W,
                              SLM_SYNC_KB_V, SLM_SYNC_SLACK_V);
     DzParams pz{dz_kind, dz_labels, ignore_index, c0, rows, N, V, stats, grad_tok, grad_scale,
                 n_valid, dz, ldz, ComboW{}};
+    // The epilogue stores dZ in 32-row x 64-column blocks through this map.
+    if (!make_map(&pz.dz_map, dz, V, rows, ldz, 64, 32)) return SLM_ERR_CUDA;
     if (!dual_kind(dz_kind)) {
       SLM_TRY_CUDA(launch_dz_ce(tHq, tW_k, gz, pz, ctl, s));
     } else {

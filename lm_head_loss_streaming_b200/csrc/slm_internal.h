@@ -99,6 +99,8 @@ struct DzParams {
   __nv_bfloat16* dz;  // [rows][ldz]
   int64_t ldz;
   ComboW cw;          // weighted combination (EpiDzCombo only)
+  CUtensorMap dz_map;  // dz as bf16 [rows][V] (row stride ldz), box 64 x 32, 128-byte
+                       // swizzle: the store map of EpiDz
 };
 
 struct DhParams {

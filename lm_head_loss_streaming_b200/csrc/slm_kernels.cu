@@ -34,6 +34,7 @@
 
 #include <algorithm>
 #include <atomic>
+#include <utility>
 
 #include "slm_internal.h"
 #include "sm100.cuh"
@@ -189,13 +190,24 @@ struct EpiStageBytes<E, decltype(void(E::kStageBytesPerWarp))> {
   static constexpr int value = E::kStageBytesPerWarp;
 };
 
+// Epilogues with asynchronous work of their own (bulk stores) declare finish(), which the
+// kernel calls once after the epilogue's last tile.
+template <class E, class = void>
+struct EpiHasFinish {
+  static constexpr bool value = false;
+};
+template <class E>
+struct EpiHasFinish<E, decltype(std::declval<E&>().finish())> {
+  static constexpr bool value = true;
+};
+
 template <int BNI, int NSUB, int NUM_A, int NBUF, int NWG, bool A_MN, bool B_MN, int STAGES,
           class Epi>
 __global__ void __launch_bounds__(64 + 128 * NWG, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0,
                      const __grid_constant__ CUtensorMap tmA1,
                      const __grid_constant__ CUtensorMap tmB, const GemmGeom g,
-                     const typename Epi::Params ep, const DevCtl ctl) {
+                     const __grid_constant__ typename Epi::Params ep, const DevCtl ctl) {
   using C = PairCfg<BNI, NSUB, NUM_A, NBUF, NWG, A_MN, B_MN, STAGES>;
   constexpr int kTileN = C::kTileN;
   constexpr int kSliceN = C::kSliceN;
@@ -385,9 +397,10 @@ __global__ void __launch_bounds__(64 + 128 * NWG, 1)
     const uint32_t tempty_leader1 = mapa_shared(smem_u32(&pc->tempty[1]), 0);
     Epi epi;
     if constexpr (EpiStageBytes<Epi>::value > 0) {
-      // Per-warp staging buffers live after the control block.
+      // Per-warp staging buffers live after the control block, 1024-byte aligned so that
+      // their rows follow the 128-byte swizzle pattern of the tensor maps.
       uint8_t* st = reinterpret_cast<uint8_t*>(
-          (reinterpret_cast<uintptr_t>(pc + 1) + 127) & ~static_cast<uintptr_t>(127));
+          (reinterpret_cast<uintptr_t>(pc + 1) + 1023) & ~static_cast<uintptr_t>(1023));
       epi.stage = reinterpret_cast<float*>(st + (warp - 2) * EpiStageBytes<Epi>::value);
     }
     uint32_t t = 0;
@@ -418,6 +431,7 @@ __global__ void __launch_bounds__(64 + 128 * NWG, 1)
       if (!ok) break;
       epi.unit_end(ep, row0, j * NWG + wg, row);
     }
+    if constexpr (EpiHasFinish<Epi>::value) epi.finish();
   }
 
   // Neither CTA leaves while the other may still signal its barriers or use its TMEM.
@@ -871,6 +885,11 @@ __device__ __forceinline__ void store_bf16_row32(__nv_bfloat16* dst, const float
 template <bool DUAL>
 struct EpiDz {
   using Params = DzParams;
+  // Per warp: a 32-row x 64-column bf16 block of dZ, laid out as the dZ tensor map's
+  // 128-byte swizzle expects (16-byte chunk k of row r at position k ^ (r % 8)), written to
+  // the chunk buffer by one TMA store.
+  static constexpr int kStageBytesPerWarp = 4096;
+  float* stage;
   float lq, lp, lq2, lp2, g, ck, cm, S;
   int32_t lab;
   int mode;
@@ -976,21 +995,53 @@ struct EpiDz {
   }
 
   template <int TN>
-  __device__ __forceinline__ void tile(const Params& p, uint32_t tb, int, int64_t n0, int c0,
-                                       int c1, int) {
-    __nv_bfloat16* out = p.dz + lrow * p.ldz + n0;
+  __device__ __forceinline__ void tile(const Params& p, uint32_t tb, int row0, int64_t n0,
+                                       int c0, int c1, int row) {
+    const int lane = threadIdx.x & 31;
+    uint8_t* srow = reinterpret_cast<uint8_t*>(stage) + lane * 128;
+    const int wrow0 = row0 + row - lane;  // chunk row of this warp's first row
 #pragma unroll 1
-    for (int c = c0; c < c1; c += 32) {
-      float vq[32], vp[32];
-      tmem_ld32(tb + c, vq);
-      if (DUAL) tmem_ld32(tb + TN + c, vp);
-      tmem_ld_wait();
-      apply(vq, vp, n0 + c);
-      if (row_ok && n0 + c < p.V) store_bf16_row32(out + c, vq, n0 + c, p.V);
+    for (int c = c0; c < c1; c += 64) {
+      // The staging block is free once the previous block's store has read it.
+      if (lane == 0) bulk_wait_read_all();
+      __syncwarp();
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        float vq[32], vp[32];
+        tmem_ld32(tb + c + 32 * h, vq);
+        if (DUAL) tmem_ld32(tb + TN + c + 32 * h, vp);
+        tmem_ld_wait();
+        apply(vq, vp, n0 + c + 32 * h);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          uint32_t w[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const __nv_bfloat162 b2 =
+                __floats2bfloat162_rn(vq[8 * k + 2 * e], vq[8 * k + 2 * e + 1]);
+            w[e] = *reinterpret_cast<const uint32_t*>(&b2);
+          }
+          *reinterpret_cast<uint4*>(srow + (((4 * h + k) ^ (lane & 7)) << 4)) =
+              make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      // Columns >= V and rows beyond the chunk fall outside the map and are not written.
+      if (lane == 0 && n0 + c < p.V) {
+        tma_store_2d(&p.dz_map, stage, static_cast<int32_t>(n0 + c), wrow0);
+        bulk_commit();
+      }
     }
   }
 
   __device__ __forceinline__ void unit_end(const Params&, int, int, int) {}
+
+  // Every store has landed before the kernel's shared memory goes away.
+  __device__ __forceinline__ void finish() {
+    if ((threadIdx.x & 31) == 0) bulk_wait_all();
+    __syncwarp();
+  }
 };
 
 // dH rows of the chunk: fp32 accumulator -> bf16.
@@ -1360,7 +1411,7 @@ static cudaError_t launch_pair(const CUtensorMap& a0, const CUtensorMap& a1,
                                const typename Epi::Params& p, const DevCtl& c, cudaStream_t s) {
   using Cfg = PairCfg<BNI, NSUB, NUM_A, NBUF, NWG, A_MN, B_MN, STAGES>;
   constexpr size_t kStage = EpiStageBytes<Epi>::value;
-  constexpr size_t kSmem = Cfg::kSmem + (kStage ? 128 + kStage * 4 * NWG : 0);
+  constexpr size_t kSmem = Cfg::kSmem + (kStage ? 1024 + kStage * 4 * NWG : 0);
   static_assert(kSmem <= 232448, "shared memory per CTA");
   auto kern = gemm_pair_kernel<BNI, NSUB, NUM_A, NBUF, NWG, A_MN, B_MN, STAGES, Epi>;
   cudaError_t e = cudaSuccess;
