@@ -141,6 +141,21 @@ bool make_map(CUtensorMap* m, const void* base, int64_t inner, int64_t outer, in
   return r == CUDA_SUCCESS;
 }
 
+// The same for an fp32 matrix (the fused path's kept logits).
+bool make_map_f32(CUtensorMap* m, const void* base, int64_t inner, int64_t outer, int64_t ld,
+                  int box_inner, int box_outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(outer)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 4};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(box_inner), static_cast<cuuint32_t>(box_outer)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool misaligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) != 0; }
 
 // `backward` selects which pass's workspace needs are checked.
@@ -599,6 +614,9 @@ int slm_loss_fwd_bwd(int kind, const void* Hq, const void* Hp, const void* W,
                              SLM_SYNC_KB_V, SLM_SYNC_SLACK_V);
     FwdParams p{labels ? labels + c0 : nullptr, ignore_index, rows, V, part, zy, nullptr, 0,
                 lq, (dual_kind(kind) && !argmax_kind) ? lp : nullptr, ldl};
+    // The epilogue stores the kept logits in 32 x 32 blocks through these maps.
+    if (!make_map_f32(&p.lq_map, lq, V, rows, ldl, 32, 32)) return SLM_ERR_CUDA;
+    if (p.lp_out && !make_map_f32(&p.lp_map, lp, V, rows, ldl, 32, 32)) return SLM_ERR_CUDA;
     if (!dual_kind(kind)) {
       SLM_TRY_CUDA(launch_fwd_ce(tHq, tW, g, p, ctl, s));
     } else {

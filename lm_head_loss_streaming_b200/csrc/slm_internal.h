@@ -83,6 +83,8 @@ struct FwdParams {
   float* lq_out;       // fused path: store the fp32 draft logits here ([N][ldl]), or NULL
   float* lp_out;       // fused path: store the fp32 target logits here, or NULL
   int64_t ldl;         // leading dimension of the stored logits (V rounded up to 4)
+  CUtensorMap lq_map;  // fused path: store maps of lq_out / lp_out as fp32 [N][V] (row
+  CUtensorMap lp_map;  // stride ldl), box 32 x 32, 128-byte swizzle
 };
 
 // Logits-gradient tile (backward recompute + dZ epilogue).

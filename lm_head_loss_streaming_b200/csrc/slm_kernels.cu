@@ -463,29 +463,33 @@ __device__ __forceinline__ void mask_tail(float (&v)[32], int64_t col0, int64_t 
     if (col0 + i >= V) v[i] = -INFINITY;
 }
 
-// Fused path: store the warp's 32 rows x 32 columns of fp32 logits (each lane holds its
-// row's 32 values).  The block goes through the warp's 4 KB staging buffer with the 16-byte
-// chunk index XOR-swizzled by the row (conflict-free writes and reads), so that each global
-// store instruction writes four full 128-byte row segments instead of 32 scattered pieces.
-// Columns >= V land in the row padding (the leading dimension is V rounded up to 4, so every
-// float4 that starts below V fits).  Warp-collective.
-__device__ __forceinline__ void store_block32_f32(float* stage, const float (&v)[32],
-                                                  float* gdst, int64_t ldl, int nrows,
-                                                  int64_t col0, int64_t V) {
+// Fused path: this warp's 32 rows x 32 columns of fp32 logits (each lane holds its row's
+// 32 values; `grow` is the lane's row) go to the warp's 4 KB staging block in the 128-byte
+// swizzle layout of the store map (16-byte chunk k of row r at position k ^ (r % 8)), and
+// from there to global memory with one TMA bulk store.  Columns >= V and rows beyond the
+// launch's rows fall outside the map and are not written.  The staging block is rewritten
+// only once the previous store has read it.  Warp-collective.
+__device__ __forceinline__ void stage_store_f32(float* stage, const CUtensorMap* map,
+                                                const float (&v)[32], int64_t col0,
+                                                int64_t grow) {
   const int lane = threadIdx.x & 31;
+  if (lane == 0) bulk_wait_read_all();
+  __syncwarp();
   float4* srow = reinterpret_cast<float4*>(stage + lane * 32);
 #pragma unroll
   for (int k = 0; k < 8; ++k)
     srow[k ^ (lane & 7)] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+  fence_proxy_async_smem();
   __syncwarp();
-  const int k = lane & 7;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int r = i * 4 + (lane >> 3);
-    const float4 x = reinterpret_cast<const float4*>(stage + r * 32)[k ^ (r & 7)];
-    if (r < nrows && col0 + 4 * k < V)
-      *reinterpret_cast<float4*>(gdst + static_cast<int64_t>(r) * ldl + 4 * k) = x;
+  if (lane == 0) {
+    tma_store_2d(map, stage, static_cast<int32_t>(col0), static_cast<int32_t>(grow));
+    bulk_commit();
   }
+}
+
+// Waits for the warp's outstanding bulk stores (the end of an epilogue that issued some).
+__device__ __forceinline__ void finish_bulk_stores() {
+  if ((threadIdx.x & 31) == 0) bulk_wait_all();
   __syncwarp();
 }
 
@@ -521,7 +525,8 @@ struct EpiFwdCE {
       tmem_ld32(tb + c, v);
       tmem_ld_wait();
       if (n0 + c + 32 > p.V) mask_tail(v, n0 + c, p.V);
-      if (p.lq_out) store_rows(p, p.lq_out, v, n0 + c);
+      if (p.lq_out && n0 + c < p.V)
+        stage_store_f32(stage, &p.lq_map, v, n0 + c, grow - (threadIdx.x & 31));
       if (static_cast<uint64_t>(rel - c) < 32u) {
         const int o = static_cast<int>(rel - c);
 #pragma unroll
@@ -546,8 +551,7 @@ struct EpiFwdCE {
     }
   }
 
-  __device__ __forceinline__ void store_rows(const Params& p, float* buf, const float (&v)[32],
-                                             int64_t col0) const;
+  __device__ __forceinline__ void finish() { finish_bulk_stores(); }
 
   __device__ __forceinline__ void unit_end(const Params& p, int, int slot, int) {
     if (!row_ok) return;
@@ -556,23 +560,6 @@ struct EpiFwdCE {
     if (has_zy) p.zy[grow] = zyv;
   }
 };
-
-// The rows of a warp are consecutive: lane 0 holds row grow - lane.  Store the warp's
-// 32 x 32 block of one logits buffer at columns [col0, col0 + 32).
-template <class E>
-__device__ __forceinline__ void epi_store_rows(const E& e, const FwdParams& p, float* buf,
-                                               const float (&v)[32], int64_t col0) {
-  const int lane = threadIdx.x & 31;
-  const int64_t r0 = e.grow - lane;
-  const int64_t left = p.N - r0;
-  const int nrows = left < 32 ? static_cast<int>(left) : 32;
-  store_block32_f32(e.stage, v, buf + r0 * p.ldl + col0, p.ldl, nrows, col0, p.V);
-}
-
-__device__ __forceinline__ void EpiFwdCE::store_rows(const Params& p, float* buf,
-                                                     const float (&v)[32], int64_t col0) const {
-  epi_store_rows(*this, p, buf, v, col0);
-}
 
 // KL / RKL forward (and the first pass of the alpha losses and of JSD): per row and for
 // both the draft (q, accumulator 0) and the target (p, accumulator 1): online max and sum
@@ -644,16 +631,20 @@ struct EpiFwdDualT {
         mask_tail(vq, n0 + c, p.V);
         mask_tail(vp, n0 + c, p.V);
       }
-      if (p.lq_out) {
-        epi_store_rows(*this, p, p.lq_out, vq, n0 + c);
-        epi_store_rows(*this, p, p.lp_out, vp, n0 + c);
-      }
+      // Fused path: the draft block's store overlaps this chunk's arithmetic, which reads
+      // vq and vp only; the target block follows.
+      const bool store = p.lq_out && n0 + c < p.V;
+      const int64_t wrow = grow - (threadIdx.x & 31);
+      if (store) stage_store_f32(stage, &p.lq_map, vq, n0 + c, wrow);
       if (tail)
         chunk<true>(vq, vp);
       else
         chunk<false>(vq, vp);
+      if (store && p.lp_out) stage_store_f32(stage, &p.lp_map, vp, n0 + c, wrow);
     }
   }
+
+  __device__ __forceinline__ void finish() { finish_bulk_stores(); }
 
   __device__ __forceinline__ void unit_end(const Params& p, int, int slot, int) {
     if (!row_ok) return;
@@ -703,7 +694,8 @@ struct EpiFwdArgmax {
         mask_tail(vq, n0 + c, p.V);
         mask_tail(vp, n0 + c, p.V);
       }
-      if (p.lq_out) epi_store_rows(*this, p, p.lq_out, vq, n0 + c);
+      if (p.lq_out && n0 + c < p.V)
+        stage_store_f32(stage, &p.lq_map, vq, n0 + c, grow - (threadIdx.x & 31));
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
         if (vp[i] > pmax) {
@@ -738,6 +730,8 @@ struct EpiFwdArgmax {
     base[3 * p.N] = __int_as_float(pidx);
     base[4 * p.N] = zqa;
   }
+
+  __device__ __forceinline__ void finish() { finish_bulk_stores(); }
 };
 
 // Second pass of the alpha losses: with the final log-sum-exps L_q and L_p known,
