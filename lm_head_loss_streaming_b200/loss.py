@@ -309,8 +309,35 @@ class StreamingLMHeadLoss(torch.autograd.Function):
         return dH, dW.to(weight.dtype), None, None, None, None, None
 
 
+class StreamingLMHeadLossFused(torch.autograd.Function):
+    """The same loss through the fused single call (``slm_loss_fwd_bwd``): the gradients
+    of the mean are computed in the forward, with each chunk's logits kept instead of
+    recomputed, and the backward only scales them by the upstream gradient."""
+
+    @staticmethod
+    def forward(ctx, hidden, weight, labels, target_hidden, kind, ignore_index, chunk_tokens):
+        fwd, dH, dW = lm_head_loss_fwd_bwd(kind, hidden, weight, labels, target_hidden,
+                                           ignore_index, chunk_tokens=chunk_tokens)
+        ctx.dH, ctx.dW, ctx.wdtype = dH, dW, weight.dtype
+        return fwd.loss_mean.reshape(())
+
+    @staticmethod
+    def backward(ctx, grad_out):
+        dH, dW = ctx.dH, ctx.dW
+        ctx.dH = ctx.dW = None
+        g = grad_out.to(torch.float32)
+        return ((dH.float() * g).to(dH.dtype), (dW * g).to(ctx.wdtype),
+                None, None, None, None, None)
+
+
 def streaming_lm_head_loss(hidden, weight, labels=None, target_hidden=None, kind="ce",
-                           ignore_index=IGNORE_INDEX, chunk_tokens=0):
-    """Mean loss over valid rows; differentiable w.r.t. ``hidden`` and ``weight``."""
-    return StreamingLMHeadLoss.apply(hidden, weight, labels, target_hidden, _kind_id(kind),
-                                     ignore_index, chunk_tokens)
+                           ignore_index=IGNORE_INDEX, chunk_tokens=0, fused=False):
+    """Mean loss over valid rows; differentiable w.r.t. ``hidden`` and ``weight``.
+
+    ``fused=False`` recomputes each chunk's logits in the backward (memory bounded by one
+    bf16 chunk of logit gradients).  ``fused=True`` computes the gradients in the forward
+    with the fused single call (each chunk's fp32 logits kept, 1.2-1.7x faster, a larger
+    workspace) and holds them until the backward."""
+    fn = StreamingLMHeadLossFused if fused else StreamingLMHeadLoss
+    return fn.apply(hidden, weight, labels, target_hidden, _kind_id(kind), ignore_index,
+                    chunk_tokens)

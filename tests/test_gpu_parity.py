@@ -155,12 +155,13 @@ def test_large_logits_finite():
     _compare(inp, "ce", what="large logits ce")
 
 
-def test_autograd_wrapper():
+@pytest.mark.parametrize("fused", [False, True])
+def test_autograd_wrapper(fused):
     from lm_head_loss_streaming_b200 import streaming_lm_head_loss
     inp = synthetic.make("kl_div", 200, 64, 1200, w_std=0.05, seed=11)
     Hq = inp.Hq.cuda().requires_grad_(True)
     W = inp.W.cuda().requires_grad_(True)
-    loss = streaming_lm_head_loss(Hq, W, None, inp.Hp.cuda(), kind="kl_div")
+    loss = streaming_lm_head_loss(Hq, W, None, inp.Hp.cuda(), kind="kl_div", fused=fused)
     (2.0 * loss).backward()
     r = oracle_fwd_bwd(inp, "kl_div")
     assert abs(loss.item() - r["loss"]) <= 2e-3 * abs(r["loss"])
