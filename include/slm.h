@@ -178,6 +178,15 @@ SLM_API int slm_loss_bwd_overlap(int kind, const void* Hq, const void* Hp, const
                  int64_t chunk_tokens, void* workspace, size_t ws_bytes, void* stream,
                  void* dw_ready_event, int reserve_sms);
 
+/* Chunk-size rule ("Choosing the chunk size": the largest chunk that keeps the loss path's
+ * memory peak below the next peak of the training step, e.g. a transformer block's).  Returns
+ * the largest chunk_tokens, a multiple of 128 (of 256 with fused != 0), whose workspace
+ * (slm_workspace_bytes, or slm_fused_workspace_bytes with fused != 0) fits in budget_bytes;
+ * a value >= N means every row fits in one chunk.  Returns 0 when not even the smallest
+ * chunk fits, or on invalid arguments.  Host only; no device is touched. */
+SLM_API int64_t slm_chunk_for_budget(int kind, int64_t N, int64_t d, int64_t V,
+                                     size_t budget_bytes, int fused);
+
 /* Synchronises `stream`, then returns and clears the device status word of `workspace`:
  * SLM_OK, SLM_ERR_LABEL_RANGE or SLM_ERR_TIMEOUT (the first found), or SLM_ERR_CUDA if
  * the stream reported an error.  Every slm_loss_fwd / slm_loss_bwd call also clears the

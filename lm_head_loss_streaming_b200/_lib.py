@@ -47,6 +47,7 @@ SIGNATURES = {
     "slm_loss_bwd_overlap": (_INT, [_INT, _P, _P, _P, _P, _I32, _I64, _I64, _I64,
                                     _P, _P, _P, _P, _P, _P, _INT, _I64, _P, _SZ, _P,
                                     _P, _INT]),
+    "slm_chunk_for_budget": (_I64, [_INT, _I64, _I64, _I64, _SZ, _INT]),
     "slm_device_status": (_INT, [_P, _P]),
     "slm_debug_set": (_INT, [_INT, ctypes.c_longlong]),
     "slm_fused_workspace_bytes": (_SZ, [_INT, _I64, _I64, _I64, _I64]),
@@ -144,6 +145,11 @@ def slm_loss_bwd_overlap(kind, Hq, Hp, W, labels, ignore_index, N, d, V, grad_to
                                        stats, dHq, dW, int(accumulate_dW), int(chunk_tokens),
                                        workspace, int(ws_bytes), stream, dw_ready_event,
                                        int(reserve_sms))
+
+
+def slm_chunk_for_budget(kind, N, d, V, budget_bytes, fused=False):
+    return load().slm_chunk_for_budget(int(kind), int(N), int(d), int(V), int(budget_bytes),
+                                       1 if fused else 0)
 
 
 def slm_device_status(workspace, stream):

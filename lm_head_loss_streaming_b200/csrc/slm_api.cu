@@ -559,6 +559,27 @@ size_t slm_fused_workspace_bytes(int kind, int64_t N, int64_t d, int64_t V,
   return fused_layout(kind, N, V, chunk_tokens).total;
 }
 
+int64_t slm_chunk_for_budget(int kind, int64_t N, int64_t d, int64_t V, size_t budget_bytes,
+                             int fused) {
+  if (!valid_kind(kind) || N <= 0 || d <= 0 || V <= 0 || (d % 8) != 0) return 0;
+  const int64_t step = fused ? 256 : kBM;
+  auto ws = [&](int64_t c) {
+    return fused ? slm_fused_workspace_bytes(kind, N, d, V, c)
+                 : slm_workspace_bytes(kind, N, d, V, c);
+  };
+  if (ws(step) > budget_bytes) return 0;
+  // The workspace grows with the chunk: bisect over multiples of `step` up to all N rows.
+  int64_t lo = 1, hi = ceil_div(N, step);
+  while (lo < hi) {
+    const int64_t mid = (lo + hi + 1) / 2;
+    if (ws(mid * step) <= budget_bytes)
+      lo = mid;
+    else
+      hi = mid - 1;
+  }
+  return lo * step;
+}
+
 int slm_loss_fwd_bwd(int kind, const void* Hq, const void* Hp, const void* W,
                      const int32_t* labels, int32_t ignore_index, int64_t N, int64_t d,
                      int64_t V, const float* grad_tok, const float* grad_scale, float* loss_tok,

@@ -247,6 +247,12 @@ def lm_head_loss_fwd_bwd(kind, hidden, weight, labels=None, target_hidden=None,
     return out, dH, dW
 
 
+def chunk_for_budget(kind, N, d, V, budget_bytes, fused=False):
+    """The largest token chunk whose workspace fits in ``budget_bytes`` (0 if none): set the
+    budget to the next memory peak of the training step so the loss path stays below it."""
+    return int(_lib.slm_chunk_for_budget(_kind_id(kind), N, d, V, budget_bytes, fused))
+
+
 def align_labels(tokens, shift, loss_mask=None, seq_ids=None, ignore_index=IGNORE_INDEX):
     """Labels of a draft head that predicts ``shift`` tokens ahead, aligned before chunking
     (through ``slm_align_labels``).  tokens int32 [B, S] (CUDA); loss_mask bool/uint8 [B, S]

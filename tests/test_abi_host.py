@@ -196,3 +196,26 @@ def test_overlap_backward_host_errors(lib):
     assert bwd_ov(8, d=12) == 2
     assert bwd_ov(8, dW=None) == 1
     assert bwd_ov(8, ws_bytes=16) == 5
+
+
+@pytest.mark.parametrize("fused", [False, True])
+def test_chunk_for_budget_is_the_largest_chunk_that_fits(lib, fused):
+    """The chunk-size rule: the largest chunk whose workspace stays within the budget."""
+    ws = _lib.slm_fused_workspace_bytes if fused else _lib.slm_workspace_bytes
+    step = 256 if fused else 128
+    for kind, N, d, V in ((_lib.SLM_KL, 16384, 4096, 128256), (_lib.SLM_CE, 8192, 2048, 128256),
+                          (_lib.SLM_TV, 1000, 64, 3000)):
+        for budget in (1 << 28, 1 << 30, 3 << 30, 1 << 40):
+            c = _lib.slm_chunk_for_budget(kind, N, d, V, budget, fused)
+            if c == 0:
+                assert ws(kind, N, d, V, step) > budget
+                continue
+            assert c % step == 0
+            assert ws(kind, N, d, V, c) <= budget
+            if c < N:
+                assert ws(kind, N, d, V, c + step) > budget
+        # An unlimited budget takes every row in one chunk.
+        assert _lib.slm_chunk_for_budget(kind, N, d, V, 1 << 60, fused) >= N
+    assert _lib.slm_chunk_for_budget(_lib.SLM_KL, 1024, 12, 100, 1 << 30, fused) == 0  # d % 8
+    assert _lib.slm_chunk_for_budget(9, 1024, 16, 100, 1 << 30, fused) == 0
+    assert _lib.slm_chunk_for_budget(_lib.SLM_KL, 16384, 4096, 128256, 1, fused) == 0
