@@ -311,15 +311,27 @@ def run_ours(args):
                                       reserve_sms=args.reserve_sms)
             return gh, gw, ready
 
+        def fused_call(scale=None):
+            return lm_head_loss_fwd_bwd(kind, Hq_, W_, lab_, Hp_, inp.ignore_index,
+                                        grad_scale=scale, chunk_tokens=args.chunk_tokens,
+                                        workspace=ws, out=res, dH=dH, dW=dW)
+
+        def count():
+            if lab_ is None:
+                return torch.full((1,), Hq_.shape[0], dtype=torch.int64, device=dev)
+            return (lab_ != inp.ignore_index).sum().reshape(1)
+
         def step(ev=None):
             if args.fused:
-                # One call: forward, logits kept per chunk, backward.  (The data-parallel
-                # exchange needs the global count before the backward, so --fused is 1 GPU.)
+                # One call: forward, logits kept per chunk, backward.  With several ranks the
+                # valid counts are summed first and passed in as the gradient's scale
+                # (lm_head_loss_streaming_b200.dp.fused_fwd_bwd).
                 if ev is not None:
                     ev[0].record(stream)
-                lm_head_loss_fwd_bwd(kind, Hq_, W_, lab_, Hp_, inp.ignore_index,
-                                     chunk_tokens=args.chunk_tokens, workspace=ws, out=res,
-                                     dH=dH, dW=dW)
+                if world > 1:
+                    dp.fused_fwd_bwd(count, fused_call)
+                else:
+                    fused_call()
                 if ev is not None:
                     ev[1].record(stream)
             elif world > 1:

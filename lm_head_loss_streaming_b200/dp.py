@@ -77,6 +77,30 @@ def fwd_bwd(fwd: Callable[[], Any], bwd: Callable[[Any, torch.Tensor], tuple],
     return DPResult(loss_mean, loss_sum, n_valid, dH, dW)
 
 
+def fused_fwd_bwd(count: Callable[[], torch.Tensor],
+                  fused: Callable[[torch.Tensor], tuple], group=None) -> DPResult:
+    """One data-parallel step through a single-call forward + backward.
+
+    The single call (``slm_loss_fwd_bwd``) forms the gradient of this rank's mean loss, i.e.
+    it divides by the rank's own valid count, scaled by ``grad_scale``.  So the counts are
+    summed first: ``count()`` returns this rank's valid-row count (int64 [1]), and
+    ``fused(scale)`` is called with scale = n_local / n_global (float32 [1]), which turns the
+    local mean's gradient into the global mean's.  It returns (res, dH, dW) with
+    ``res.loss_sum``.  dW and the loss sum are then summed across ranks, as in ``fwd_bwd``.
+    """
+    n_local = count().reshape(1).to(torch.int64)
+    n_valid = n_local.clone()
+    dist.all_reduce(n_valid, group=group)
+    scale = (n_local.to(torch.float64) / n_valid.clamp_min(1).to(torch.float64)).to(torch.float32)
+    res, dH, dW = fused(scale)
+    dist.all_reduce(dW, group=group)
+    loss_sum = res.loss_sum.clone()
+    dist.all_reduce(loss_sum, group=group)
+    den = n_valid.clamp_min(1).to(loss_sum.dtype)
+    loss_mean = torch.where(n_valid > 0, loss_sum / den, torch.zeros_like(loss_sum))
+    return DPResult(loss_mean, loss_sum, n_valid, dH, dW)
+
+
 _COMM_STREAMS = {}
 
 
@@ -116,3 +140,25 @@ def cuda_step(kind, hidden, weight, labels=None, target_hidden=None, ignore_inde
         return gh, gw, ready
 
     return fwd_bwd(_fwd, _bwd, group, comm_stream_for(hidden.device) if overlap else None)
+
+
+def cuda_step_fused(kind, hidden, weight, labels=None, target_hidden=None, ignore_index=-100,
+                    group=None, chunk_tokens=0, workspace=None, out=None, dH=None, dW=None):
+    """Data-parallel step over the fused single call (each chunk's logits kept).
+
+    The rank's valid count is taken from its labels (rows whose label is not ignore_index;
+    every row without labels) before the call.  A CE label outside [0, V) is masked by the
+    library and flagged in its status word, but counted here: such a batch is invalid."""
+    from .loss import lm_head_loss_fwd_bwd
+
+    def _count():
+        if labels is None:
+            return torch.full((1,), hidden.shape[0], dtype=torch.int64, device=hidden.device)
+        return (labels != ignore_index).sum().reshape(1)
+
+    def _fused(scale):
+        return lm_head_loss_fwd_bwd(kind, hidden, weight, labels, target_hidden, ignore_index,
+                                    grad_scale=scale, chunk_tokens=chunk_tokens,
+                                    workspace=workspace, out=out, dH=dH, dW=dW)
+
+    return fused_fwd_bwd(_count, _fused, group)

@@ -70,8 +70,23 @@ def _worker(rank, world, port, kind, outdir, mode):
                 return torch.from_numpy(dH), torch.from_numpy(dW), None
             return torch.from_numpy(dH), torch.from_numpy(dW)
 
+        def count():
+            return torch.tensor([int((lab != inp.ignore_index).sum())], dtype=torch.int64)
+
+        def fused(scale):
+            # A single call whose gradient is that of the local mean, scaled by `scale`.
+            res = fwd()
+            n_local = max(int(res.n_valid.item()), 1)
+            valid = (lab != inp.ignore_index).numpy()
+            g = np.where(valid, float(scale.item()) / n_local, 0.0)
+            dH, dW = oracle.backward(kind, Hq, W, lab, Hp, g, inp.ignore_index)
+            return res, torch.from_numpy(dH), torch.from_numpy(dW)
+
         try:
-            r = dp.fwd_bwd(fwd, bwd)
+            if mode == "fused":
+                r = dp.fused_fwd_bwd(count, fused)
+            else:
+                r = dp.fwd_bwd(fwd, bwd)
         except Exception as e:  # noqa: BLE001
             with open(os.path.join(outdir, f"err{rank}.txt"), "w") as f:
                 f.write(type(e).__name__)
@@ -86,7 +101,8 @@ def _worker(rank, world, port, kind, outdir, mode):
 
 
 @pytest.mark.parametrize("kind,mode", [("ce", "ok"), ("kl_div", "ok"), ("lk_hybrid", "ok"),
-                                       ("kl_div", "ready3")])
+                                       ("kl_div", "ready3"), ("ce", "fused"),
+                                       ("kl_div", "fused")])
 def test_two_rank_data_parallel_matches_whole_batch(kind, mode):
     import oracle
     with tempfile.TemporaryDirectory() as d:
@@ -100,8 +116,14 @@ def test_two_rank_data_parallel_matches_whole_batch(kind, mode):
             r = np.load(os.path.join(d, f"rank{rank}.npz"))
             assert int(r["n_valid"][0]) == ref["n_valid"]
             assert abs(float(r["loss"][0]) - ref["loss"]) <= 1e-12 * max(1.0, abs(ref["loss"]))
-            assert np.allclose(r["dW"], rdW, rtol=1e-10, atol=1e-14)
-            assert np.allclose(r["dH"], rdH[r["rows"]], rtol=1e-10, atol=1e-14)
+            if mode == "fused":
+                # The fused form passes its scale as the library's float32 grad_scale:
+                # relative-to-max-norm agreement at float32 resolution.
+                for got, want in ((r["dW"], rdW), (r["dH"], rdH[r["rows"]])):
+                    assert np.abs(got - want).max() <= 1e-6 * np.abs(want).max()
+            else:
+                assert np.allclose(r["dW"], rdW, rtol=1e-10, atol=1e-14)
+                assert np.allclose(r["dH"], rdH[r["rows"]], rtol=1e-10, atol=1e-14)
 
 
 def test_rank_that_leaves_makes_the_other_fail_not_hang():

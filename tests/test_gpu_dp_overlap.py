@@ -113,3 +113,29 @@ def test_nccl_step_with_overlap_equals_plain_step_and_oracle(kind):
     sh, sw = tie_slack(inp, kind)
     assert_grad_close(h1.double().cpu().numpy(), rh, "dp dH", sh)
     assert_grad_close(w1.double().cpu().numpy(), rw, "dp dW", sw)
+
+
+@pytest.mark.parametrize("kind", ["ce", "kl_div"])
+def test_nccl_fused_step_matches_oracle(kind):
+    """The data-parallel step over the fused single call (valid counts summed first and
+    passed in as the gradient's scale), as a one-rank NCCL group."""
+    inp = synthetic.make(kind, 700, 128, 3000, w_std=0.05, ignore_frac=0.1, seed=76)
+    Hq, W, Hp, lab = _dev(inp)
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{_free_port()}", rank=0,
+                            world_size=1, timeout=timedelta(seconds=60),
+                            device_id=torch.device("cuda", 0))
+    try:
+        r = dp.cuda_step_fused(kind, Hq, W, lab, Hp, inp.ignore_index, chunk_tokens=256)
+        torch.cuda.synchronize()
+        loss, n, h, w = r.loss_mean.item(), r.n_valid.item(), r.dH.clone(), r.dW.clone()
+    finally:
+        dist.destroy_process_group()
+    ref = oracle.forward(kind, inp.Hq, inp.W, inp.labels, inp.Hp, inp.ignore_index)
+    assert n == ref["n_valid"]
+    mean = ref["loss_sum"] / ref["n_valid"]
+    assert abs(loss - mean) <= 2e-3 * abs(mean)
+    valid = inp.labels.numpy() != inp.ignore_index
+    gt = np.where(valid, 1.0 / ref["n_valid"], 0.0)
+    rh, rw = oracle.backward(kind, inp.Hq, inp.W, inp.labels, inp.Hp, gt, inp.ignore_index)
+    assert_grad_close(h.double().cpu().numpy(), rh, "dp fused dH")
+    assert_grad_close(w.double().cpu().numpy(), rw, "dp fused dW")
