@@ -13,13 +13,17 @@
 //               multicast tcgen05.commit;
 //   warps 2..   epilogue (both CTAs): one or two warpgroups, one thread per tile row, each
 //               warpgroup over its share of the tile's columns, reading TMEM with
-//               tcgen05.ld and applying the fused epilogue.
+//               tcgen05.ld and applying the fused epilogue.  Epilogues that write wide
+//               outputs stage each warp's block in swizzled shared memory and hand it to
+//               one TMA bulk store.
+// Work units (M tile, run of N tiles[, K slice]) go to the pairs round robin; the pairs of
+// the GEMMs over the vocabulary keep a loose lockstep so that W tiles are shared in L2.
 // The epilogues are what make the path streaming ("Training speculative decoders:
 // removing the logits and attention bottlenecks", "Streaming Cross Entropy" and
 // "Backward pass"): logits tiles live only in TMEM and registers.
 //   EpiFwdCE    online row max / sum of exp and the label logit          (CE forward)
-//   EpiFwdDual  the same for target and draft plus the forward- and reverse-KL
-//               accumulators                                             (KL / RKL forward,
+//   EpiFwdDualT the same for target and draft plus the forward-KL (A) and/or reverse-KL
+//               (B) accumulator                                          (KL / RKL forward,
 //               first pass of the alpha losses and of JSD)
 //   EpiFwdArgmax draft log-sum-exp plus the target's running argmax      (CE against argmax p)
 //   EpiAlpha    alpha = sum min(p, q) and S = sum_{q<p} q                 (second pass)
@@ -27,6 +31,9 @@
 //   EpiDz       the logits gradient, rounded to bf16 into the chunk buffer (backward)
 //   EpiDh       dH chunk rows (bf16)                                      (dH = dZ W)
 //   EpiDw       fp32 read-add-write of disjoint dW tiles, no atomics      (dW += dZ^T H)
+//   EpiFwdUnion, EpiPass2Union, EpiDzCombo   the same for weighted combinations
+//   EpiFlat     sum of exp and of its square                             (target flatness)
+// In the fused single call the forward epilogues also store the chunk's fp32 logits.
 // Every pipeline wait is bounded: on expiry the kernel records kFlagTimeout, lets its own
 // copies and MMAs finish, frees TMEM and returns.
 
