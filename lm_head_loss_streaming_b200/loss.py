@@ -33,18 +33,69 @@ def _kind_id(kind):
         raise ValueError(f"unknown loss kind {kind!r}; expected one of {list(_lib.KIND)}")
 
 
-def _check_inputs(kind, hidden, weight, labels, target_hidden):
+def _check_inputs(kind, hidden, weight, labels, target_hidden, grad_tok=None):
+    """The kernels see raw pointers and the sizes taken from ``hidden`` and ``weight``: every
+    tensor must be on the current CUDA device with the layout and extent those sizes imply,
+    or the kernels would read past it.  Raises ValueError before anything is launched."""
     for name, t in (("hidden", hidden), ("weight", weight), ("target_hidden", target_hidden)):
         if t is None:
             continue
-        if not t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous():
-            raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor")
-    if labels is not None and (labels.dtype != torch.int32 or not labels.is_contiguous()):
-        raise ValueError("labels must be a contiguous int32 tensor")
+        if not t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous() or t.dim() != 2:
+            raise ValueError(f"{name} must be a contiguous 2-D bf16 CUDA tensor")
+    N, d = hidden.shape
+    if weight.shape[1] != d:
+        raise ValueError(f"weight is {tuple(weight.shape)}; expected [V, {d}]")
+    if target_hidden is not None and target_hidden.shape != hidden.shape:
+        raise ValueError(f"target_hidden is {tuple(target_hidden.shape)}; expected {(N, d)}")
+    if labels is not None:
+        if (not labels.is_cuda or labels.dtype != torch.int32 or not labels.is_contiguous()
+                or labels.shape != (N,)):
+            raise ValueError(f"labels must be a contiguous int32 CUDA tensor of shape ({N},)")
+    if grad_tok is not None:
+        if (not grad_tok.is_cuda or grad_tok.dtype != torch.float32
+                or not grad_tok.is_contiguous() or grad_tok.shape != (N,)):
+            raise ValueError(f"grad_tok must be a contiguous float32 CUDA tensor of shape ({N},)")
+    dev = torch.cuda.current_device()
+    for name, t in (("hidden", hidden), ("weight", weight), ("target_hidden", target_hidden),
+                    ("labels", labels), ("grad_tok", grad_tok)):
+        if t is not None and t.device.index != dev:
+            raise ValueError(f"{name} is on {t.device}, not on the current device cuda:{dev}")
+    if kind is None:       # weighted combinations: the library checks what each term needs
+        return
     if kind != _lib.SLM_CE and target_hidden is None:
         raise ValueError("distribution losses need target_hidden (H_p)")
     if kind == _lib.SLM_CE and labels is None:
         raise ValueError("ce needs labels")
+
+
+def _check_out(name, t, shape, dtype):
+    """A caller-provided output buffer must have exactly the extent the kernels write."""
+    if t is None:
+        return
+    if (not t.is_cuda or t.dtype != dtype or not t.is_contiguous() or tuple(t.shape) != shape
+            or t.device.index != torch.cuda.current_device()):
+        raise ValueError(f"{name} must be a contiguous {dtype} tensor of shape {shape} on the "
+                         f"current CUDA device")
+
+
+def _check_fwd_out(out, k, N):
+    """Caller-provided forward results must match the sizes the kernels write."""
+    _check_out("out.loss_mean", out.loss_mean, (1,), torch.float32)
+    _check_out("out.loss_sum", out.loss_sum, (1,), torch.float64)
+    _check_out("out.n_valid", out.n_valid, (1,), torch.int64)
+    _check_out("out.loss_tok", out.loss_tok, (N,), torch.float32)
+    _check_out("out.alpha_tok", out.alpha_tok, (N,), torch.float32)
+    _check_out("out.stats", out.stats, (_lib.slm_stats_floats(k), N), torch.float32)
+
+
+def _check_grads(dH, dW, N, d, V):
+    _check_out("dH", dH, (N, d), torch.bfloat16)
+    _check_out("dW", dW, (V, d), torch.float32)
+
+
+def _check_scale(grad_scale):
+    if grad_scale is not None:
+        _check_out("grad_scale", grad_scale, (1,), torch.float32)
 
 
 @dataclass
@@ -88,6 +139,7 @@ def lm_head_loss_fwd(kind, hidden, weight, labels=None, target_hidden=None,
             torch.empty(nk, N, dtype=torch.float32, device=dev),
             workspace)
     else:
+        _check_fwd_out(out, k, N)
         out.workspace = workspace
     st = _lib.slm_loss_fwd(k, _ptr(hidden), _ptr(target_hidden), _ptr(weight), _ptr(labels),
                            ignore_index, N, d, V, _ptr(out.loss_tok), _ptr(out.alpha_tok),
@@ -110,9 +162,14 @@ def lm_head_loss_bwd(fwd: FwdResult, hidden, weight, labels=None, target_hidden=
     that a reduction of dW on another stream can overlap it.  The results are the same.
     Returns (dH bf16 [N, d], dW fp32 [V, d])."""
     k = fwd.kind
+    _check_inputs(k, hidden, weight, labels, target_hidden, grad_tok)
     N, d = hidden.shape
     V = weight.shape[0]
     dev = hidden.device
+    if tuple(fwd.stats.shape) != (_lib.slm_stats_floats(k), N):
+        raise ValueError("fwd does not come from a forward over these hidden states")
+    _check_grads(dH, dW, N, d, V)
+    _check_scale(grad_scale)
     if dH is None:
         dH = torch.empty(N, d, dtype=torch.bfloat16, device=dev)
     if dW is None:
@@ -162,6 +219,7 @@ def lm_head_loss_combo_fwd(weights, hidden, weight, labels=None, target_hidden=N
     """Forward of a weighted combination {kind: weight} through ``slm_combo_fwd``."""
     for k in weights:
         _kind_id(k)
+    _check_inputs(None, hidden, weight, labels, target_hidden)
     N, d = hidden.shape
     V = weight.shape[0]
     dev = hidden.device
@@ -187,9 +245,14 @@ def lm_head_loss_combo_bwd(fwd: ComboResult, hidden, weight, labels=None, target
                            normalize=True, dH=None, dW=None, accumulate_dW=False,
                            chunk_tokens=0):
     """Backward of a weighted combination through ``slm_combo_bwd``."""
+    _check_inputs(None, hidden, weight, labels, target_hidden, grad_tok)
     N, d = hidden.shape
     V = weight.shape[0]
     dev = hidden.device
+    if tuple(fwd.stats.shape) != (_lib.SLM_COMBO_STATS, N):
+        raise ValueError("fwd does not come from a forward over these hidden states")
+    _check_grads(dH, dW, N, d, V)
+    _check_scale(grad_scale)
     if dH is None:
         dH = torch.empty(N, d, dtype=torch.bfloat16, device=dev)
     if dW is None:
@@ -215,10 +278,12 @@ def lm_head_loss_fwd_bwd(kind, hidden, weight, labels=None, target_hidden=None,
     kept instead of recomputed).  Returns (FwdResult, dH, dW); the gradient is that of the
     mean loss, scaled by grad_tok / grad_scale when given."""
     k = _kind_id(kind)
-    _check_inputs(k, hidden, weight, labels, target_hidden)
+    _check_inputs(k, hidden, weight, labels, target_hidden, grad_tok)
     N, d = hidden.shape
     V = weight.shape[0]
     dev = hidden.device
+    _check_grads(dH, dW, N, d, V)
+    _check_scale(grad_scale)
     need = max(_lib.slm_fused_workspace_bytes(k, N, d, V, chunk_tokens), 256)
     if workspace is None or workspace.numel() < need:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
@@ -232,6 +297,7 @@ def lm_head_loss_fwd_bwd(kind, hidden, weight, labels=None, target_hidden=None,
             torch.empty(_lib.slm_stats_floats(k), N, dtype=torch.float32, device=dev),
             workspace)
     else:
+        _check_fwd_out(out, k, N)
         out.workspace = workspace
     if dH is None:
         dH = torch.empty(N, d, dtype=torch.bfloat16, device=dev)
@@ -260,6 +326,12 @@ def align_labels(tokens, shift, loss_mask=None, seq_ids=None, ignore_index=IGNOR
     if tokens.dtype != torch.int32 or not tokens.is_cuda or tokens.dim() != 2:
         raise ValueError("tokens must be a 2-D int32 CUDA tensor")
     B, S = tokens.shape
+    for name, t in (("loss_mask", loss_mask), ("seq_ids", seq_ids)):
+        if t is not None and (not t.is_cuda or t.device != tokens.device
+                              or tuple(t.shape) != (B, S)):
+            raise ValueError(f"{name} must be a CUDA tensor of shape {(B, S)} on {tokens.device}")
+    if tokens.device.index != torch.cuda.current_device():
+        raise ValueError(f"tokens is on {tokens.device}, not on the current CUDA device")
     tokens = tokens.contiguous()
     mask = None if loss_mask is None else loss_mask.to(torch.uint8).contiguous()
     seq = None if seq_ids is None else seq_ids.to(torch.int32).contiguous()
