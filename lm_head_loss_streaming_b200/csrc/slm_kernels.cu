@@ -2065,6 +2065,9 @@ template <bool DUAL>
 __global__ void __launch_bounds__(256)
     logits_dz_kernel(const DzParams p, const float* __restrict__ lq,
                      const float* __restrict__ lp, int64_t ldl) {
+  // One block per row.  Each pass covers 32 * blockDim consecutive columns as 8 groups of
+  // 4 per thread, the lanes of a warp on consecutive groups, so that every load reads and
+  // every store writes one contiguous span per warp (512 and 256 bytes).
   const int64_t r = blockIdx.x;
   EpiDz<DUAL> e;
   e.unit_begin(p, 0, static_cast<int>(r));
@@ -2072,15 +2075,17 @@ __global__ void __launch_bounds__(256)
   const float* rq = lq + r * ldl;
   const float* rp = DUAL ? lp + r * ldl : lq;
   __nv_bfloat16* out = p.dz + r * p.ldz;
-  for (int64_t c = static_cast<int64_t>(threadIdx.x) * 32; c < p.V; c += 32 * blockDim.x) {
+  const int64_t span = 4 * static_cast<int64_t>(blockDim.x);
+  for (int64_t base = 4 * static_cast<int64_t>(threadIdx.x); base < p.V; base += 8 * span) {
     float vq[32], vp[32];
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
-      if (c + 4 * k < p.V) {
-        const float4 a = *reinterpret_cast<const float4*>(rq + c + 4 * k);
+      const int64_t c = base + k * span;
+      if (c < p.V) {  // a float4 that starts below V lies within the row (ldl % 4 == 0)
+        const float4 a = *reinterpret_cast<const float4*>(rq + c);
         vq[4 * k] = a.x, vq[4 * k + 1] = a.y, vq[4 * k + 2] = a.z, vq[4 * k + 3] = a.w;
         if (DUAL) {
-          const float4 b = *reinterpret_cast<const float4*>(rp + c + 4 * k);
+          const float4 b = *reinterpret_cast<const float4*>(rp + c);
           vp[4 * k] = b.x, vp[4 * k + 1] = b.y, vp[4 * k + 2] = b.z, vp[4 * k + 3] = b.w;
         }
       } else {
@@ -2088,8 +2093,33 @@ __global__ void __launch_bounds__(256)
         for (int j = 0; j < 4; ++j) vq[4 * k + j] = vp[4 * k + j] = -INFINITY;
       }
     }
-    e.apply(vq, vp, c);
-    store_bf16_row32(out + c, vq, c, p.V);
+    if (DUAL) {
+      e.apply(vq, vp, 0);  // elementwise: no column enters the divergences' formulas
+    } else {
+      // CE: the same formula as the GEMM epilogue's, with each value's own column.
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int64_t c = base + k * span + j;
+          const float qv = exp2f(fmaf(vq[4 * k + j], kLog2e, -e.lq2));
+          vq[4 * k + j] = e.g * (qv - (c == e.lab ? 1.f : 0.f));
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int64_t c = base + k * span;
+      if (c + 4 <= p.V) {
+        const __nv_bfloat162 lo = __floats2bfloat162_rn(vq[4 * k], vq[4 * k + 1]);
+        const __nv_bfloat162 hi = __floats2bfloat162_rn(vq[4 * k + 2], vq[4 * k + 3]);
+        uint2 w;
+        w.x = *reinterpret_cast<const uint32_t*>(&lo);
+        w.y = *reinterpret_cast<const uint32_t*>(&hi);
+        *reinterpret_cast<uint2*>(out + c) = w;
+      } else {
+        for (int j = 0; j < 4 && c + j < p.V; ++j) out[c + j] = __float2bfloat16_rn(vq[4 * k + j]);
+      }
+    }
   }
 }
 
