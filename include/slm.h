@@ -182,8 +182,9 @@ SLM_API int slm_loss_bwd_overlap(int kind, const void* Hq, const void* Hp, const
  * memory peak below the next peak of the training step, e.g. a transformer block's).  Returns
  * the largest chunk_tokens, a multiple of 128 (of 256 with fused != 0), whose workspace
  * (slm_workspace_bytes, or slm_fused_workspace_bytes with fused != 0) fits in budget_bytes;
- * a value >= N means every row fits in one chunk.  Returns 0 when not even the smallest
- * chunk fits, or on invalid arguments.  Host only; no device is touched. */
+ * the result never exceeds N: a value equal to N means every row fits in one chunk (it is
+ * then not a multiple of 128 when N is not).  Returns 0 when not even the smallest chunk
+ * fits, or on invalid arguments.  Host only; no device is touched. */
 SLM_API int64_t slm_chunk_for_budget(int kind, int64_t N, int64_t d, int64_t V,
                                      size_t budget_bytes, int fused);
 
@@ -192,6 +193,46 @@ SLM_API int64_t slm_chunk_for_budget(int kind, int64_t N, int64_t d, int64_t V,
  * the stream reported an error.  Every slm_loss_fwd / slm_loss_bwd call also clears the
  * word when it starts, so the status describes the most recent call. */
 SLM_API int slm_device_status(const void* workspace, void* stream);
+
+/* Number of valid rows, counted the way the kernels mask them ("Streaming Cross Entropy":
+ * the mean divides by the number of valid, non-masked tokens of the whole batch).  A row is
+ * valid when its label is not ignore_index and, for SLM_CE, lies in [0, V); with labels
+ * NULL (every kind but SLM_CE) all N rows are valid.  Data-parallel training sums this
+ * count over the ranks before the backward, so that each rank divides by the global count
+ * and out-of-range CE labels are left out of it exactly as the kernels leave them out.
+ *   labels   int32 [N] device, or NULL (required for SLM_CE when N > 0).
+ *   n_valid  int64 [1] device, overwritten.
+ * Asynchronous on `stream`.  Returns SLM_ERR_KIND, SLM_ERR_SHAPE (N < 0, V <= 0, or either
+ * >= 2^31) or SLM_ERR_NULL on bad arguments, before anything is enqueued. */
+SLM_API int slm_count_valid(int kind, const int32_t* labels, int32_t ignore_index,
+                            int64_t N, int64_t V, int64_t* n_valid, void* stream);
+
+/* Kernel-class timing.  The pages define no counterpart: this is the library's own
+ * measurement hook, used to report each GEMM of the path against its roofline.
+ * slm_trace_enable(1) makes every following kernel launch of the library (any entry point,
+ * any host thread) record a CUDA event on its stream before and after it; slm_trace_enable(0)
+ * stops recording.  slm_trace_read waits for the recorded events, adds up their elapsed
+ * times per kernel class and clears the record:
+ *   ms[c]        milliseconds spent in class c since the last read (launch to launch end
+ *                on its stream);
+ *   launches[c]  number of launches of class c.
+ * The classes (index c) are SLM_TRACE_*.  n_classes may be smaller than SLM_TRACE_CLASSES
+ * (the rest is not reported).  The events are host-side CUDA resources created on first
+ * use and reused; no device memory is allocated.  At most 65536 launches are recorded
+ * between reads; further ones are dropped and slm_trace_read then returns
+ * SLM_ERR_WORKSPACE (the sums cover the recorded ones).  Returns SLM_ERR_CUDA if an event
+ * failed, SLM_ERR_NULL for NULL outputs.  Do not trace inside a stream capture. */
+#define SLM_TRACE_FWD_GEMM 0     /* forward statistics GEMMs (pass 1, flatness)          */
+#define SLM_TRACE_PASS2_GEMM 1   /* second-pass GEMMs (alpha and S, JSD halves)          */
+#define SLM_TRACE_DZ_GEMM 2      /* backward logits recompute + logits-gradient GEMMs    */
+#define SLM_TRACE_DH_GEMM 3      /* dH = dZ W                                            */
+#define SLM_TRACE_DW_GEMM 4      /* dW (+)= dZ^T H                                       */
+#define SLM_TRACE_BWD_FUSED 5    /* the persistent fused backward (dZ, dH, dW together)  */
+#define SLM_TRACE_LOGITS_ROW 6   /* row kernels over kept logits (slm_loss_fwd_bwd)      */
+#define SLM_TRACE_ROW 7          /* combines, reductions, counts, alignment              */
+#define SLM_TRACE_CLASSES 8
+SLM_API int slm_trace_enable(int on);
+SLM_API int slm_trace_read(double* ms, int64_t* launches, int n_classes);
 
 /* Fused forward + backward in one call ("Backward pass": for each token chunk, compute the
  * logits, the loss and the gradients; the chunk's logits plus gradient buffer bounds the
@@ -314,7 +355,9 @@ SLM_API int slm_debug_set(int fault_mode, long long timeout_cycles);
  *   device_flags  int [1] device memory or NULL: receives the device status bits of this
  *                 call (0 = none; 1 = a CE label outside [0, V); 2 = a wait ran out of time).
  * The first call on each device looks up the array's device address (and may load the
- * library's device code), so make it before any stream capture.  Every call shares the one
+ * library's device code), so make it before any stream capture.  The address is kept per
+ * device and CUDA context: after the context is torn down and re-created (cudaDeviceReset),
+ * the next call looks it up again, and that call too should come before any capture.  Every call shares the one
  * array: calls that overlap on the GPU race and must be serialised by the caller.  Nothing
  * is allocated.  The backward still takes a caller workspace (slm_loss_bwd). */
 SLM_API int slm_loss_fwd_noalloc(int kind, const void* Hq, const void* Hp, const void* W,

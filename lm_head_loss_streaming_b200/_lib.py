@@ -63,7 +63,14 @@ SIGNATURES = {
                              _P, _P, _P, _P, _P, _P, _INT, _I64, _P, _SZ, _P]),
     "slm_loss_fwd_noalloc": (_INT, [_INT, _P, _P, _P, _P, _I32, _I64, _I64, _I64,
                                     _P, _P, _P, _P, _P, _P, _P, _P]),
+    "slm_count_valid": (_INT, [_INT, _P, _I32, _I64, _I64, _P, _P]),
+    "slm_trace_enable": (_INT, [_INT]),
+    "slm_trace_read": (_INT, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_I64), _INT]),
 }
+
+# Kernel classes of slm_trace_read, in order.
+TRACE_CLASSES = ("fwd_gemm", "pass2_gemm", "dz_gemm", "dh_gemm", "dw_gemm", "bwd_fused",
+                 "logits_row", "row")
 
 
 class SLMError(RuntimeError):
@@ -229,3 +236,21 @@ def slm_flatness_workspace_bytes(N, d, V):
 def slm_target_flatness(Hp, W, N, d, V, flat, workspace, ws_bytes, stream):
     return load().slm_target_flatness(Hp, W, int(N), int(d), int(V), flat, workspace,
                                       int(ws_bytes), stream)
+
+
+def slm_count_valid(kind, labels, ignore_index, N, V, n_valid, stream):
+    return load().slm_count_valid(int(kind), labels, int(ignore_index), int(N), int(V),
+                                  n_valid, stream)
+
+
+def slm_trace_enable(on):
+    return load().slm_trace_enable(1 if on else 0)
+
+
+def slm_trace_read():
+    """(status, {class name: (ms, launches)}) since the previous read."""
+    n = len(TRACE_CLASSES)
+    ms = (ctypes.c_double * n)()
+    cnt = (_I64 * n)()
+    st = load().slm_trace_read(ms, cnt, n)
+    return st, {name: (ms[i], int(cnt[i])) for i, name in enumerate(TRACE_CLASSES)}

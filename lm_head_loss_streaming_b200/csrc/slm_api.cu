@@ -21,6 +21,8 @@
 #include <algorithm>
 #include <atomic>
 #include <mutex>
+#include <utility>
+#include <vector>
 
 #include "../../include/slm.h"
 #include "slm_internal.h"
@@ -30,6 +32,18 @@ namespace slm {
 namespace {
 
 constexpr size_t kAlign = 256;
+// Kernel classes of slm_trace_read (the order of SLM_TRACE_* in slm.h).
+enum TraceClass : int {
+  kTrFwdGemm = 0,    // forward statistics GEMMs (pass 1; flatness)
+  kTrPass2Gemm = 1,  // second-pass GEMMs (alpha / S, JSD halves)
+  kTrDzGemm = 2,     // backward logits recompute + logits-gradient GEMMs
+  kTrDhGemm = 3,     // dH = dZ W
+  kTrDwGemm = 4,     // dW (+)= dZ^T H
+  kTrBwdFused = 5,   // the persistent fused backward (dZ, dH and dW in one launch)
+  kTrLogitsRow = 6,  // row kernels over kept logits (fused single call)
+  kTrRow = 7,        // combines, reductions, counts, alignment
+  kTraceClasses = 8
+};
 constexpr int kMaxReserveSms = 128;  // slm_loss_bwd_overlap's reserve_sms, at most
 constexpr long long kTimeoutCycles = 4000000000LL;  // ~2 s at the B200's boost clock
 
@@ -40,6 +54,81 @@ std::atomic<long long> g_timeout{kTimeoutCycles};
 DevCtl make_ctl(int* status) {
   return DevCtl{status, g_timeout.load(), g_fault.load()};
 }
+
+// Kernel-class timing (slm_trace_enable / slm_trace_read).  While enabled, every kernel
+// launch of the library is bracketed by two CUDA events on its stream; reading
+// synchronises on the recorded events and sums their elapsed times per class.  Events
+// come from a per-device pool that is created on first use and reused; nothing is
+// recorded (one relaxed atomic load per launch) while tracing is off.
+constexpr size_t kMaxTraceRecords = size_t(1) << 16;
+std::atomic<int> g_trace_on{0};
+std::mutex g_trace_mu;
+struct TraceRec {
+  int cls;
+  cudaEvent_t a, b;
+};
+std::vector<TraceRec> g_trace_recs;
+std::vector<std::pair<int, cudaEvent_t>> g_trace_pool;  // (device, free event)
+long long g_trace_dropped = 0;
+
+// A free event of the current device (under g_trace_mu), or nullptr.
+cudaEvent_t trace_event() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+  for (size_t i = 0; i < g_trace_pool.size(); ++i) {
+    if (g_trace_pool[i].first == dev) {
+      cudaEvent_t e = g_trace_pool[i].second;
+      g_trace_pool[i] = g_trace_pool.back();
+      g_trace_pool.pop_back();
+      return e;
+    }
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+  return e;
+}
+
+void trace_release(cudaEvent_t e) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  g_trace_pool.emplace_back(dev, e);
+}
+
+// Brackets the launches of one kernel class in a scope.
+class Trace {
+ public:
+  Trace(int cls, cudaStream_t s) : cls_(cls), s_(s) {
+    if (!g_trace_on.load(std::memory_order_relaxed)) return;
+    std::lock_guard<std::mutex> lock(g_trace_mu);
+    if (g_trace_recs.size() >= kMaxTraceRecords) {
+      ++g_trace_dropped;
+      return;
+    }
+    a_ = trace_event();
+    if (a_ && cudaEventRecord(a_, s_) != cudaSuccess) {
+      trace_release(a_);
+      a_ = nullptr;
+    }
+  }
+  ~Trace() {
+    if (!a_) return;
+    std::lock_guard<std::mutex> lock(g_trace_mu);
+    cudaEvent_t b = trace_event();
+    if (b && cudaEventRecord(b, s_) == cudaSuccess) {
+      g_trace_recs.push_back(TraceRec{cls_, a_, b});
+      return;
+    }
+    trace_release(a_);
+    if (b) trace_release(b);
+  }
+  Trace(const Trace&) = delete;
+  Trace& operator=(const Trace&) = delete;
+
+ private:
+  int cls_;
+  cudaStream_t s_;
+  cudaEvent_t a_ = nullptr;
+};
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -299,6 +388,13 @@ FusedLayout fused_layout(int kind, int64_t N, int64_t V, int64_t chunk_tokens) {
     if ((expr) != cudaSuccess) return SLM_ERR_CUDA; \
   } while (0)
 
+// A kernel launch of the given trace class on the function's stream `s`.
+#define SLM_LAUNCH(cls, expr)                         \
+  do {                                                \
+    Trace slm_trace_scope_(cls, s);                   \
+    if ((expr) != cudaSuccess) return SLM_ERR_CUDA;   \
+  } while (0)
+
 }  // namespace
 }  // namespace slm
 
@@ -366,29 +462,29 @@ int slm_loss_fwd(int kind, const void* Hq, const void* Hp, const void* W, const 
     FwdParams p{labels, ignore_index, N, V, part, zy, stats, kind == SLM_JSD ? 1 : 0,
                 nullptr, nullptr, 0};
     if (!dual_kind(kind)) {
-      SLM_TRY_CUDA(launch_fwd_ce(tHq, tW, g, p, ctl, s));
+      SLM_LAUNCH(kTrFwdGemm, launch_fwd_ce(tHq, tW, g, p, ctl, s));
     } else {
       if (!make_map(&tHp, Hp, d, N, d, kBK, kBM)) return SLM_ERR_CUDA;
       if (kind == SLM_CE_ARGMAX_P)
-        SLM_TRY_CUDA(launch_fwd_argmax(tHq, tHp, tW, g, p, ctl, s));
+        SLM_LAUNCH(kTrFwdGemm, launch_fwd_argmax(tHq, tHp, tW, g, p, ctl, s));
       else
-        SLM_TRY_CUDA(launch_fwd_dual(tHq, tHp, tW, g, p, ctl, kind == SLM_RKL, s));
+        SLM_LAUNCH(kTrFwdGemm, launch_fwd_dual(tHq, tHp, tW, g, p, ctl, kind == SLM_RKL, s));
     }
-    SLM_TRY_CUDA(launch_combine(kind, 1, part, f.slots, zy, labels, ignore_index, N, V,
+    SLM_LAUNCH(kTrRow, launch_combine(kind, 1, part, f.slots, zy, labels, ignore_index, N, V,
                                 loss_tok, alpha_tok, stats, blk_sum, blk_cnt, status, s));
     if (two_pass_kind(kind)) {
       if (kind == SLM_JSD)
-        SLM_TRY_CUDA(launch_jsd(tHq, tHp, tW, g, p, ctl, s));
+        SLM_LAUNCH(kTrPass2Gemm, launch_jsd(tHq, tHp, tW, g, p, ctl, s));
       else
-        SLM_TRY_CUDA(launch_alpha(tHq, tHp, tW, g, p, ctl, s));
-      SLM_TRY_CUDA(launch_combine(kind, 2, part, f.slots, zy, labels, ignore_index, N, V,
+        SLM_LAUNCH(kTrPass2Gemm, launch_alpha(tHq, tHp, tW, g, p, ctl, s));
+      SLM_LAUNCH(kTrRow, launch_combine(kind, 2, part, f.slots, zy, labels, ignore_index, N, V,
                                   loss_tok, alpha_tok, stats, blk_sum, blk_cnt, status, s));
     }
-    SLM_TRY_CUDA(launch_finalize(blk_sum, blk_cnt, static_cast<int>(L.nblk), loss_sum, n_valid,
+    SLM_LAUNCH(kTrRow, launch_finalize(blk_sum, blk_cnt, static_cast<int>(L.nblk), loss_sum, n_valid,
                                  loss_mean, s));
   } else {
     SLM_TRY_CUDA(cudaMemsetAsync(blk_sum, 0, L.nblk * (sizeof(double) + sizeof(long long)), s));
-    SLM_TRY_CUDA(launch_finalize(blk_sum, blk_cnt, static_cast<int>(L.nblk), loss_sum, n_valid,
+    SLM_LAUNCH(kTrRow, launch_finalize(blk_sum, blk_cnt, static_cast<int>(L.nblk), loss_sum, n_valid,
                                  loss_mean, s));
   }
   return SLM_OK;
@@ -418,7 +514,7 @@ static int loss_bwd(int kind, const void* Hq, const void* Hp, const void* W,
   const DevCtl ctl = make_ctl(status);
 
   if (N == 0) {
-    if (!accumulate_dW) SLM_TRY_CUDA(launch_zero_f32(dW, V * d, s));
+    if (!accumulate_dW) SLM_LAUNCH(kTrRow, launch_zero_f32(dW, V * d, s));
     if (dw_ready) SLM_TRY_CUDA(cudaEventRecord(dw_ready, s));
     return SLM_OK;
   }
@@ -449,11 +545,11 @@ static int loss_bwd(int kind, const void* Hq, const void* Hp, const void* W,
     // The epilogue stores dZ in 32-row x 64-column blocks through this map.
     if (!make_map(&pz.dz_map, dz, V, rows, ldz, 64, 32)) return SLM_ERR_CUDA;
     if (!dual_kind(dz_kind)) {
-      SLM_TRY_CUDA(launch_dz_ce(tHq, tW_k, gz, pz, ctl, s));
+      SLM_LAUNCH(kTrDzGemm, launch_dz_ce(tHq, tW_k, gz, pz, ctl, s));
     } else {
       const __nv_bfloat16* hp = static_cast<const __nv_bfloat16*>(Hp) + c0 * d;
       if (!make_map(&tHp, hp, d, rows, d, kBK, kBM)) return SLM_ERR_CUDA;
-      SLM_TRY_CUDA(launch_dz_dual(tHq, tHp, tW_k, gz, pz, ctl, s));
+      SLM_LAUNCH(kTrDzGemm, launch_dz_dual(tHq, tHp, tW_k, gz, pz, ctl, s));
     }
     // 2) dH[chunk] = dZ W   (M = rows, N = d, K = V; W read MN-major).
     CUtensorMap tDz_k, tDz_mn, tH_mn;
@@ -469,13 +565,13 @@ static int loss_bwd(int kind, const void* Hq, const void* Hp, const void* W,
     if (overlap && c0 + rows >= N) {
       // Last chunk: dW is final once its GEMM is done; the dH GEMM that follows leaves
       // SMs free for the caller's reduction of dW.
-      SLM_TRY_CUDA(launch_dw(tDz_mn, tH_mn, gw, pw, ctl, s));
+      SLM_LAUNCH(kTrDwGemm, launch_dw(tDz_mn, tH_mn, gw, pw, ctl, s));
       if (dw_ready) SLM_TRY_CUDA(cudaEventRecord(dw_ready, s));
       gh.reserve_pairs = reserve_pairs;
-      SLM_TRY_CUDA(launch_dh(tDz_k, tW_mn, gh, ph, ctl, s));
+      SLM_LAUNCH(kTrDhGemm, launch_dh(tDz_k, tW_mn, gh, ph, ctl, s));
     } else {
-      SLM_TRY_CUDA(launch_dh(tDz_k, tW_mn, gh, ph, ctl, s));
-      SLM_TRY_CUDA(launch_dw(tDz_mn, tH_mn, gw, pw, ctl, s));
+      SLM_LAUNCH(kTrDhGemm, launch_dh(tDz_k, tW_mn, gh, ph, ctl, s));
+      SLM_LAUNCH(kTrDwGemm, launch_dw(tDz_mn, tH_mn, gw, pw, ctl, s));
     }
   }
   return SLM_OK;
@@ -511,8 +607,9 @@ int slm_align_labels(const int32_t* tokens, const uint8_t* loss_mask, const int3
   if (!tokens || !labels) return SLM_ERR_NULL;
   int st = check_device();
   if (st != SLM_OK) return st;
-  SLM_TRY_CUDA(launch_align_labels(tokens, loss_mask, seq_ids, B, S, shift, ignore_index, labels,
-                                   static_cast<cudaStream_t>(stream)));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  SLM_LAUNCH(kTrRow, launch_align_labels(tokens, loss_mask, seq_ids, B, S, shift, ignore_index,
+                                         labels, s));
   return SLM_OK;
 }
 
@@ -548,8 +645,8 @@ int slm_target_flatness(const void* Hp, const void* W, int64_t N, int64_t d, int
   if (!make_map(&tHp, Hp, d, N, d, kBK, kBM)) return SLM_ERR_CUDA;
   if (!make_map(&tW, W, d, V, d, kBK, 128)) return SLM_ERR_CUDA;
   FwdParams p{nullptr, 0, N, V, part, nullptr, nullptr, 0, nullptr, nullptr, 0};
-  SLM_TRY_CUDA(launch_fwd_flat(tHp, tW, g, p, ctl, s));
-  SLM_TRY_CUDA(launch_flat_combine(part, f.slots, N, V, flat, s));
+  SLM_LAUNCH(kTrFwdGemm, launch_fwd_flat(tHp, tW, g, p, ctl, s));
+  SLM_LAUNCH(kTrRow, launch_flat_combine(part, f.slots, N, V, flat, s));
   return SLM_OK;
 }
 
@@ -577,7 +674,8 @@ int64_t slm_chunk_for_budget(int kind, int64_t N, int64_t d, int64_t V, size_t b
     else
       hi = mid - 1;
   }
-  return lo * step;
+  // A chunk of all N rows is the largest that can be used: never report more.
+  return std::min<int64_t>(lo * step, N);
 }
 
 int slm_loss_fwd_bwd(int kind, const void* Hq, const void* Hp, const void* W,
@@ -610,13 +708,13 @@ int slm_loss_fwd_bwd(int kind, const void* Hq, const void* Hp, const void* W,
   const DevCtl ctl = make_ctl(status);
   if (N == 0) {
     SLM_TRY_CUDA(cudaMemsetAsync(blk_sum, 0, L.nblk * (sizeof(double) + sizeof(long long)), s));
-    SLM_TRY_CUDA(launch_finalize(blk_sum, blk_cnt, static_cast<int>(L.nblk), loss_sum, n_valid,
+    SLM_LAUNCH(kTrRow, launch_finalize(blk_sum, blk_cnt, static_cast<int>(L.nblk), loss_sum, n_valid,
                                  loss_mean, s));
-    if (!accumulate_dW) SLM_TRY_CUDA(launch_zero_f32(dW, V * d, s));
+    if (!accumulate_dW) SLM_LAUNCH(kTrRow, launch_zero_f32(dW, V * d, s));
     return SLM_OK;
   }
   // The mean's denominator is needed before the first chunk's gradient.
-  SLM_TRY_CUDA(launch_count_valid(labels, ignore_index, N, V, kind == SLM_CE ? 1 : 0, n_valid, s));
+  SLM_LAUNCH(kTrRow, launch_count_valid(labels, ignore_index, N, V, kind == SLM_CE ? 1 : 0, n_valid, s));
   const int64_t C = fused_chunk(N, chunk_tokens);
   const FwdSched f = fwd_sched(kind, V);
   const bool argmax_kind = kind == SLM_CE_ARGMAX_P;
@@ -639,41 +737,41 @@ int slm_loss_fwd_bwd(int kind, const void* Hq, const void* Hp, const void* W,
     if (!make_map_f32(&p.lq_map, lq, V, rows, ldl, 32, 32)) return SLM_ERR_CUDA;
     if (p.lp_out && !make_map_f32(&p.lp_map, lp, V, rows, ldl, 32, 32)) return SLM_ERR_CUDA;
     if (!dual_kind(kind)) {
-      SLM_TRY_CUDA(launch_fwd_ce(tHq, tW, g, p, ctl, s));
+      SLM_LAUNCH(kTrFwdGemm, launch_fwd_ce(tHq, tW, g, p, ctl, s));
     } else {
       const __nv_bfloat16* hp = static_cast<const __nv_bfloat16*>(Hp) + c0 * d;
       if (!make_map(&tHp, hp, d, rows, d, kBK, kBM)) return SLM_ERR_CUDA;
       if (argmax_kind)
-        SLM_TRY_CUDA(launch_fwd_argmax(tHq, tHp, tW, g, p, ctl, s));
+        SLM_LAUNCH(kTrFwdGemm, launch_fwd_argmax(tHq, tHp, tW, g, p, ctl, s));
       else
-        SLM_TRY_CUDA(launch_fwd_dual(tHq, tHp, tW, g, p, ctl, kind == SLM_RKL, s));
+        SLM_LAUNCH(kTrFwdGemm, launch_fwd_dual(tHq, tHp, tW, g, p, ctl, kind == SLM_RKL, s));
     }
-    SLM_TRY_CUDA(launch_combine(kind, 1, part, f.slots, zy, labels, ignore_index, rows, V,
+    SLM_LAUNCH(kTrRow, launch_combine(kind, 1, part, f.slots, zy, labels, ignore_index, rows, V,
                                 loss_tok, alpha_tok, stats, blk_sum, blk_cnt, status, s, c0, N));
     // 2) Second pass of the alpha losses / JSD over the kept logits.
     if (two_pass_kind(kind)) {
-      SLM_TRY_CUDA(launch_logits_pass2(kind, lq, lp, ldl, stats, c0, N, rows, V, part, s));
-      SLM_TRY_CUDA(launch_combine(kind, 2, part, 1, zy, labels, ignore_index, rows, V, loss_tok,
+      SLM_LAUNCH(kTrLogitsRow, launch_logits_pass2(kind, lq, lp, ldl, stats, c0, N, rows, V, part, s));
+      SLM_LAUNCH(kTrRow, launch_combine(kind, 2, part, 1, zy, labels, ignore_index, rows, V, loss_tok,
                                   alpha_tok, stats, blk_sum, blk_cnt, status, s, c0, N));
     }
     // 3) Logits gradient of the chunk from the kept logits.
     DzParams pz{dz_kind, dz_labels, ignore_index, c0, rows, N, V, stats, grad_tok, grad_scale,
                 n_valid, dz, ldz, ComboW{}};
-    SLM_TRY_CUDA(launch_logits_dz(pz, lq, lp, ldl, s));
+    SLM_LAUNCH(kTrLogitsRow, launch_logits_dz(pz, lq, lp, ldl, s));
     // 4) dH[chunk] = dZ W and dW (+)= dZ^T H[chunk].
     if (!make_map(&tDz_k, dz, V, rows, ldz, kBK, kBM)) return SLM_ERR_CUDA;
     const GemmGeom gh = geom(rows, d, V, kTileDh, 1, 1, kPairM,
                               SLM_SYNC_KB_B, SLM_SYNC_SLACK_B);
     DhParams ph{static_cast<__nv_bfloat16*>(dHq), c0, rows, d};
-    SLM_TRY_CUDA(launch_dh(tDz_k, tW_mn, gh, ph, ctl, s));
+    SLM_LAUNCH(kTrDhGemm, launch_dh(tDz_k, tW_mn, gh, ph, ctl, s));
     if (!make_map(&tDz_mn, dz, V, rows, ldz, 64, 64)) return SLM_ERR_CUDA;
     if (!make_map(&tH_mn, hq, d, rows, d, 64, 64)) return SLM_ERR_CUDA;
     const GemmGeom gw = geom(V, d, rows, kTileDw, 1, 1, kPairM,
                               SLM_SYNC_KB_B, SLM_SYNC_SLACK_B);
     DwParams pw{dW, V, d, (accumulate_dW || c0 > 0) ? 1 : 0};
-    SLM_TRY_CUDA(launch_dw(tDz_mn, tH_mn, gw, pw, ctl, s));
+    SLM_LAUNCH(kTrDwGemm, launch_dw(tDz_mn, tH_mn, gw, pw, ctl, s));
   }
-  SLM_TRY_CUDA(launch_finalize(blk_sum, blk_cnt, static_cast<int>(L.nblk), loss_sum, n_valid,
+  SLM_LAUNCH(kTrRow, launch_finalize(blk_sum, blk_cnt, static_cast<int>(L.nblk), loss_sum, n_valid,
                                loss_mean, s));
   return SLM_OK;
 }
@@ -719,18 +817,18 @@ int slm_combo_fwd(const float* weights, const void* Hq, const void* Hp, const vo
     if (!make_map(&tW, W, d, V, d, kBK, 128)) return SLM_ERR_CUDA;
     FwdParams p{labels, ignore_index, N, V, part, zy, stats, cw.w[SLM_JSD] != 0.f ? 1 : 0,
                 nullptr, nullptr, 0};
-    SLM_TRY_CUDA(launch_fwd_union(tHq, tHp, tW, g, p, ctl, s));
-    SLM_TRY_CUDA(launch_combo_combine(1, cw, part, f.slots, zy, labels, ignore_index, N, V,
+    SLM_LAUNCH(kTrFwdGemm, launch_fwd_union(tHq, tHp, tW, g, p, ctl, s));
+    SLM_LAUNCH(kTrRow, launch_combo_combine(1, cw, part, f.slots, zy, labels, ignore_index, N, V,
                                       stats, tl, status, s));
     if (two_pass) {
-      SLM_TRY_CUDA(launch_pass2_union(tHq, tHp, tW, g, p, ctl, s));
-      SLM_TRY_CUDA(launch_combo_combine(2, cw, part, f.slots, zy, labels, ignore_index, N, V,
+      SLM_LAUNCH(kTrPass2Gemm, launch_pass2_union(tHq, tHp, tW, g, p, ctl, s));
+      SLM_LAUNCH(kTrRow, launch_combo_combine(2, cw, part, f.slots, zy, labels, ignore_index, N, V,
                                         stats, tl, status, s));
     }
   }
-  SLM_TRY_CUDA(launch_combo_total(cw, tl, labels, ignore_index, N, V, loss_tok, term_loss_tok,
+  SLM_LAUNCH(kTrRow, launch_combo_total(cw, tl, labels, ignore_index, N, V, loss_tok, term_loss_tok,
                                   blk_sums, blk_cnt, s));
-  SLM_TRY_CUDA(launch_combo_finalize(blk_sums, blk_cnt, static_cast<int>(L.nblk), loss_sum,
+  SLM_LAUNCH(kTrRow, launch_combo_finalize(blk_sums, blk_cnt, static_cast<int>(L.nblk), loss_sum,
                                      term_loss_sum, n_valid, loss_mean, s));
   return SLM_OK;
 }
@@ -756,7 +854,7 @@ int slm_combo_bwd(const float* weights, const void* Hq, const void* Hp, const vo
   SLM_TRY_CUDA(cudaMemsetAsync(status, 0, sizeof(int), s));
   const DevCtl ctl = make_ctl(status);
   if (N == 0) {
-    if (!accumulate_dW) SLM_TRY_CUDA(launch_zero_f32(dW, V * d, s));
+    if (!accumulate_dW) SLM_LAUNCH(kTrRow, launch_zero_f32(dW, V * d, s));
     return SLM_OK;
   }
   const int64_t C = default_chunk(N, d, chunk_tokens);
@@ -777,20 +875,64 @@ int slm_combo_bwd(const float* weights, const void* Hq, const void* Hp, const vo
                              SLM_SYNC_KB_V, SLM_SYNC_SLACK_V);
     DzParams pz{-1, labels, ignore_index, c0, rows, N, V, stats, grad_tok, grad_scale,
                 n_valid, dz, ldz, cw};
-    SLM_TRY_CUDA(launch_dz_combo(tHq, tHp, tW_k, gz, pz, ctl, s));
+    SLM_LAUNCH(kTrDzGemm, launch_dz_combo(tHq, tHp, tW_k, gz, pz, ctl, s));
     if (!make_map(&tDz_k, dz, V, rows, ldz, kBK, kBM)) return SLM_ERR_CUDA;
     const GemmGeom gh = geom(rows, d, V, kTileDh, 1, 1, kPairM,
                               SLM_SYNC_KB_B, SLM_SYNC_SLACK_B);
     DhParams ph{static_cast<__nv_bfloat16*>(dHq), c0, rows, d};
-    SLM_TRY_CUDA(launch_dh(tDz_k, tW_mn, gh, ph, ctl, s));
+    SLM_LAUNCH(kTrDhGemm, launch_dh(tDz_k, tW_mn, gh, ph, ctl, s));
     if (!make_map(&tDz_mn, dz, V, rows, ldz, 64, 64)) return SLM_ERR_CUDA;
     if (!make_map(&tH_mn, hq, d, rows, d, 64, 64)) return SLM_ERR_CUDA;
     const GemmGeom gw = geom(V, d, rows, kTileDw, 1, 1, kPairM,
                               SLM_SYNC_KB_B, SLM_SYNC_SLACK_B);
     DwParams pw{dW, V, d, (accumulate_dW || c0 > 0) ? 1 : 0};
-    SLM_TRY_CUDA(launch_dw(tDz_mn, tH_mn, gw, pw, ctl, s));
+    SLM_LAUNCH(kTrDwGemm, launch_dw(tDz_mn, tH_mn, gw, pw, ctl, s));
   }
   return SLM_OK;
+}
+
+int slm_count_valid(int kind, const int32_t* labels, int32_t ignore_index, int64_t N,
+                    int64_t V, int64_t* n_valid, void* stream) {
+  if (!valid_kind(kind)) return SLM_ERR_KIND;
+  if (N < 0 || V <= 0 || N >= (int64_t(1) << 31) || V >= (int64_t(1) << 31))
+    return SLM_ERR_SHAPE;
+  if (!n_valid || (kind == SLM_CE && N > 0 && !labels)) return SLM_ERR_NULL;
+  int st = check_device();
+  if (st != SLM_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  SLM_LAUNCH(kTrRow, launch_count_valid(N > 0 ? labels : nullptr, ignore_index, N, V,
+                                        kind == SLM_CE ? 1 : 0, n_valid, s));
+  return SLM_OK;
+}
+
+int slm_trace_enable(int on) {
+  g_trace_on.store(on ? 1 : 0);
+  return SLM_OK;
+}
+
+int slm_trace_read(double* ms, int64_t* launches, int n_classes) {
+  if (n_classes < 0 || ((!ms || !launches) && n_classes > 0)) return SLM_ERR_NULL;
+  std::lock_guard<std::mutex> lock(g_trace_mu);
+  for (int c = 0; c < n_classes; ++c) {
+    ms[c] = 0.0;
+    launches[c] = 0;
+  }
+  int st = SLM_OK;
+  for (const TraceRec& r : g_trace_recs) {
+    float t = 0.f;
+    if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&t, r.a, r.b) != cudaSuccess)
+      st = SLM_ERR_CUDA;
+    else if (r.cls < n_classes) {
+      ms[r.cls] += t;
+      launches[r.cls] += 1;
+    }
+    trace_release(r.a);
+    trace_release(r.b);
+  }
+  g_trace_recs.clear();
+  if (g_trace_dropped != 0 && st == SLM_OK) st = SLM_ERR_WORKSPACE;
+  g_trace_dropped = 0;
+  return st;
 }
 
 int slm_debug_set(int fault_mode, long long timeout_cycles) {

@@ -321,7 +321,20 @@ __global__ void __launch_bounds__(64 + 128 * NWG, 1)
     if (sync_pub && lane == 0)
       st_relaxed_u64(&g_pair_progress[pair],
                      (static_cast<unsigned long long>(g.epoch) << 32) | 0xffffffffull);
-    if (!ok) {
+    if (ok) {
+      // Producer tail: the leader's MMA warp releases every stage of BOTH CTAs with a
+      // multicast commit that arrives on this CTA's "empty" barrier once the stage's MMAs
+      // are done.  Wait for the releases of the last STAGES stages, so that no such remote
+      // arrive can reach this CTA's shared memory after it has exited.
+      // If the pair is aborting, the last releases may never come: then give the ones in
+      // flight a moment instead.
+      const uint32_t first = it > (uint32_t)STAGES ? it - STAGES : 0u;
+      bool tail_ok = true;
+      for (uint32_t i = first; tail_ok && i < it; ++i)
+        tail_ok = wait_warp(&pc->empty[i % STAGES], (i / STAGES) & 1u, abort, ctl);
+      if (!tail_ok)
+        for (int i = 0; i < 100; ++i) __nanosleep(1000);
+    } else {
       if (leader) {
         // The full barriers count both CTAs' copies: waiting on them lets the pair's
         // copies in flight land before either CTA leaves the final cluster barrier.
@@ -329,6 +342,9 @@ __global__ void __launch_bounds__(64 + 128 * NWG, 1)
         for (uint32_t i = first; i < it; ++i)
           wait_warp(&pc->full[i % STAGES], (i / STAGES) & 1u, abort, ctl, false);
       } else {
+        // The non-leader's copies complete on the leader's barriers, which this CTA cannot
+        // wait on: give any copy still in flight (issued at most STAGES stages ahead of the
+        // last one the leader counted) time to land before the final cluster barrier.
         for (int i = 0; i < 100; ++i) __nanosleep(1000);
       }
     }

@@ -10,9 +10,13 @@
 // device code is loaded there and held until the process exits.
 //
 // The array's name is only a host-side stand-in for the symbol; its device address is
-// looked up with cudaGetSymbolAddress, once per device, with that device current, on the
-// first call that runs on it.  That lookup may load the library's device code, so the first
-// call on each device should come before any stream capture.
+// looked up with cudaGetSymbolAddress, with the device current, on the first call that runs
+// on a device, and kept for that device's CUDA context.  A context that is torn down and
+// re-created (cudaDeviceReset, or a primary context released and retained again) reloads
+// the library's device code at another address, so the cached address is keyed on the
+// context's unique id and looked up again when the current context is a different one.
+// The lookup may load the library's device code, so the first call on each device (and
+// the first after a context is re-created) should come before any stream capture.
 //
 // Every call shares the one array and leaves its contents behind.  The forward rewrites
 // everything it reads before reading it (the status word is cleared on entry, the partials,
@@ -22,6 +26,8 @@
 // serialised by the caller.
 //
 // Nothing here allocates: no cudaMalloc, no cudaFree, no allocating library routine.
+
+#include <cuda.h>
 
 #include <mutex>
 
@@ -33,21 +39,55 @@ namespace {
 static __device__ __align__(256) unsigned char g_noalloc_scratch[SLM_NOALLOC_SCRATCH_BYTES];
 
 constexpr int kMaxDevices = 64;
-void* g_scratch_ptr[kMaxDevices] = {nullptr};
+struct ScratchAddr {
+  unsigned long long ctx_id;  // unique id of the context the address belongs to (0: none)
+  void* ptr;
+};
+ScratchAddr g_scratch[kMaxDevices] = {};
 std::mutex g_scratch_mu;
 
-// Device address of the scratch array on the current device (looked up once per device).
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+// Unique id of the current CUDA context, or 0 when there is none or it cannot be read.
+unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  if (!get_current || !get_id) return 0;
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+// Device address of the scratch array in the current device's current context: looked up
+// once per device and context (again whenever the context's id cannot be read).
 int scratch_address(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SLM_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (g_scratch_ptr[dev] == nullptr) {
+  const unsigned long long id = current_context_id();
+  if (id == 0 || g_scratch[dev].ctx_id != id || g_scratch[dev].ptr == nullptr) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
       return SLM_ERR_CUDA;
-    g_scratch_ptr[dev] = p;
+    // The lookup creates the primary context when there was none: key on the id after it.
+    g_scratch[dev] = ScratchAddr{current_context_id(), p};
   }
-  *out = g_scratch_ptr[dev];
+  *out = g_scratch[dev].ptr;
   return SLM_OK;
 }
 
@@ -62,7 +102,7 @@ extern "C" SLM_API int slm_loss_fwd_noalloc(int kind, const void* Hq, const void
                                             void* stream) {
   // Reject an unknown kind or an invalid shape before touching the device.
   if (slm_workspace_bytes(kind, N, d, V, 1) == 0) {
-    if (kind < SLM_CE || kind > SLM_LK_HYBRID) return SLM_ERR_KIND;
+    if (kind < SLM_CE || kind > SLM_CE_ARGMAX_P) return SLM_ERR_KIND;
     return SLM_ERR_SHAPE;
   }
   void* scratch = nullptr;

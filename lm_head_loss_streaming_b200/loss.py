@@ -114,6 +114,26 @@ def workspace_bytes(kind, N, d, V, chunk_tokens=0):
     return _lib.slm_workspace_bytes(_kind_id(kind), N, d, V, chunk_tokens)
 
 
+def count_valid(kind, labels, N, V, ignore_index=IGNORE_INDEX, out=None):
+    """Valid-row count through ``slm_count_valid``: rows whose label is not
+    ``ignore_index`` and, for CE, lies in [0, V) -- the rows the kernels do not mask.
+    ``labels`` may be None for the distribution kinds (every row counts).  Returns an int64
+    [1] CUDA tensor (``out`` if given), filled asynchronously on the current stream."""
+    k = _kind_id(kind)
+    if labels is not None:
+        if (not labels.is_cuda or labels.dtype != torch.int32 or not labels.is_contiguous()
+                or labels.shape != (N,) or labels.device.index != torch.cuda.current_device()):
+            raise ValueError(f"labels must be a contiguous int32 tensor of shape ({N},) on the "
+                             f"current CUDA device")
+    if out is None:
+        out = torch.empty(1, dtype=torch.int64, device=torch.cuda.current_device())
+    else:
+        _check_out("out", out, (1,), torch.int64)
+    _lib.check(_lib.slm_count_valid(k, _ptr(labels), ignore_index, N, V, _ptr(out), _stream()),
+               "slm_count_valid")
+    return out
+
+
 def lm_head_loss_fwd(kind, hidden, weight, labels=None, target_hidden=None,
                      ignore_index=IGNORE_INDEX, workspace=None, chunk_tokens=0,
                      out=None) -> FwdResult:

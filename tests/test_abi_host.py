@@ -210,12 +210,43 @@ def test_chunk_for_budget_is_the_largest_chunk_that_fits(lib, fused):
             if c == 0:
                 assert ws(kind, N, d, V, step) > budget
                 continue
-            assert c % step == 0
+            assert c % step == 0 or c == N
+            assert c <= N
             assert ws(kind, N, d, V, c) <= budget
             if c < N:
                 assert ws(kind, N, d, V, c + step) > budget
         # An unlimited budget takes every row in one chunk.
-        assert _lib.slm_chunk_for_budget(kind, N, d, V, 1 << 60, fused) >= N
+        assert _lib.slm_chunk_for_budget(kind, N, d, V, 1 << 60, fused) == N
+    # N not a multiple of the step: the chunk is never reported larger than N, and the
+    # workspace of the reported chunk is the one the call uses.
+    for N in (1, 127, 129, 300, 1000, 4097):
+        c = _lib.slm_chunk_for_budget(_lib.SLM_KL, N, 64, 3000, 1 << 40, fused)
+        assert c == N
+    # With a budget between two steps the chunk stays a multiple of the step below N.
+    N = 1000
+    c = _lib.slm_chunk_for_budget(_lib.SLM_KL, N, 64, 3000, ws(_lib.SLM_KL, N, 64, 3000, 3 * step),
+                                  fused)
+    assert c == min(3 * step, N)
     assert _lib.slm_chunk_for_budget(_lib.SLM_KL, 1024, 12, 100, 1 << 30, fused) == 0  # d % 8
     assert _lib.slm_chunk_for_budget(9, 1024, 16, 100, 1 << 30, fused) == 0
     assert _lib.slm_chunk_for_budget(_lib.SLM_KL, 16384, 4096, 128256, 1, fused) == 0
+
+
+def test_count_valid_rejects_bad_arguments_on_the_host(lib):
+    fake = 1 << 20  # aligned, never dereferenced: every call below returns before enqueuing
+    assert _lib.slm_count_valid(9, fake, -100, 10, 100, fake, None) == 4       # kind
+    assert _lib.slm_count_valid(_lib.SLM_CE, fake, -100, -1, 100, fake, None) == 2  # N < 0
+    assert _lib.slm_count_valid(_lib.SLM_CE, fake, -100, 10, 0, fake, None) == 2    # V <= 0
+    assert _lib.slm_count_valid(_lib.SLM_CE, fake, -100, 1 << 31, 100, fake, None) == 2
+    assert _lib.slm_count_valid(_lib.SLM_CE, None, -100, 10, 100, fake, None) == 1   # labels
+    assert _lib.slm_count_valid(_lib.SLM_KL, fake, -100, 10, 100, None, None) == 1   # out
+
+
+def test_trace_switch_and_empty_read(lib):
+    assert _lib.slm_trace_enable(False) == 0
+    st, got = _lib.slm_trace_read()
+    assert st == 0
+    assert set(got) == set(_lib.TRACE_CLASSES)
+    assert all(ms == 0.0 and n == 0 for ms, n in got.values())
+    assert lib.slm_trace_read(None, None, 3) == 1
+    assert lib.slm_trace_read(None, None, 0) == 0

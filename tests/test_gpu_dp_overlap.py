@@ -139,3 +139,61 @@ def test_nccl_fused_step_matches_oracle(kind):
     rh, rw = oracle.backward(kind, inp.Hq, inp.W, inp.labels, inp.Hp, gt, inp.ignore_index)
     assert_grad_close(h.double().cpu().numpy(), rh, "dp fused dH")
     assert_grad_close(w.double().cpu().numpy(), rw, "dp fused dW")
+
+
+@pytest.mark.parametrize("fused", [False, True])
+def test_nccl_step_with_dW_sharded_by_vocabulary_rows(fused):
+    """dW reduce-scattered by vocabulary rows (FSDP-style) over a one-rank NCCL group: the
+    single shard is the whole summed dW, equal bit for bit to the all-reduced one."""
+    inp = synthetic.make("kl_div", 500, 128, 3001, w_std=0.05, ignore_frac=0.1, seed=77,
+                         with_labels=True)
+    Hq, W, Hp, lab = _dev(inp)
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{_free_port()}", rank=0,
+                            world_size=1, timeout=timedelta(seconds=60),
+                            device_id=torch.device("cuda", 0))
+    try:
+        step = dp.cuda_step_fused if fused else dp.cuda_step
+        a = step("kl_div", Hq, W, lab, Hp, inp.ignore_index, chunk_tokens=256)
+        wa = a.dW.clone()
+        b = step("kl_div", Hq, W, lab, Hp, inp.ignore_index, chunk_tokens=256, shard_dW=True)
+        torch.cuda.synchronize()
+    finally:
+        dist.destroy_process_group()
+    assert b.dW_rows == (0, inp.V) and b.dW.shape == wa.shape
+    assert torch.equal(b.dW, wa)
+    assert a.n_valid.item() == b.n_valid.item()
+
+
+def test_fused_dp_count_leaves_out_rows_the_kernels_mask():
+    """The fused data-parallel step takes its valid count from the library: a CE label
+    outside [0, V) is masked by the kernels and left out of the count, so the mean and the
+    gradient agree with the oracle on the remaining rows."""
+    inp = synthetic.make("ce", 400, 128, 2000, w_std=0.05, ignore_frac=0.1, seed=78)
+    labels = inp.labels.clone()
+    bad = int(np.flatnonzero(labels.numpy() != inp.ignore_index)[3])
+    labels[bad] = inp.V + 5
+    Hq, W, _, _ = _dev(inp)
+    lab = labels.to(Hq.device)
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{_free_port()}", rank=0,
+                            world_size=1, timeout=timedelta(seconds=60),
+                            device_id=torch.device("cuda", 0))
+    try:
+        ws = torch.empty(_lib.slm_fused_workspace_bytes(_lib.SLM_CE, inp.N, inp.d, inp.V, 256),
+                         dtype=torch.uint8, device=Hq.device)
+        r = dp.cuda_step_fused("ce", Hq, W, lab, None, inp.ignore_index, chunk_tokens=256,
+                               workspace=ws)
+        torch.cuda.synchronize()
+        n, loss = r.n_valid.item(), r.loss_mean.item()
+        w = r.dW.clone()
+        st = _lib.slm_device_status(ws.data_ptr(), torch.cuda.current_stream().cuda_stream)
+    finally:
+        dist.destroy_process_group()
+    assert st == 6  # SLM_ERR_LABEL_RANGE
+    keep = labels.numpy().copy()
+    keep[bad] = inp.ignore_index      # the oracle's reading: that row is masked
+    ref = oracle.forward("ce", inp.Hq, inp.W, torch.from_numpy(keep), None, inp.ignore_index)
+    assert n == ref["n_valid"]
+    assert abs(loss - ref["loss"]) <= 2e-3 * abs(ref["loss"])
+    rh, rw = oracle.backward("ce", inp.Hq, inp.W, torch.from_numpy(keep), None, None,
+                             inp.ignore_index)
+    assert_grad_close(w.double().cpu().numpy(), rw, "dp fused dW, masked label")
