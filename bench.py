@@ -64,6 +64,13 @@ def parse_args():
                          "overlapping the sum with the last chunk's dH GEMM")
     ap.add_argument("--reserve-sms", type=int, default=8,
                     help="N > 1: SMs the last dH GEMM leaves to the dW reduction")
+    ap.add_argument("--no-ab", action="store_true",
+                    help="skip timing the other backward launch shape")
+    ap.add_argument("--no-ce-line", action="store_true",
+                    help="skip timing hard-label CE at the same shape")
+    ap.add_argument("--bwd-mode", type=int, default=0, choices=[0, 1],
+                    help="backward launch shape: 1 = one persistent launch per chunk "
+                         "(logits gradient, dH and dW), 0 = three launches per chunk")
     return ap.parse_args()
 
 
@@ -101,18 +108,19 @@ def class_flops(kind, N, V, d, fused=False):
     return out
 
 
-def fused_launches_per_step(kind, N, chunk_tokens):
+def fused_launches_per_step(kind, N, chunk_tokens, bwd_mode=1):
     """Kernels of the fused call: count, then per chunk GEMM + combine (+ second pass +
-    combine) + logits-gradient + dH + dW, then finalize."""
+    combine) + logits-gradient + dH and dW (one persistent launch, or two), then finalize."""
     C = min(chunk_tokens if chunk_tokens > 0 else 4096, N)
     C = ((C + 255) // 256) * 256 if chunk_tokens > 0 else C
     chunks = (N + C - 1) // C
-    per = 7 if kind in ("tv", "nla", "lk_hybrid", "jsd") else 5
+    per = (7 if kind in ("tv", "nla", "lk_hybrid", "jsd") else 5) - (1 if bwd_mode == 1 else 0)
     return 2 + per * chunks
 
 
-def launches_per_step(kind, N, d, chunk_tokens):
-    """Kernels of libslm.so launched by one forward + backward (memsets excluded)."""
+def launches_per_step(kind, N, d, chunk_tokens, bwd_mode=1):
+    """Kernels of libslm.so launched by one forward + backward (memsets excluded): per
+    backward chunk one persistent launch (bwd_mode 1) or three (0)."""
     if N == 0:
         return 1 + 1
     # GEMM, combine, [second GEMM pass, combine], finalize
@@ -120,7 +128,7 @@ def launches_per_step(kind, N, d, chunk_tokens):
     C = chunk_tokens if chunk_tokens > 0 else ((2 * d + 127) // 128) * 128
     C = max(1, min(C, N))
     chunks = (N + C - 1) // C
-    return fwd + 3 * chunks
+    return fwd + (1 if bwd_mode == 1 else 3) * chunks
 
 
 def load_peaks():
@@ -363,6 +371,7 @@ def run_ours(args):
         return step
 
     step = make_step(Hq, W, lab, Hp)
+    _lib.slm_set_backward_mode(args.bwd_mode)
 
     for _ in range(args.warmup):
         step()
@@ -414,6 +423,81 @@ def run_ours(args):
         "grads_gib": round((dH.numel() * 2 + dW.numel() * 4) / gib, 3),
         "fp32_logits_avoided_gib": round(N * V * 4 * (2 if dual else 1) / gib, 2),
     }
+
+    # The same step with the other backward launch shape (one persistent launch per chunk,
+    # or three launches per chunk), timed the same way right after, for an A/B.
+    other_mode = None
+    if world == 1 and not args.fused and not args.no_ab:
+        other = 1 - args.bwd_mode
+        _lib.slm_set_backward_mode(other)
+        for _ in range(max(1, args.warmup)):
+            step()
+        torch.cuda.synchronize()
+        oa, ob = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        _lib.check(_lib.slm_trace_read()[0], "slm_trace_read")
+        _lib.slm_trace_enable(True)
+        oa.record(stream)
+        for _ in range(args.steps):
+            step()
+        ob.record(stream)
+        torch.cuda.synchronize()
+        _lib.slm_trace_enable(False)
+        o_st, o_trace = _lib.slm_trace_read()
+        _lib.check(o_st, "slm_trace_read")
+        _lib.slm_set_backward_mode(args.bwd_mode)
+        o_ms = oa.elapsed_time(ob) / args.steps
+        o_flops = class_flops(kind, N, V, d)
+        o_kernels = {}
+        for name, (ms_tot, n_launch) in o_trace.items():
+            if n_launch == 0:
+                continue
+            ms_per = ms_tot / args.steps
+            e = {"ms_per_step": round(ms_per, 3), "launches_per_step": n_launch / args.steps}
+            if o_flops.get(name, 0.0) > 0:
+                tf = o_flops[name] / (ms_per / 1e3) / 1e12
+                e.update({"tflops": round(tf, 1),
+                          "frac": round(tf / load_peaks()[0]["bf16_tflops_sustained"], 4)})
+            o_kernels[name] = e
+        other_mode = {"bwd_mode": other,
+                      "bwd_launches": ("one persistent launch per chunk" if other == 1
+                                       else "three launches per chunk"),
+                      "ms_per_step": round(o_ms, 3), "value": round(N / (o_ms / 1e3), 1),
+                      "kernels": o_kernels}
+
+    # Hard-label CE at the same shape (the LM-head loss proper, 8*N*V*d flops per fwd+bwd,
+    # which is the metric's formula exactly), timed the same way on the same draft hidden
+    # states with seeded labels (5% ignored), beside the workload's own kind.
+    ce_same = None
+    if world == 1 and not args.fused and kind != "ce" and not args.no_ce_line:
+        g = torch.Generator(device=dev).manual_seed(4321)
+        lab_ce = torch.randint(0, V, (N,), generator=g, device=dev, dtype=torch.int32)
+        lab_ce[torch.randperm(N, generator=g, device=dev)[: round(0.05 * N)]] = inp.ignore_index
+        ws_ce = torch.empty(workspace_bytes("ce", N, d, V, args.chunk_tokens),
+                            dtype=torch.uint8, device=dev)
+
+        def ce_step():
+            r = lm_head_loss_fwd("ce", Hq, W, lab_ce, None, inp.ignore_index, workspace=ws_ce,
+                                 chunk_tokens=args.chunk_tokens)
+            lm_head_loss_bwd(r, Hq, W, lab_ce, None, inp.ignore_index, dH=dH, dW=dW,
+                             chunk_tokens=args.chunk_tokens)
+
+        for _ in range(max(1, args.warmup)):
+            ce_step()
+        torch.cuda.synchronize()
+        ca, cb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ca.record(stream)
+        for _ in range(args.steps):
+            ce_step()
+        cb.record(stream)
+        torch.cuda.synchronize()
+        c_ms = ca.elapsed_time(cb) / args.steps
+        peaks0, _ = load_peaks()
+        ce_same = {"kind": "ce", "ms_per_step": round(c_ms, 3),
+                   "value": round(N / (c_ms / 1e3), 1), "unit": "tokens/s",
+                   "tflops_8NVd": round(8.0 * N * V * d / (c_ms / 1e3) / 1e12, 1),
+                   "frac_bf16_peak": round(8.0 * N * V * d / (c_ms / 1e3) / 1e12
+                                           / peaks0["bf16_tflops"], 4)}
+        del ws_ce
 
     # The fused single call (each chunk's logits kept instead of recomputed), timed the same
     # way on the same inputs, for reference beside the default path.
@@ -593,13 +677,19 @@ def run_ours(args):
                      "kernels": kernels, "traced_ms_per_step": round(traced_ms, 3),
                      "fwd_call_ms": round(fwd_ms, 3)},
         "gpu_launches": sum(n for _, n in trace.values()),
-        "gpu_launches_expected": (fused_launches_per_step(kind, N, args.chunk_tokens)
+        "gpu_launches_expected": (fused_launches_per_step(kind, N, args.chunk_tokens,
+                                                          args.bwd_mode)
                                   if args.fused
-                                  else launches_per_step(kind, N, d, args.chunk_tokens))
+                                  else launches_per_step(kind, N, d, args.chunk_tokens,
+                                                         args.bwd_mode))
                                  * args.steps,
         "clocks": clocks,
         "memory": memory,
         "e2e": e2e,
+        "bwd_launches": ("one persistent launch per chunk" if args.bwd_mode == 1
+                         else "three launches per chunk"),
+        "other_bwd_mode": other_mode,
+        "ce_same_shape": ce_same,
         "fused": fused_info,
         "kernel_sha": kernel_source_hash(),
     }

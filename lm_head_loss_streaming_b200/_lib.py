@@ -64,6 +64,7 @@ SIGNATURES = {
     "slm_loss_fwd_noalloc": (_INT, [_INT, _P, _P, _P, _P, _I32, _I64, _I64, _I64,
                                     _P, _P, _P, _P, _P, _P, _P, _P]),
     "slm_count_valid": (_INT, [_INT, _P, _I32, _I64, _I64, _P, _P]),
+    "slm_set_backward_mode": (_INT, [_INT]),
     "slm_trace_enable": (_INT, [_INT]),
     "slm_trace_read": (_INT, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_I64), _INT]),
 }
@@ -254,3 +255,9 @@ def slm_trace_read():
     cnt = (_I64 * n)()
     st = load().slm_trace_read(ms, cnt, n)
     return st, {name: (ms[i], int(cnt[i])) for i, name in enumerate(TRACE_CLASSES)}
+
+
+def slm_set_backward_mode(mode):
+    """1: one persistent launch per backward chunk (default); 0: three launches per chunk.
+    Returns the previous mode (-1: invalid mode, nothing changed)."""
+    return load().slm_set_backward_mode(int(mode))

@@ -49,6 +49,9 @@ constexpr long long kTimeoutCycles = 4000000000LL;  // ~2 s at the B200's boost 
 
 // Test hooks set through slm_debug_set (process-wide, read at every launch).
 std::atomic<int> g_fault{0};
+// Backward launch shape (slm_set_backward_mode): 1 = one persistent launch per chunk
+// (bwd_fused_kernel), 0 = three launches per chunk (logits gradient, dH, dW).
+std::atomic<int> g_bwd_mode{0};
 std::atomic<long long> g_timeout{kTimeoutCycles};
 
 DevCtl make_ctl(int* status) {
@@ -144,8 +147,14 @@ int64_t default_chunk(int64_t N, int64_t d, int64_t chunk_tokens) {
   return std::max<int64_t>(1, std::min<int64_t>(c, N));
 }
 
+// Counters of the persistent fused backward (bwd_fused_kernel): one per 256-row M tile of a
+// chunk and one per vocabulary run of its logits-gradient schedule.
+size_t fused_ctr_count(int64_t C) {
+  return 1 + static_cast<size_t>(std::max<int64_t>(1, ceil_div(C, kPairM))) + kMaxRuns + 1;
+}
+
 struct Layout {
-  size_t status_off, red_off, nblk, big_off, part_off, zy_off, dz_off, ldz;
+  size_t status_off, red_off, nblk, ctr_off, big_off, part_off, zy_off, dz_off, ldz;
   size_t fwd_total;  // bytes the forward uses
   size_t bwd_total;  // bytes the backward uses with this chunk size
   size_t total;      // max of the two
@@ -157,6 +166,8 @@ Layout layout(int kind, int64_t N, int64_t d, int64_t V, int64_t chunk_tokens) {
   L.nblk = static_cast<size_t>(std::max<int64_t>(1, ceil_div(N, kCombineThreads)));
   L.red_off = kAlign;
   size_t off = align_up(L.red_off + L.nblk * (sizeof(double) + sizeof(long long)), kAlign);
+  L.ctr_off = off;
+  off = align_up(off + fused_ctr_count(default_chunk(N, d, chunk_tokens)) * sizeof(int), kAlign);
   L.big_off = off;
   const FwdSched f = fwd_sched(kind, V);
   const size_t part = static_cast<size_t>(f.slots) * f.fields * static_cast<size_t>(N) * 4;
@@ -273,7 +284,7 @@ int common_checks(int kind, const void* Hq, const void* Hp, const void* W, const
 // partials (kUnionFields per slot), the label logits, the per-term losses [kNumKinds][N],
 // and per-block sums of the total and of every term.
 struct ComboLayout {
-  size_t status_off, red_off, nblk, cnt_off, part_off, zy_off, tl_off, dz_off, ldz;
+  size_t status_off, red_off, nblk, cnt_off, ctr_off, part_off, zy_off, tl_off, dz_off, ldz;
   size_t fwd_total, bwd_total, total;
 };
 
@@ -283,7 +294,9 @@ ComboLayout combo_layout(int64_t N, int64_t d, int64_t V, int64_t chunk_tokens) 
   L.nblk = static_cast<size_t>(std::max<int64_t>(1, ceil_div(N, kCombineThreads)));
   L.red_off = kAlign;
   L.cnt_off = align_up(L.red_off + L.nblk * (1 + kNumKinds) * sizeof(double), 16);
-  const size_t big = align_up(L.cnt_off + L.nblk * sizeof(long long), kAlign);
+  L.ctr_off = align_up(L.cnt_off + L.nblk * sizeof(long long), kAlign);
+  const size_t big = align_up(
+      L.ctr_off + fused_ctr_count(default_chunk(N, d, chunk_tokens)) * sizeof(int), kAlign);
   const FwdSched f = fwd_sched(SLM_KL, V);
   L.part_off = big;
   const size_t part = static_cast<size_t>(f.slots) * kUnionFields * static_cast<size_t>(N) * 4;
@@ -356,7 +369,8 @@ int64_t fused_chunk(int64_t N, int64_t chunk_tokens) {
 }
 
 struct FusedLayout {
-  size_t status_off, red_off, nblk, part_off, zy_off, lq_off, lp_off, dz_off, ldl, ldz, total;
+  size_t status_off, red_off, nblk, ctr_off, part_off, zy_off, lq_off, lp_off, dz_off, ldl, ldz,
+      total;
 };
 
 FusedLayout fused_layout(int kind, int64_t N, int64_t V, int64_t chunk_tokens) {
@@ -365,6 +379,8 @@ FusedLayout fused_layout(int kind, int64_t N, int64_t V, int64_t chunk_tokens) {
   L.nblk = static_cast<size_t>(std::max<int64_t>(1, ceil_div(N, kCombineThreads)));
   L.red_off = kAlign;
   size_t off = align_up(L.red_off + L.nblk * (sizeof(double) + sizeof(long long)), kAlign);
+  L.ctr_off = off;  // the claim counter of the persistent dH + dW launch
+  off += kAlign;
   const size_t C = static_cast<size_t>(fused_chunk(N, chunk_tokens));
   const FwdSched f = fwd_sched(kind, V);
   L.part_off = off;
@@ -490,6 +506,37 @@ int slm_loss_fwd(int kind, const void* Hq, const void* Hp, const void* W, const 
   return SLM_OK;
 }
 
+// One chunk of the backward as one persistent launch (bwd_fused_kernel): the chunk's
+// logits gradient (zkind 0: CE, 1: divergences, 2: weighted combination; -1: dZ is already
+// in the chunk buffer, only dH and dW run), then dH and dW, ordered by the counters at
+// `ctr` (zeroed here).
+static int launch_chunk_fused(int zkind, const CUtensorMap& tHq, const CUtensorMap& tHp,
+                       const CUtensorMap& tWk, const CUtensorMap& tDzK, const CUtensorMap& tWmn,
+                       const CUtensorMap& tDzMn, const CUtensorMap& tHmn, const FwdSched& f,
+                       int64_t rows, int64_t d, int64_t V, int* ctr, const DzParams& pz,
+                       const DhParams& ph, const DwParams& pw, const DevCtl& ctl,
+                       cudaStream_t s) {
+  BwdFusedGeom fg{};
+  fg.claim = ctr;
+  if (zkind >= 0) {
+    fg.gz = geom(rows, V, d, f.bn, f.vc, kGroupPairs, kPairM, SLM_SYNC_KB_V, SLM_SYNC_SLACK_V);
+    fg.bn_z = f.bn;
+    fg.rows_done = ctr + 1;
+    fg.runs_done = ctr + 1 + fg.gz.num_m;
+  }
+  SLM_TRY_CUDA(
+      cudaMemsetAsync(ctr, 0, (1 + fg.gz.num_m + fg.gz.units_n) * sizeof(int), s));
+  fg.num_mh = static_cast<int>(ceil_div(rows, kPairM));
+  fg.num_nh = static_cast<int>(ceil_div(d, kTileDh));
+  fg.kb_h = static_cast<int>(ceil_div(V, kBK));
+  fg.num_mw = static_cast<int>(ceil_div(V, kPairM));
+  fg.num_nw = static_cast<int>(ceil_div(d, kTileDw));
+  fg.kb_w = static_cast<int>(ceil_div(rows, kBK));
+  SLM_LAUNCH(kTrBwdFused, launch_bwd_fused(zkind < 0 ? 0 : zkind, tHq, tHp, tWk, tDzK, tWmn,
+                                           tDzMn, tHmn, fg, pz, ph, pw, ctl, s));
+  return SLM_OK;
+}
+
 // The backward of slm_loss_bwd and slm_loss_bwd_overlap.  With `overlap`, the last chunk
 // runs its dW GEMM before its dH GEMM, records `dw_ready` (if given) between the two, and
 // launches that dH GEMM on `reserve_pairs` fewer CTA pairs.
@@ -510,6 +557,7 @@ static int loss_bwd(int kind, const void* Hq, const void* Hp, const void* W,
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   int* status = reinterpret_cast<int*>(ws + L.status_off);
   __nv_bfloat16* dz = reinterpret_cast<__nv_bfloat16*>(ws + L.dz_off);
+  int* ctr = reinterpret_cast<int*>(ws + L.ctr_off);
   SLM_TRY_CUDA(cudaMemsetAsync(status, 0, sizeof(int), s));
   const DevCtl ctl = make_ctl(status);
 
@@ -544,6 +592,26 @@ static int loss_bwd(int kind, const void* Hq, const void* Hp, const void* W,
                 n_valid, dz, ldz, ComboW{}};
     // The epilogue stores dZ in 32-row x 64-column blocks through this map.
     if (!make_map(&pz.dz_map, dz, V, rows, ldz, 64, 32)) return SLM_ERR_CUDA;
+    CUtensorMap tDz_k, tDz_mn, tH_mn;
+    if (!make_map(&tDz_k, dz, V, rows, ldz, kBK, kBM)) return SLM_ERR_CUDA;
+    if (!make_map(&tDz_mn, dz, V, rows, ldz, 64, 64)) return SLM_ERR_CUDA;
+    if (!make_map(&tH_mn, hq, d, rows, d, 64, 64)) return SLM_ERR_CUDA;
+    DhParams ph{static_cast<__nv_bfloat16*>(dHq), c0, rows, d};
+    DwParams pw{dW, V, d, (accumulate_dW || c0 > 0) ? 1 : 0};
+    if (!overlap && g_bwd_mode.load() == 1) {
+      // 1-3) in one persistent launch.
+      if (dual_kind(dz_kind)) {
+        const __nv_bfloat16* hp = static_cast<const __nv_bfloat16*>(Hp) + c0 * d;
+        if (!make_map(&tHp, hp, d, rows, d, kBK, kBM)) return SLM_ERR_CUDA;
+      } else {
+        tHp = tHq;
+      }
+      st = launch_chunk_fused(dual_kind(dz_kind) ? 1 : 0, tHq, tHp, tW_k, tDz_k, tW_mn, tDz_mn,
+                              tH_mn, f, rows, d, V, ctr, pz, ph, pw, ctl, s);
+      if (st != SLM_OK) return st;
+      continue;
+    }
+    // 1) as its own launch.
     if (!dual_kind(dz_kind)) {
       SLM_LAUNCH(kTrDzGemm, launch_dz_ce(tHq, tW_k, gz, pz, ctl, s));
     } else {
@@ -552,16 +620,10 @@ static int loss_bwd(int kind, const void* Hq, const void* Hp, const void* W,
       SLM_LAUNCH(kTrDzGemm, launch_dz_dual(tHq, tHp, tW_k, gz, pz, ctl, s));
     }
     // 2) dH[chunk] = dZ W   (M = rows, N = d, K = V; W read MN-major).
-    CUtensorMap tDz_k, tDz_mn, tH_mn;
-    if (!make_map(&tDz_k, dz, V, rows, ldz, kBK, kBM)) return SLM_ERR_CUDA;
     GemmGeom gh = geom(rows, d, V, kTileDh, 1, 1, kPairM, SLM_SYNC_KB_B, SLM_SYNC_SLACK_B);
-    DhParams ph{static_cast<__nv_bfloat16*>(dHq), c0, rows, d};
     // 3) dW (+)= dZ^T H[chunk]   (M = V, N = d, K = rows; both operands MN-major).
-    if (!make_map(&tDz_mn, dz, V, rows, ldz, 64, 64)) return SLM_ERR_CUDA;
-    if (!make_map(&tH_mn, hq, d, rows, d, 64, 64)) return SLM_ERR_CUDA;
     const GemmGeom gw = geom(V, d, rows, kTileDw, 1, 1, kPairM,
                               SLM_SYNC_KB_B, SLM_SYNC_SLACK_B);
-    DwParams pw{dW, V, d, (accumulate_dW || c0 > 0) ? 1 : 0};
     if (overlap && c0 + rows >= N) {
       // Last chunk: dW is final once its GEMM is done; the dH GEMM that follows leaves
       // SMs free for the caller's reduction of dW.
@@ -760,15 +822,22 @@ int slm_loss_fwd_bwd(int kind, const void* Hq, const void* Hp, const void* W,
     SLM_LAUNCH(kTrLogitsRow, launch_logits_dz(pz, lq, lp, ldl, s));
     // 4) dH[chunk] = dZ W and dW (+)= dZ^T H[chunk].
     if (!make_map(&tDz_k, dz, V, rows, ldz, kBK, kBM)) return SLM_ERR_CUDA;
-    const GemmGeom gh = geom(rows, d, V, kTileDh, 1, 1, kPairM,
-                              SLM_SYNC_KB_B, SLM_SYNC_SLACK_B);
-    DhParams ph{static_cast<__nv_bfloat16*>(dHq), c0, rows, d};
-    SLM_LAUNCH(kTrDhGemm, launch_dh(tDz_k, tW_mn, gh, ph, ctl, s));
     if (!make_map(&tDz_mn, dz, V, rows, ldz, 64, 64)) return SLM_ERR_CUDA;
     if (!make_map(&tH_mn, hq, d, rows, d, 64, 64)) return SLM_ERR_CUDA;
+    DhParams ph{static_cast<__nv_bfloat16*>(dHq), c0, rows, d};
+    DwParams pw{dW, V, d, (accumulate_dW || c0 > 0) ? 1 : 0};
+    if (g_bwd_mode.load() == 1) {
+      // Both GEMMs in one persistent launch (dZ is already complete: no counters).
+      st = launch_chunk_fused(-1, tHq, tHq, tW, tDz_k, tW_mn, tDz_mn, tH_mn, f, rows, d, V,
+                              reinterpret_cast<int*>(ws + L.ctr_off), pz, ph, pw, ctl, s);
+      if (st != SLM_OK) return st;
+      continue;
+    }
+    const GemmGeom gh = geom(rows, d, V, kTileDh, 1, 1, kPairM,
+                              SLM_SYNC_KB_B, SLM_SYNC_SLACK_B);
+    SLM_LAUNCH(kTrDhGemm, launch_dh(tDz_k, tW_mn, gh, ph, ctl, s));
     const GemmGeom gw = geom(V, d, rows, kTileDw, 1, 1, kPairM,
                               SLM_SYNC_KB_B, SLM_SYNC_SLACK_B);
-    DwParams pw{dW, V, d, (accumulate_dW || c0 > 0) ? 1 : 0};
     SLM_LAUNCH(kTrDwGemm, launch_dw(tDz_mn, tH_mn, gw, pw, ctl, s));
   }
   SLM_LAUNCH(kTrRow, launch_finalize(blk_sum, blk_cnt, static_cast<int>(L.nblk), loss_sum, n_valid,
@@ -851,6 +920,7 @@ int slm_combo_bwd(const float* weights, const void* Hq, const void* Hp, const vo
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   int* status = reinterpret_cast<int*>(ws + L.status_off);
   __nv_bfloat16* dz = reinterpret_cast<__nv_bfloat16*>(ws + L.dz_off);
+  int* ctr = reinterpret_cast<int*>(ws + L.ctr_off);
   SLM_TRY_CUDA(cudaMemsetAsync(status, 0, sizeof(int), s));
   const DevCtl ctl = make_ctl(status);
   if (N == 0) {
@@ -875,17 +945,23 @@ int slm_combo_bwd(const float* weights, const void* Hq, const void* Hp, const vo
                              SLM_SYNC_KB_V, SLM_SYNC_SLACK_V);
     DzParams pz{-1, labels, ignore_index, c0, rows, N, V, stats, grad_tok, grad_scale,
                 n_valid, dz, ldz, cw};
-    SLM_LAUNCH(kTrDzGemm, launch_dz_combo(tHq, tHp, tW_k, gz, pz, ctl, s));
     if (!make_map(&tDz_k, dz, V, rows, ldz, kBK, kBM)) return SLM_ERR_CUDA;
-    const GemmGeom gh = geom(rows, d, V, kTileDh, 1, 1, kPairM,
-                              SLM_SYNC_KB_B, SLM_SYNC_SLACK_B);
-    DhParams ph{static_cast<__nv_bfloat16*>(dHq), c0, rows, d};
-    SLM_LAUNCH(kTrDhGemm, launch_dh(tDz_k, tW_mn, gh, ph, ctl, s));
     if (!make_map(&tDz_mn, dz, V, rows, ldz, 64, 64)) return SLM_ERR_CUDA;
     if (!make_map(&tH_mn, hq, d, rows, d, 64, 64)) return SLM_ERR_CUDA;
+    DhParams ph{static_cast<__nv_bfloat16*>(dHq), c0, rows, d};
+    DwParams pw{dW, V, d, (accumulate_dW || c0 > 0) ? 1 : 0};
+    if (g_bwd_mode.load() == 1) {
+      st = launch_chunk_fused(2, tHq, tHp, tW_k, tDz_k, tW_mn, tDz_mn, tH_mn, f, rows, d, V,
+                              ctr, pz, ph, pw, ctl, s);
+      if (st != SLM_OK) return st;
+      continue;
+    }
+    SLM_LAUNCH(kTrDzGemm, launch_dz_combo(tHq, tHp, tW_k, gz, pz, ctl, s));
+    const GemmGeom gh = geom(rows, d, V, kTileDh, 1, 1, kPairM,
+                              SLM_SYNC_KB_B, SLM_SYNC_SLACK_B);
+    SLM_LAUNCH(kTrDhGemm, launch_dh(tDz_k, tW_mn, gh, ph, ctl, s));
     const GemmGeom gw = geom(V, d, rows, kTileDw, 1, 1, kPairM,
                               SLM_SYNC_KB_B, SLM_SYNC_SLACK_B);
-    DwParams pw{dW, V, d, (accumulate_dW || c0 > 0) ? 1 : 0};
     SLM_LAUNCH(kTrDwGemm, launch_dw(tDz_mn, tH_mn, gw, pw, ctl, s));
   }
   return SLM_OK;
@@ -903,6 +979,11 @@ int slm_count_valid(int kind, const int32_t* labels, int32_t ignore_index, int64
   SLM_LAUNCH(kTrRow, launch_count_valid(N > 0 ? labels : nullptr, ignore_index, N, V,
                                         kind == SLM_CE ? 1 : 0, n_valid, s));
   return SLM_OK;
+}
+
+int slm_set_backward_mode(int mode) {
+  if (mode < 0 || mode > 1) return -1;
+  return g_bwd_mode.exchange(mode);
 }
 
 int slm_trace_enable(int on) {

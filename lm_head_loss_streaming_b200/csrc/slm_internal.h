@@ -116,6 +116,24 @@ struct DwParams {
   int beta;  // 1: add to dW, 0: overwrite
 };
 
+// Persistent fused backward of one token chunk (bwd_fused_kernel): the logits-gradient
+// units (Z), then the dH units (H) and the dW units (W) in one launch, claimed by the CTA
+// pairs in that order from a counter.  Every epilogue warp counts the Z units it finished
+// per M tile and per vocabulary run; a producer waits for the counts its next dH or dW unit
+// needs.
+constexpr int kFusedEpiWarps = 16;  // epilogue warps of a pair (2 CTAs x 2 warpgroups)
+struct BwdFusedGeom {
+  GemmGeom gz;           // Z units (M = chunk rows, N = V, K = d); gz.num_units = 0: none
+  int bn_z;              // dZ tile width (vocabulary columns per Z tile)
+  int num_mh, num_nh;    // H units: 256-row M tiles of the chunk x 512-column tiles of d
+  int kb_h;              // H K blocks (over V)
+  int num_mw, num_nw;    // W units: 256-row tiles of the vocabulary x 256-column tiles of d
+  int kb_w;              // W K blocks (over the chunk's rows)
+  int* claim;            // next unit to claim (zero at launch)
+  int* rows_done;        // [gz.num_m] finished Z units per M tile, x kFusedEpiWarps
+  int* runs_done;        // [gz.units_n] finished Z units per vocabulary run, x kFusedEpiWarps
+};
+
 // Kernel launchers (slm_kernels.cu).  Each returns the launch's error status.
 int sm_count();
 cudaError_t launch_fwd_ce(const CUtensorMap& tH, const CUtensorMap& tW, const GemmGeom& g,
@@ -140,6 +158,17 @@ cudaError_t launch_dh(const CUtensorMap& tDz, const CUtensorMap& tW, const GemmG
                       const DhParams& p, const DevCtl& c, cudaStream_t s);
 cudaError_t launch_dw(const CUtensorMap& tDzT, const CUtensorMap& tH, const GemmGeom& g,
                       const DwParams& p, const DevCtl& c, cudaStream_t s);
+// The persistent fused backward of one chunk.  zkind: 0 = CE logits gradient (one
+// operand), 1 = the divergences' (two operands), 2 = weighted combination; with
+// fg.gz.num_units == 0 only phases H and W run (dZ already in the chunk buffer).  The
+// launcher sets the lockstep tag of the Z units; the claim counter and the completion
+// counters must be zero when the launch starts.
+cudaError_t launch_bwd_fused(int zkind, const CUtensorMap& tHq, const CUtensorMap& tHp,
+                             const CUtensorMap& tWk, const CUtensorMap& tDzK,
+                             const CUtensorMap& tWmn, const CUtensorMap& tDzMn,
+                             const CUtensorMap& tHmn, const BwdFusedGeom& fg,
+                             const DzParams& pz, const DhParams& ph, const DwParams& pw,
+                             const DevCtl& c, cudaStream_t s);
 
 // Fused forward + backward over stored chunk logits.
 // Valid rows (label != ignore_index; for CE also in [0, V)) -> *n_valid.

@@ -184,6 +184,15 @@ struct PairCfg {
   static_assert(NBUF * kAccCols <= kTmemCols, "accumulator buffers must fit in TMEM");
   static_assert(BNI % 128 == 0 && BNI <= 256, "UMMA N (M = 256) and whole 64-wide B boxes");
   static_assert(kEpiCols % 32 == 0, "epilogue column share");
+  // The bytes the leader's "full" barrier expects per CTA equal the boxes the producer
+  // issues per stage: per A operand one 64 x 128 box (K-major) or two 64 x 64 boxes
+  // (MN-major), per B slice one 64 x kSliceN box (K-major) or kSliceN / 64 boxes of 64 x 64
+  // (MN-major); bf16 throughout.
+  static constexpr uint32_t kABoxBytes = A_MN ? 2u * 64u * 64u * 2u : 64u * kBM * 2u;
+  static constexpr uint32_t kBBoxBytes =
+      B_MN ? static_cast<uint32_t>(kSliceN / 64) * 64u * 64u * 2u : 64u * kSliceN * 2u;
+  static_assert(NUM_A * kABoxBytes + NSUB * kBBoxBytes == kStageBytes,
+                "expect_tx must count exactly the bytes the producer loads");
   static_assert(kSmem <= 232448, "shared memory per CTA");
 };
 
@@ -2226,3 +2235,6 @@ cudaError_t launch_flat_combine(const float* part, int nch, int64_t N, int64_t V
 }
 
 }  // namespace slm
+
+// The persistent fused backward (one launch per chunk for the logits gradient, dH and dW).
+#include "slm_bwd_fused.cuh"

@@ -68,5 +68,7 @@ def pytest_terminal_summary(terminalreporter, exitstatus, config):
         tw.line("near-tie comparisons (entries in band / entries, slack used / tolerance, "
                 "error without slack / tolerance):")
         for r in ties:
+            off = r.get("raw_frac_off_tie_rows")
+            off_s = "" if off is None else f"  off-tie-rows raw {off:.3f} ({r.get('tie_rows')} tie rows)"
             tw.line(f"  {r['near_ties']}/{r['entries']}  slack {r['slack_used_frac']:.4f}  "
-                    f"raw {r['raw_frac']:.3f}  {r['test']} [{r['what']}]")
+                    f"raw {r['raw_frac']:.3f}{off_s}  {r['test']} [{r['what']}]")

@@ -151,6 +151,10 @@ def tie_slack(inp, kind, rows=None, grad_tok=None):
     near &= valid[:, None] & (g[:, None] != 0.0)
     tie_slack.last_count = int(near.sum())
     tie_slack.last_entries = int(near.size)
+    # Rows whose gradient a flip changes to first order: token rows with a near-tie (dH) and
+    # vocabulary rows with a near-tie in some token row (dW).
+    tie_slack.last_rows = near.any(axis=1)
+    tie_slack.last_cols = near.any(axis=0)
     qn = np.where(near, q, 0.0)
     qsum = qn.sum(axis=1)
     aW, aH = np.abs(W), np.abs(Hq)
@@ -179,6 +183,14 @@ def assert_grad_close(g, r, what="", slack=0.0):
                      raw_frac=float(diff.max()) / (GRAD_RTOL * den),
                      near_ties=getattr(tie_slack, "last_count", None),
                      entries=getattr(tie_slack, "last_entries", None))
+        # The raw error (no slack) on the rows no near-tie touches to first order.
+        for mask in (getattr(tie_slack, "last_cols", None), getattr(tie_slack, "last_rows", None)):
+            if mask is not None and g.ndim == 2 and len(mask) == g.shape[0]:
+                off = ~mask
+                extra["raw_frac_off_tie_rows"] = (
+                    float(diff[off].max()) / (GRAD_RTOL * den) if off.any() else 0.0)
+                extra["tie_rows"] = int(mask.sum())
+                break
     _record(f"{what} grad", err / den / GRAD_RTOL, **extra)
     assert err / den <= GRAD_RTOL, f"{what}: grad rel err {err / den:.3e} > {GRAD_RTOL}"
 

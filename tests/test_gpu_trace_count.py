@@ -4,7 +4,8 @@ its kernel-class timing (slm_trace_enable / slm_trace_read).
 The count must equal the forward's own n_valid, and the oracle's reading of the mask
 ("Streaming Cross Entropy": the mean divides by the valid, non-masked tokens).  The trace
 must report one launch per GEMM of the launch sequence (forward statistics GEMM, then per
-token chunk the logits-gradient, dH and dW GEMMs) with positive device times.
+token chunk the logits-gradient, dH and dW GEMMs, or one persistent launch for all three)
+with positive device times.
 """
 
 import numpy as np
@@ -44,21 +45,25 @@ def test_count_valid_matches_forward_and_mask():
     assert count_valid("tv", None, 0, inp.V, inp.ignore_index).item() == 0
 
 
-@pytest.mark.parametrize("kind,launches", [
-    ("kl_div", {"fwd_gemm": 1, "dz_gemm": 3, "dh_gemm": 3, "dw_gemm": 3, "row": 2}),
-    ("tv", {"fwd_gemm": 1, "pass2_gemm": 1, "dz_gemm": 3, "dh_gemm": 3, "dw_gemm": 3,
-            "row": 3})])
-def test_trace_reports_every_gemm_launch(kind, launches):
+@pytest.mark.parametrize("kind,mode,launches", [
+    ("kl_div", 0, {"fwd_gemm": 1, "dz_gemm": 3, "dh_gemm": 3, "dw_gemm": 3, "row": 2}),
+    ("tv", 0, {"fwd_gemm": 1, "pass2_gemm": 1, "dz_gemm": 3, "dh_gemm": 3, "dw_gemm": 3,
+               "row": 3}),
+    ("kl_div", 1, {"fwd_gemm": 1, "bwd_fused": 3, "row": 2}),
+    ("ce", 1, {"fwd_gemm": 1, "bwd_fused": 3, "row": 2})])
+def test_trace_reports_every_gemm_launch(kind, mode, launches):
     inp = synthetic.make(kind, 700, 128, 3000, w_std=0.05, seed=82)
     Hq, W, Hp, lab = _dev(inp)
     torch.cuda.synchronize()
     _lib.check(_lib.slm_trace_read()[0])
+    prev = _lib.slm_set_backward_mode(mode)
     _lib.slm_trace_enable(True)
     try:
         f = lm_head_loss_fwd(kind, Hq, W, lab, Hp, inp.ignore_index, chunk_tokens=256)
         lm_head_loss_bwd(f, Hq, W, lab, Hp, inp.ignore_index, chunk_tokens=256)
     finally:
         _lib.slm_trace_enable(False)
+        _lib.slm_set_backward_mode(prev)
     st, got = _lib.slm_trace_read()
     assert st == 0
     for name, (ms, n) in got.items():
