@@ -68,7 +68,7 @@ def parse_args():
                     help="skip timing the other backward launch shape")
     ap.add_argument("--no-ce-line", action="store_true",
                     help="skip timing hard-label CE at the same shape")
-    ap.add_argument("--bwd-mode", type=int, default=0, choices=[0, 1],
+    ap.add_argument("--bwd-mode", type=int, default=1, choices=[0, 1],
                     help="backward launch shape: 1 = one persistent launch per chunk "
                          "(logits gradient, dH and dW), 0 = three launches per chunk")
     return ap.parse_args()

@@ -210,13 +210,13 @@ SLM_API int slm_count_valid(int kind, const int32_t* labels, int32_t ignore_inde
 /* Launch shape of the backward (slm_loss_bwd, slm_combo_bwd and the backward half of
  * slm_loss_fwd_bwd).  The pages' backward ("Backward pass") is, per token chunk: recompute
  * the logits, form their gradient, produce the chunk's dH, accumulate dW.
- *   mode 1: each chunk is ONE persistent launch.  Its CTA pairs first compute the
+ *   mode 1 (default): each chunk is ONE persistent launch.  Its CTA pairs first compute the
  *          logits-gradient tiles, then the dH and dW tiles; a dH tile starts as soon as the
  *          logits gradient of its 256 rows is complete, a dW tile as soon as that of its 256
  *          vocabulary rows is, ordered by counters in the workspace (bounded waits: a wait
  *          that runs out records SLM_ERR_TIMEOUT).  The pairs' dW shares are sized so that
  *          every pair ends at about the same time.
- *   mode 0 (default): three launches per chunk (logits gradient, dH, dW).
+ *   mode 0: three launches per chunk (logits gradient, dH, dW).
  * Both give the same results (dW bit for bit; the same arithmetic in the same order).
  * slm_loss_bwd_overlap always uses three launches (its dW must be final before the last dH).
  * Process-wide; takes effect at the next call.  Returns the previous mode, or -1 for an

@@ -51,7 +51,7 @@ constexpr long long kTimeoutCycles = 4000000000LL;  // ~2 s at the B200's boost 
 std::atomic<int> g_fault{0};
 // Backward launch shape (slm_set_backward_mode): 1 = one persistent launch per chunk
 // (bwd_fused_kernel), 0 = three launches per chunk (logits gradient, dH, dW).
-std::atomic<int> g_bwd_mode{0};
+std::atomic<int> g_bwd_mode{1};
 std::atomic<long long> g_timeout{kTimeoutCycles};
 
 DevCtl make_ctl(int* status) {

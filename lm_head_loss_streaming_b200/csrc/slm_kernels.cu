@@ -489,6 +489,51 @@ __device__ __forceinline__ float max32(const float (&v)[32]) {
   return fmaxf(m0, m1);
 }
 
+// Packed fp32 pairs (sm_100 fma / add / sub / mul .f32x2): two independent fp32 operations,
+// each rounded to nearest as its scalar form, in one instruction.  SLM_PACKED_EPI = 0 selects
+// the scalar forms (same results, except where a packed pair of partial sums replaces one
+// running sum).
+#ifndef SLM_PACKED_EPI
+#define SLM_PACKED_EPI 1
+#endif
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "sub.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+__device__ __forceinline__ float2 exp2_2(float2 a) { return make_float2(exp2f(a.x), exp2f(a.y)); }
+
 __device__ __forceinline__ void mask_tail(float (&v)[32], int64_t col0, int64_t V) {
 #pragma unroll
   for (int i = 0; i < 32; ++i)
@@ -572,6 +617,14 @@ struct EpiFwdCE {
         m = mx;
       }
       if (m != -INFINITY) {
+#if SLM_PACKED_EPI
+        const float2 l2 = make_float2(kLog2e, kLog2e), nm = make_float2(-m, -m);
+        float2 a = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < 32; i += 2)
+          a = add2(a, exp2_2(fma2(make_float2(v[i], v[i + 1]), l2, nm)));
+        s += a.x + a.y;
+#else
         float a0 = 0.f, a1 = 0.f;
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
@@ -579,6 +632,7 @@ struct EpiFwdCE {
           a1 += exp2f(fmaf(v[i + 1], kLog2e, -m));
         }
         s += a0 + a1;
+#endif
       }
     }
   }
@@ -631,6 +685,31 @@ struct EpiFwdDualT {
       mp = xp;
     }
     if (mq == -INFINITY || mp == -INFINITY) return;
+#if SLM_PACKED_EPI
+    if (!TAIL) {
+      // Column pairs: each sum runs as two partial sums (even and odd columns), added at
+      // the end of the 32 columns.
+      const float2 l2 = make_float2(kLog2e, kLog2e);
+      const float2 nmq = make_float2(-mq, -mq), nmp = make_float2(-mp, -mp);
+      float2 sq2 = make_float2(0.f, 0.f), sp2 = sq2, a2 = sq2, b2 = sq2;
+#pragma unroll
+      for (int i = 0; i < 32; i += 2) {
+        const float2 zq = make_float2(vq[i], vq[i + 1]);
+        const float2 zp = make_float2(vp[i], vp[i + 1]);
+        const float2 eq = exp2_2(fma2(zq, l2, nmq));
+        const float2 e = exp2_2(fma2(zp, l2, nmp));
+        sq2 = add2(sq2, eq);
+        sp2 = add2(sp2, e);
+        if (ACC & 1) a2 = fma2(e, sub2(zp, zq), a2);
+        if (ACC & 2) b2 = fma2(eq, sub2(zq, zp), b2);
+      }
+      sq += sq2.x + sq2.y;
+      sp += sp2.x + sp2.y;
+      if (ACC & 1) A += a2.x + a2.y;
+      if (ACC & 2) B += b2.x + b2.y;
+      return;
+    }
+#endif
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
       const float eq = exp2f(fmaf(vq[i], kLog2e, -mq));
@@ -976,12 +1055,26 @@ struct EpiDz {
     if (DUAL) {
       {
         if (mode == 0) {
+#if SLM_PACKED_EPI
+          const float2 l2 = make_float2(kLog2e, kLog2e);
+          const float2 nq = make_float2(-lq2, -lq2), np = make_float2(-lp2, -lp2);
+          const float2 ck2 = make_float2(ck, ck);
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) {
+            const float2 qv = exp2_2(fma2(make_float2(vq[i], vq[i + 1]), l2, nq));
+            const float2 pv = exp2_2(fma2(make_float2(vp[i], vp[i + 1]), l2, np));
+            const float2 r = mul2(ck2, sub2(qv, pv));
+            vq[i] = r.x;
+            vq[i + 1] = r.y;
+          }
+#else
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             const float qv = exp2f(fmaf(vq[i], kLog2e, -lq2));
             const float pv = exp2f(fmaf(vp[i], kLog2e, -lp2));
             vq[i] = ck * (qv - pv);
           }
+#endif
         } else if (mode == 3) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
@@ -1012,11 +1105,24 @@ struct EpiDz {
       }
     } else {
       const int64_t rel = static_cast<int64_t>(lab) - col0;
+#if SLM_PACKED_EPI
+      const float2 l2 = make_float2(kLog2e, kLog2e), nq = make_float2(-lq2, -lq2);
+      const float2 g2 = make_float2(g, g);
+#pragma unroll
+      for (int i = 0; i < 32; i += 2) {
+        const float2 qv = exp2_2(fma2(make_float2(vq[i], vq[i + 1]), l2, nq));
+        const float2 oh = make_float2(rel == i ? 1.f : 0.f, rel == i + 1 ? 1.f : 0.f);
+        const float2 r = mul2(g2, sub2(qv, oh));
+        vq[i] = r.x;
+        vq[i + 1] = r.y;
+      }
+#else
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
         const float qv = exp2f(fmaf(vq[i], kLog2e, -lq2));
         vq[i] = g * (qv - (rel == i ? 1.f : 0.f));
       }
+#endif
     }
   }
 
