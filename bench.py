@@ -35,6 +35,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # The kernels and the host code that picks their tiles, schedule and launch shape: DRAM
 # counters taken with other sources do not describe this build.
 KERNEL_SOURCES = ["lm_head_loss_streaming_b200/csrc/slm_kernels.cu",
+                  "lm_head_loss_streaming_b200/csrc/slm_bwd_fused.cuh",
                   "lm_head_loss_streaming_b200/csrc/sm100.cuh",
                   "lm_head_loss_streaming_b200/csrc/slm_internal.h",
                   "lm_head_loss_streaming_b200/csrc/slm_schedule.h"]
