@@ -425,45 +425,65 @@ def run_ours(args):
         "fp32_logits_avoided_gib": round(N * V * 4 * (2 if dual else 1) / gib, 2),
     }
 
-    # The same step with the other backward launch shape (one persistent launch per chunk,
-    # or three launches per chunk), timed the same way right after, for an A/B.
+    # The same step with the other backward launch shape, as an interleaved A/B on the same
+    # inputs: `reps` repetitions of `steps // 2` steps with each shape, the order swapped
+    # from one repetition to the next (whichever shape runs second in a pair tends to be
+    # ahead), each with its own per-class trace; medians reported.
     other_mode = None
     if world == 1 and not args.fused and not args.no_ab:
+        import statistics
         other = 1 - args.bwd_mode
-        _lib.slm_set_backward_mode(other)
-        for _ in range(max(1, args.warmup)):
-            step()
+        ab_steps = max(2, args.steps // 2)
+        reps = 4
+        times = {args.bwd_mode: [], other: []}
+        traces = {args.bwd_mode: {}, other: {}}
+        for m in (other, args.bwd_mode):
+            _lib.slm_set_backward_mode(m)
+            for _ in range(max(1, args.warmup)):
+                step()
         torch.cuda.synchronize()
-        oa, ob = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        _lib.check(_lib.slm_trace_read()[0], "slm_trace_read")
-        _lib.slm_trace_enable(True)
-        oa.record(stream)
-        for _ in range(args.steps):
-            step()
-        ob.record(stream)
-        torch.cuda.synchronize()
-        _lib.slm_trace_enable(False)
-        o_st, o_trace = _lib.slm_trace_read()
-        _lib.check(o_st, "slm_trace_read")
+        for rep in range(reps):
+            for m in ((other, args.bwd_mode) if rep % 2 == 0 else (args.bwd_mode, other)):
+                _lib.slm_set_backward_mode(m)
+                step()
+                torch.cuda.synchronize()
+                _lib.check(_lib.slm_trace_read()[0], "slm_trace_read")
+                _lib.slm_trace_enable(True)
+                oa, ob = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                oa.record(stream)
+                for _ in range(ab_steps):
+                    step()
+                ob.record(stream)
+                torch.cuda.synchronize()
+                _lib.slm_trace_enable(False)
+                o_st, o_trace = _lib.slm_trace_read()
+                _lib.check(o_st, "slm_trace_read")
+                times[m].append(oa.elapsed_time(ob) / ab_steps)
+                for name, (ms_tot, n_launch) in o_trace.items():
+                    if n_launch:
+                        traces[m].setdefault(name, []).append(ms_tot / ab_steps)
         _lib.slm_set_backward_mode(args.bwd_mode)
-        o_ms = oa.elapsed_time(ob) / args.steps
         o_flops = class_flops(kind, N, V, d)
-        o_kernels = {}
-        for name, (ms_tot, n_launch) in o_trace.items():
-            if n_launch == 0:
-                continue
-            ms_per = ms_tot / args.steps
-            e = {"ms_per_step": round(ms_per, 3), "launches_per_step": n_launch / args.steps}
-            if o_flops.get(name, 0.0) > 0:
-                tf = o_flops[name] / (ms_per / 1e3) / 1e12
-                e.update({"tflops": round(tf, 1),
-                          "frac": round(tf / load_peaks()[0]["bf16_tflops_sustained"], 4)})
-            o_kernels[name] = e
-        other_mode = {"bwd_mode": other,
-                      "bwd_launches": ("one persistent launch per chunk" if other == 1
-                                       else "three launches per chunk"),
-                      "ms_per_step": round(o_ms, 3), "value": round(N / (o_ms / 1e3), 1),
-                      "kernels": o_kernels}
+        sustained = load_peaks()[0]["bf16_tflops_sustained"]
+
+        def summary(m):
+            ms = statistics.median(times[m])
+            ks = {}
+            for name, v in traces[m].items():
+                e = {"ms_per_step": round(statistics.median(v), 3)}
+                if o_flops.get(name, 0.0) > 0:
+                    tf = o_flops[name] / (e["ms_per_step"] / 1e3) / 1e12
+                    e.update({"tflops": round(tf, 1), "frac": round(tf / sustained, 4)})
+                ks[name] = e
+            return {"bwd_mode": m,
+                    "bwd_launches": ("one persistent launch per chunk" if m == 1
+                                     else "three launches per chunk"),
+                    "ms_per_step": round(ms, 3), "value": round(N / (ms / 1e3), 1),
+                    "ms_per_rep": [round(x, 3) for x in times[m]], "kernels": ks}
+
+        other_mode = {"interleaved": f"{reps} repetitions x {ab_steps} steps per shape, "
+                                     f"order alternating", "other": summary(other),
+                      "this": summary(args.bwd_mode)}
 
     # Hard-label CE at the same shape (the LM-head loss proper, 8*N*V*d flops per fwd+bwd,
     # which is the metric's formula exactly), timed the same way on the same draft hidden

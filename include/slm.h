@@ -218,7 +218,8 @@ SLM_API int slm_count_valid(int kind, const int32_t* labels, int32_t ignore_inde
  *          every pair ends at about the same time.
  *   mode 0: three launches per chunk (logits gradient, dH, dW).
  * Both give the same results (dW bit for bit; the same arithmetic in the same order).
- * slm_loss_bwd_overlap always uses three launches (its dW must be final before the last dH).
+ * slm_loss_bwd_overlap runs its last chunk as three launches in any mode (that chunk's dW
+ * must be final before its dH GEMM).
  * Process-wide; takes effect at the next call.  Returns the previous mode, or -1 for an
  * invalid mode (nothing changes). */
 SLM_API int slm_set_backward_mode(int mode);

@@ -598,8 +598,10 @@ static int loss_bwd(int kind, const void* Hq, const void* Hp, const void* W,
     if (!make_map(&tH_mn, hq, d, rows, d, 64, 64)) return SLM_ERR_CUDA;
     DhParams ph{static_cast<__nv_bfloat16*>(dHq), c0, rows, d};
     DwParams pw{dW, V, d, (accumulate_dW || c0 > 0) ? 1 : 0};
-    if (!overlap && g_bwd_mode.load() == 1) {
-      // 1-3) in one persistent launch.
+    const bool last_overlapped = overlap && c0 + rows >= N;
+    if (!last_overlapped && g_bwd_mode.load() == 1) {
+      // 1-3) in one persistent launch (with the overlap, every chunk but the last: that
+      // one runs its dW GEMM before its dH GEMM, below).
       if (dual_kind(dz_kind)) {
         const __nv_bfloat16* hp = static_cast<const __nv_bfloat16*>(Hp) + c0 * d;
         if (!make_map(&tHp, hp, d, rows, d, kBK, kBM)) return SLM_ERR_CUDA;
@@ -624,7 +626,7 @@ static int loss_bwd(int kind, const void* Hq, const void* Hp, const void* W,
     // 3) dW (+)= dZ^T H[chunk]   (M = V, N = d, K = rows; both operands MN-major).
     const GemmGeom gw = geom(V, d, rows, kTileDw, 1, 1, kPairM,
                               SLM_SYNC_KB_B, SLM_SYNC_SLACK_B);
-    if (overlap && c0 + rows >= N) {
+    if (last_overlapped) {
       // Last chunk: dW is final once its GEMM is done; the dH GEMM that follows leaves
       // SMs free for the caller's reduction of dW.
       SLM_LAUNCH(kTrDwGemm, launch_dw(tDz_mn, tH_mn, gw, pw, ctl, s));

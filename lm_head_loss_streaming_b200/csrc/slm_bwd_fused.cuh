@@ -33,6 +33,7 @@ constexpr uint32_t kFSlot = 48u * 1024u;  // one ring slot: the largest stage of
 constexpr int kFNwg = 2;                  // epilogue warpgroups per CTA
 constexpr int kFThreads = 64 + 128 * kFNwg;
 constexpr int kFQueue = 4;                // claimed units in flight between the warps
+constexpr int kFStageBytesPerWarp = 4096;  // epilogue staging per warp (dZ and dW blocks)
 // Readers of a queue slot, each arriving once on the leader's "empty" barrier: the leader's
 // MMA warp and epilogue warps, the other CTA's producer and epilogue warps.
 constexpr int kFQueueReaders = 1 + 4 * kFNwg + 1 + 4 * kFNwg;
@@ -500,14 +501,17 @@ __global__ void __launch_bounds__(kFThreads, 1)
         if (wide || b == 1) mbar_arrive_cluster(tempty_leader1);
       }
     };
+    // One staging buffer per epilogue warp, shared by the Z epilogue (dZ blocks on their way
+    // to a TMA store) and the dW epilogue (its read-add-write blocks): a warp works on one
+    // unit at a time.
+    uint8_t* stage_base = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(fq + 1) + 1023) & ~static_cast<uintptr_t>(1023));
+    float* warp_stage = reinterpret_cast<float*>(stage_base + (warp - 2) * kFStageBytesPerWarp);
     EpiZ ez;
-    if constexpr (EpiStageBytes<EpiZ>::value > 0) {
-      uint8_t* st = reinterpret_cast<uint8_t*>(
-          (reinterpret_cast<uintptr_t>(fq + 1) + 1023) & ~static_cast<uintptr_t>(1023));
-      ez.stage = reinterpret_cast<float*>(st + (warp - 2) * EpiStageBytes<EpiZ>::value);
-    }
+    if constexpr (EpiStageBytes<EpiZ>::value > 0) ez.stage = warp_stage;
     EpiDh eh;
-    EpiDw ew;
+    EpiDwStaged ew;
+    ew.stage = warp_stage;
     bool ok = true;
     for (uint32_t q = 0; ok; ++q) {
       const int u = read_unit(q);
@@ -578,10 +582,12 @@ static cudaError_t launch_bwd_fused_t(const CUtensorMap& tHq, const CUtensorMap&
                                       const CUtensorMap& tHmn, const BwdFusedGeom& fg_in,
                                       const DzParams& pz, const DhParams& ph,
                                       const DwParams& pw, const DevCtl& c, cudaStream_t s) {
-  constexpr size_t kStage = EpiStageBytes<EpiZ>::value;
+  static_assert(EpiStageBytes<EpiZ>::value <= kFStageBytesPerWarp &&
+                    EpiStageBytes<EpiDwStaged>::value <= kFStageBytesPerWarp,
+                "epilogue staging per warp");
   constexpr size_t kSmem = 1024 + kFStages * static_cast<size_t>(kFSlot) +
-                           sizeof(PairCtl<kFStages>) + sizeof(FusedQueue) +
-                           (kStage ? 1024 + kStage * 4 * kFNwg : 0);
+                           sizeof(PairCtl<kFStages>) + sizeof(FusedQueue) + 1024 +
+                           static_cast<size_t>(kFStageBytesPerWarp) * 4 * kFNwg;
   static_assert(kSmem <= 232448, "shared memory per CTA");
   auto kern = bwd_fused_kernel<DUAL, EpiZ>;
   cudaError_t e = cudaSuccess;

@@ -30,7 +30,7 @@
 //   EpiJsd      the two halves of the Jensen-Shannon divergence         (second pass)
 //   EpiDz       the logits gradient, rounded to bf16 into the chunk buffer (backward)
 //   EpiDh       dH chunk rows (bf16)                                      (dH = dZ W)
-//   EpiDw       fp32 read-add-write of disjoint dW tiles, no atomics      (dW += dZ^T H)
+//   EpiDwT      fp32 read-add-write of disjoint dW tiles, no atomics      (dW += dZ^T H)
 //   EpiFwdUnion, EpiPass2Union, EpiDzCombo   the same for weighted combinations
 //   EpiFlat     sum of exp and of its square                             (target flatness)
 // In the fused single call the forward epilogues also store the chunk's fp32 logits.
@@ -1197,28 +1197,44 @@ struct EpiDh {
   }
 };
 
-// dW tile: fp32 read-add-write (or plain write) of rows this CTA owns exclusively.
-struct EpiDw {
+// dW tile: fp32 read-add-write (or plain write) of rows this CTA owns exclusively, without
+// atomics.
+//   STAGED = true: each warp passes its 32 rows x 32 columns through a 4 KB shared-memory
+//     stage (16-byte chunk k of row r at position k ^ (r % 8), so that neither the writes
+//     nor the reads conflict), so that each global load and store instruction covers four
+//     whole 128-byte row segments, 8 lanes per row.  The persistent fused backward uses it.
+//   STAGED = false: each lane adds its own row's 32 columns, a 16-byte piece at a time.  The
+//     standalone dW GEMM uses it: there, with one epilogue warpgroup, the staged form was
+//     about 1% slower, while in the fused backward it made the kernel 1.4% faster.
+template <bool STAGED>
+struct EpiDwT {
   using Params = DwParams;
+  static constexpr int kStageBytesPerWarp = STAGED ? 4096 : 0;
+  float* stage;
   __device__ __forceinline__ void unit_begin(const Params&, int, int) {}
   __device__ __forceinline__ void unit_end(const Params&, int, int, int) {}
   template <int TN>
   __device__ __forceinline__ void tile(const Params& p, uint32_t tb, int row0, int64_t n0,
                                        int c0, int c1, int row) {
-    const int64_t v = static_cast<int64_t>(row0) + row;
-    const bool ok = v < p.V;
-    float* out = p.dW + v * p.d + n0;
+    const int lane = threadIdx.x & 31;
+    float4* st = reinterpret_cast<float4*>(stage);
+    const int64_t wrow0 = static_cast<int64_t>(row0) + row - lane;  // the warp's first row
+    const int sub = lane >> 3;  // row within each group of four
+    const int k = lane & 7;     // 16-byte chunk within the row's 32 columns
 #pragma unroll 1
     for (int c = c0; c < c1; c += 32) {
       float x[32];
       tmem_ld32(tb + c, x);
       tmem_ld_wait();
-      if (!ok || n0 + c >= p.d) continue;
+      if (!STAGED) {
+        const int64_t v = static_cast<int64_t>(row0) + row;
+        if (v >= p.V || n0 + c >= p.d) continue;
+        float* out = p.dW + v * p.d + n0 + c;
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        if (n0 + c + 4 * k + 4 <= p.d) {
-          float4* dst = reinterpret_cast<float4*>(out + c + 4 * k);
-          float4 r = make_float4(x[4 * k], x[4 * k + 1], x[4 * k + 2], x[4 * k + 3]);
+        for (int q = 0; q < 8; ++q) {
+          if (n0 + c + 4 * q >= p.d) break;
+          float4* dst = reinterpret_cast<float4*>(out + 4 * q);
+          float4 r = make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
           if (p.beta) {
             const float4 o = *dst;
             r.x += o.x;
@@ -1228,10 +1244,40 @@ struct EpiDw {
           }
           *dst = r;
         }
+        continue;
+      }
+      const int64_t col = n0 + c + 4 * k;
+      if (n0 + c >= p.d) continue;  // the whole block lies past d (warp-uniform)
+      __syncwarp();                 // every lane has read the previous block
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        st[lane * 8 + (q ^ (lane & 7))] =
+            make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
+      __syncwarp();
+#pragma unroll
+      for (int rr = 0; rr < 8; ++rr) {
+        const int r = rr * 4 + sub;
+        const int64_t v = wrow0 + r;
+        const float4 a = st[r * 8 + (k ^ (r & 7))];
+        // d % 8 == 0: a 4-column chunk that starts below d ends within the row.
+        if (v < p.V && col < p.d) {
+          float4* dst = reinterpret_cast<float4*>(p.dW + v * p.d + col);
+          float4 out = a;
+          if (p.beta) {
+            const float4 o = *dst;
+            out.x = a.x + o.x;
+            out.y = a.y + o.y;
+            out.z = a.z + o.z;
+            out.w = a.w + o.w;
+          }
+          *dst = out;
+        }
       }
     }
   }
 };
+using EpiDw = EpiDwT<false>;
+using EpiDwStaged = EpiDwT<true>;
 
 // ----------------------------------------------------------------------------------------
 // Target flatness ("Flatter Tokens are More Valuable for Speculative Draft Model
