@@ -356,6 +356,14 @@ SLM_API int slm_target_flatness(const void* Hp, const void* W, int64_t N, int64_
  * takes effect at the next launch.  Returns SLM_ERR_SHAPE for an invalid mode or bound. */
 SLM_API int slm_debug_set(int fault_mode, long long timeout_cycles);
 
+/* Test hook (not for production use): evaluates, for each x[i] (device float [n]), the
+ * 2^x that the loss epilogues compute on the FMA pipe for part of their exponentials
+ * (y_fma[i]), and CUDA's exp2f (y_mufu[i]).  The former rounds x to an integer j and
+ * evaluates 2^(x - j) by a degree-5 polynomial whose coefficients this library fitted; it is
+ * meant for x <= 0 and clamps x at -126.  Asynchronous on `stream`.  Returns SLM_ERR_SHAPE
+ * for n < 0 or n >= 2^31, SLM_ERR_NULL for a NULL buffer when n > 0. */
+SLM_API int slm_debug_exp2(const float* x, float* y_fma, float* y_mufu, int64_t n, void* stream);
+
 /* Size of the device scratch array behind slm_loss_fwd_noalloc: 32 MiB per GPU that loads
  * the library's device code, held until the process exits. */
 #define SLM_NOALLOC_SCRATCH_BYTES (32u << 20)

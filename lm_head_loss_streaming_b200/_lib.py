@@ -65,6 +65,7 @@ SIGNATURES = {
                                     _P, _P, _P, _P, _P, _P, _P, _P]),
     "slm_count_valid": (_INT, [_INT, _P, _I32, _I64, _I64, _P, _P]),
     "slm_set_backward_mode": (_INT, [_INT]),
+    "slm_debug_exp2": (_INT, [_P, _P, _P, _I64, _P]),
     "slm_trace_enable": (_INT, [_INT]),
     "slm_trace_read": (_INT, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_I64), _INT]),
 }
@@ -261,3 +262,8 @@ def slm_set_backward_mode(mode):
     """1: one persistent launch per backward chunk (default); 0: three launches per chunk.
     Returns the previous mode (-1: invalid mode, nothing changed)."""
     return load().slm_set_backward_mode(int(mode))
+
+
+def slm_debug_exp2(x, y_fma, y_mufu, n, stream):
+    """Test hook: the epilogues' FMA-pipe 2^x and CUDA's exp2f on the same device inputs."""
+    return load().slm_debug_exp2(x, y_fma, y_mufu, int(n), stream)

@@ -1018,6 +1018,17 @@ int slm_trace_read(double* ms, int64_t* launches, int n_classes) {
   return st;
 }
 
+int slm_debug_exp2(const float* x, float* y_fma, float* y_mufu, int64_t n, void* stream) {
+  if (n < 0 || n >= (int64_t(1) << 31)) return SLM_ERR_SHAPE;
+  if (n == 0) return SLM_OK;
+  if (!x || !y_fma || !y_mufu) return SLM_ERR_NULL;
+  int st = check_device();
+  if (st != SLM_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  SLM_LAUNCH(kTrRow, launch_exp2_pair(x, y_fma, y_mufu, n, s));
+  return SLM_OK;
+}
+
 int slm_debug_set(int fault_mode, long long timeout_cycles) {
   if (fault_mode < 0 || fault_mode > 2 || timeout_cycles < 0) return SLM_ERR_SHAPE;
   g_fault.store(fault_mode);

@@ -182,6 +182,10 @@ cudaError_t launch_logits_pass2(int kind, const float* lq, const float* lp, int6
 cudaError_t launch_logits_dz(const DzParams& p, const float* lq, const float* lp, int64_t ldl,
                              cudaStream_t s);
 
+// Test hook: the epilogues' FMA-pipe 2^x beside exp2f, elementwise.
+cudaError_t launch_exp2_pair(const float* x, float* y_fma, float* y_mufu, int64_t n,
+                             cudaStream_t s);
+
 // Draft-head helpers.
 constexpr int kFlatFields = 3;  // m, s, s2 = sum 2^(2 (z log2e - m))
 cudaError_t launch_align_labels(const int32_t* tokens, const uint8_t* loss_mask,

@@ -534,6 +534,49 @@ __device__ __forceinline__ float2 mul2(float2 a, float2 b) {
 }
 __device__ __forceinline__ float2 exp2_2(float2 a) { return make_float2(exp2f(a.x), exp2f(a.y)); }
 
+// 2^x for x <= 0 on the FMA pipe instead of the MUFU pipe, for a pair of values.  The
+// epilogues' exponentials are MUFU-bound while the FMA pipe idles, so a share of them is
+// computed this way (a share of the column pairs, see exp2_mix).  x = j + r with j = round(x) (adding 1.5 * 2^23 rounds to an
+// integer) and r in [-0.5, 0.5]; 2^r is a degree-5 polynomial in r whose coefficients were
+// fitted here to 2^r on [-0.5, 0.5] (relative error weighted least squares on Chebyshev
+// nodes: 7.5e-8 in exact arithmetic, 2.2e-7 in fp32 Horner form); 2^j is added into the
+// exponent field.  Arguments are clamped at -126 so that the exponent field stays
+// non-negative: the result is then at most 2^-126, which only ever enters sums of terms
+// >= 1.  Not for -inf arguments (the tail chunks, with masked columns, keep exp2f).
+__device__ __forceinline__ float2 exp2_fma2(float2 x) {
+  constexpr float kRound = 12582912.f;  // 1.5 * 2^23
+  x.x = fmaxf(x.x, -126.f);
+  x.y = fmaxf(x.y, -126.f);
+  const float2 kr = make_float2(kRound, kRound);
+  const float2 t = add2(x, kr);
+  const float2 r = sub2(x, sub2(t, kr));
+  float2 p = fma2(make_float2(0.001327647129073739f, 0.001327647129073739f), r,
+                  make_float2(0.009675540961325169f, 0.009675540961325169f));
+  p = fma2(p, r, make_float2(0.05550713092088699f, 0.05550713092088699f));
+  p = fma2(p, r, make_float2(0.24022120237350464f, 0.24022120237350464f));
+  p = fma2(p, r, make_float2(0.6931469440460205f, 0.6931469440460205f));
+  p = fma2(p, r, make_float2(1.0000001192092896f, 1.0000001192092896f));
+  const int jx = __float_as_int(t.x) - 0x4B400000;  // j, from the rounded sum's low bits
+  const int jy = __float_as_int(t.y) - 0x4B400000;
+  return make_float2(__int_as_float(__float_as_int(p.x) + (jx << 23)),
+                     __int_as_float(__float_as_int(p.y) + (jy << 23)));
+}
+
+// exp2_2 or exp2_fma2 for column pair `pair` of a 32-column chunk: pairs with
+// (pair % 8) < eighths take the FMA-pipe form.  `pair` is a constant once the chunk loop is
+// unrolled, so the choice costs nothing at run time.
+__device__ __forceinline__ float2 exp2_mix(int pair, int eighths, float2 x) {
+  return (pair & 7) < eighths ? exp2_fma2(x) : exp2_2(x);
+}
+// Shares for the kernels with two exponentials per column (target and draft: the second one
+// is mixed) and with one (hard-label CE).
+#ifndef SLM_EXP2_FMA_DUAL
+#define SLM_EXP2_FMA_DUAL 6
+#endif
+#ifndef SLM_EXP2_FMA_CE
+#define SLM_EXP2_FMA_CE 0
+#endif
+
 __device__ __forceinline__ void mask_tail(float (&v)[32], int64_t col0, int64_t V) {
 #pragma unroll
   for (int i = 0; i < 32; ++i)
@@ -622,7 +665,7 @@ struct EpiFwdCE {
         float2 a = make_float2(0.f, 0.f);
 #pragma unroll
         for (int i = 0; i < 32; i += 2)
-          a = add2(a, exp2_2(fma2(make_float2(v[i], v[i + 1]), l2, nm)));
+          a = add2(a, exp2_mix(i / 2, SLM_EXP2_FMA_CE, fma2(make_float2(v[i], v[i + 1]), l2, nm)));
         s += a.x + a.y;
 #else
         float a0 = 0.f, a1 = 0.f;
@@ -697,7 +740,7 @@ struct EpiFwdDualT {
         const float2 zq = make_float2(vq[i], vq[i + 1]);
         const float2 zp = make_float2(vp[i], vp[i + 1]);
         const float2 eq = exp2_2(fma2(zq, l2, nmq));
-        const float2 e = exp2_2(fma2(zp, l2, nmp));
+        const float2 e = exp2_mix(i / 2, SLM_EXP2_FMA_DUAL, fma2(zp, l2, nmp));
         sq2 = add2(sq2, eq);
         sp2 = add2(sp2, e);
         if (ACC & 1) a2 = fma2(e, sub2(zp, zq), a2);
@@ -1050,8 +1093,13 @@ struct EpiDz {
 
   // vq (draft logits of columns [col0, col0 + 32)) becomes dz; vp holds the target logits
   // of the same columns (unused for CE).
-  __device__ __forceinline__ void apply(float (&vq)[32], const float (&vp)[32],
-                                        int64_t col0) const {
+  // fma_cols: which columns take the FMA-pipe 2^x for the target (KL): -1 = element i is
+  // column col0 + i with col0 a multiple of 32 (the GEMM epilogue), so the share rule of
+  // exp2_mix applies by position; 0 / 1 = every element of this call is / is not in such a
+  // column (the row kernel, whose elements come from columns with one rule per thread).
+  // Either way a column's exponential is computed the same way on both paths.
+  __device__ __forceinline__ void apply(float (&vq)[32], const float (&vp)[32], int64_t col0,
+                                        int fma_cols = -1) const {
     if (DUAL) {
       {
         if (mode == 0) {
@@ -1062,7 +1110,9 @@ struct EpiDz {
 #pragma unroll
           for (int i = 0; i < 32; i += 2) {
             const float2 qv = exp2_2(fma2(make_float2(vq[i], vq[i + 1]), l2, nq));
-            const float2 pv = exp2_2(fma2(make_float2(vp[i], vp[i + 1]), l2, np));
+            const float2 ap = fma2(make_float2(vp[i], vp[i + 1]), l2, np);
+            const float2 pv = fma_cols < 0 ? exp2_mix(i / 2, SLM_EXP2_FMA_DUAL, ap)
+                                           : (fma_cols ? exp2_fma2(ap) : exp2_2(ap));
             const float2 r = mul2(ck2, sub2(qv, pv));
             vq[i] = r.x;
             vq[i + 1] = r.y;
@@ -1110,7 +1160,8 @@ struct EpiDz {
       const float2 g2 = make_float2(g, g);
 #pragma unroll
       for (int i = 0; i < 32; i += 2) {
-        const float2 qv = exp2_2(fma2(make_float2(vq[i], vq[i + 1]), l2, nq));
+        const float2 qv =
+            exp2_mix(i / 2, SLM_EXP2_FMA_CE, fma2(make_float2(vq[i], vq[i + 1]), l2, nq));
         const float2 oh = make_float2(rel == i ? 1.f : 0.f, rel == i + 1 ? 1.f : 0.f);
         const float2 r = mul2(g2, sub2(qv, oh));
         vq[i] = r.x;
@@ -2271,7 +2322,15 @@ __global__ void __launch_bounds__(256)
       }
     }
     if (DUAL) {
-      e.apply(vq, vp, 0);  // elementwise: no column enters the divergences' formulas
+      // Elementwise: no column enters the divergences' formulas, except in choosing how
+      // the target's 2^x is computed, which must match the GEMM epilogue's choice for the
+      // same column: the FMA-pipe form for columns with ((c / 2) % 8) < the share.  This
+      // thread's columns are 4 t + j + multiples of 16 (j < 4): their (c / 2) % 8 is
+      // 2 (t % 4) or 2 (t % 4) + 1, on the same side of an even share, so the rule is one per
+      // thread.
+      static_assert(SLM_EXP2_FMA_DUAL % 2 == 0, "one rule per thread needs an even share");
+      const int c16 = static_cast<int>((4 * threadIdx.x) & 15);
+      e.apply(vq, vp, 0, (c16 >> 1) < SLM_EXP2_FMA_DUAL ? 1 : 0);
     } else {
       // CE: the same formula as the GEMM epilogue's, with each value's own column.
 #pragma unroll
@@ -2386,6 +2445,32 @@ cudaError_t launch_flat_combine(const float* part, int nch, int64_t N, int64_t V
   return cudaGetLastError();
 }
 
+}  // namespace slm
+
+namespace slm {
+// Test hook: the FMA-pipe exponential and the MUFU one (exp2f) side by side.
+__global__ void exp2_pair_kernel(const float* __restrict__ x, float* y_fma, float* y_mufu,
+                                 int64_t n) {
+  const int64_t i = 2 * (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  const float2 a = make_float2(x[i], i + 1 < n ? x[i + 1] : 0.f);
+  const float2 f = exp2_fma2(a);
+  y_fma[i] = f.x;
+  y_mufu[i] = exp2f(a.x);
+  if (i + 1 < n) {
+    y_fma[i + 1] = f.y;
+    y_mufu[i + 1] = exp2f(a.y);
+  }
+}
+
+cudaError_t launch_exp2_pair(const float* x, float* y_fma, float* y_mufu, int64_t n,
+                             cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  const int64_t pairs = (n + 1) / 2;
+  exp2_pair_kernel<<<static_cast<unsigned>((pairs + 255) / 256), 256, 0, s>>>(x, y_fma, y_mufu,
+                                                                               n);
+  return cudaGetLastError();
+}
 }  // namespace slm
 
 // The persistent fused backward (one launch per chunk for the logits gradient, dH and dW).
