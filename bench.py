@@ -160,8 +160,8 @@ def kernel_source_hash():
 def traffic_for(workload, kind, kernel):
     """DRAM bytes per launch of `kernel` from the committed ncu summary, or None when the
     kernel sources changed since the counters were taken."""
-    if not os.path.exists(TRAFFIC_FILE):
-        return None
+    if not os.path.exists(TRAFFIC_FILE) or os.environ.get("SLM_LIBRARY"):
+        return None  # the counters belong to the in-tree build of these sources
     cur = kernel_source_hash()
     with open(TRAFFIC_FILE) as f:
         for line in f:
@@ -714,6 +714,8 @@ def run_ours(args):
         "fused": fused_info,
         "kernel_sha": kernel_source_hash(),
     }
+    if os.environ.get("SLM_LIBRARY"):
+        out["library"] = os.environ["SLM_LIBRARY"]
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rows = args.cpu_sample_rows or 128
         out["cpu_baseline"] = cpu_baseline_block(args.workload, kind, rows)

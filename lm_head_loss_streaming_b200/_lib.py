@@ -11,7 +11,8 @@ import ctypes
 import os
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libslm.so")
+# The in-tree build, or a variant built with `build --out PATH -D ...` named by SLM_LIBRARY.
+LIB_PATH = os.path.abspath(os.environ.get("SLM_LIBRARY") or os.path.join(HERE, "libslm.so"))
 
 SLM_CE, SLM_KL, SLM_TV, SLM_NLA, SLM_LK_HYBRID = 0, 1, 2, 3, 4
 SLM_RKL, SLM_JSD, SLM_CE_ARGMAX_P = 5, 6, 7

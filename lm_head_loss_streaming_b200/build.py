@@ -1,6 +1,12 @@
 """Build ``libslm.so`` in-tree with nvcc for sm_100a (B200).
 
-    python -m lm_head_loss_streaming_b200.build [--verbose]
+    python -m lm_head_loss_streaming_b200.build [--verbose] [--force]
+    python -m lm_head_loss_streaming_b200.build --out _build/g1/libslm.so -D SLM_GROUP_B=1
+
+The second form builds a variant library elsewhere with extra preprocessor definitions:
+the GEMM schedule's knobs in ``csrc/slm_schedule.h`` (``SLM_GROUP_PAIRS``, ``SLM_MAX_RUNS``,
+``SLM_GROUP_B``, ``SLM_SYNC_*``) are overridable that way.  ``SLM_LIBRARY=<path>`` makes
+the Python binding load such a library instead of the in-tree one.
 
 The library is plain CUDA C++ behind a C ABI: no PyTorch headers, no JIT cache.  The CUDA
 runtime is linked statically; the driver's tensor-map encoder is fetched at run time, so
@@ -42,18 +48,27 @@ def _newer(target, deps):
     return all(os.path.getmtime(d) <= t for d in deps)
 
 
-def build(verbose=False, force=False, ptxas_verbose=False):
-    os.makedirs(BUILD_DIR, exist_ok=True)
+def build(verbose=False, force=False, ptxas_verbose=False, out=None, defines=()):
+    """Build the library (in-tree by default; at `out`, with `defines` as extra -D
+    definitions, for a variant).  Returns its path."""
+    lib = os.path.abspath(out) if out else LIB
+    defines = list(defines)
+    for dfn in defines:
+        if not dfn.replace("=", "").replace("_", "").replace("-", "").isalnum():
+            raise ValueError(f"bad definition {dfn!r}: expected NAME or NAME=VALUE")
+    obj_dir = BUILD_DIR if not out else os.path.join(os.path.dirname(lib), "_obj")
+    os.makedirs(obj_dir, exist_ok=True)
     headers = [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".h", ".cuh"))]
     headers.append(os.path.join(INCLUDE, "slm.h"))
     srcs = [os.path.join(CSRC, s) for s in SOURCES]
-    if not force and _newer(LIB, srcs + headers + [os.path.abspath(__file__)]):
-        return LIB
+    if not force and not out and _newer(lib, srcs + headers + [os.path.abspath(__file__)]):
+        return lib
     exe = nvcc()
     extra = ["-Xptxas", "-v"] if ptxas_verbose else []
+    extra += ["-D" + dfn for dfn in defines]
 
     def compile_one(src):
-        obj = os.path.join(BUILD_DIR, os.path.basename(src) + ".o")
+        obj = os.path.join(obj_dir, os.path.basename(src) + ".o")
         cmd = [exe, *ARCH, *FLAGS, *extra, "-c", src, "-o", obj]
         if verbose:
             print(" ".join(cmd), flush=True)
@@ -66,18 +81,29 @@ def build(verbose=False, force=False, ptxas_verbose=False):
 
     with ThreadPoolExecutor(len(srcs)) as ex:
         objs = list(ex.map(compile_one, srcs))
-    tmp = LIB + ".tmp"
+    tmp = lib + ".tmp"
     cmd = [exe, *ARCH, "-shared", "-o", tmp, *objs, "-cudart", "static"]
     if verbose:
         print(" ".join(cmd), flush=True)
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    build(verbose="--verbose" in sys.argv, force="--force" in sys.argv,
-          ptxas_verbose="--ptxas-verbose" in sys.argv)
-    print(LIB)
+    import argparse
+
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--verbose", action="store_true")
+    ap.add_argument("--force", action="store_true")
+    ap.add_argument("--ptxas-verbose", action="store_true")
+    ap.add_argument("--out", default=None, help="build a variant library at this path")
+    ap.add_argument("-D", dest="defines", action="append", default=[],
+                    help="extra preprocessor definition (NAME or NAME=VALUE) for --out")
+    a = ap.parse_args()
+    if a.defines and not a.out:
+        ap.error("-D needs --out: the in-tree library keeps the default schedule")
+    print(build(verbose=a.verbose, force=a.force, ptxas_verbose=a.ptxas_verbose, out=a.out,
+                defines=a.defines))

@@ -106,6 +106,20 @@ __device__ __forceinline__ bool wait_count(const int* ctr, int target, volatile 
   return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
+// Unit u of a num_m x num_n grid in raster groups of `group` M tiles: the groups in order,
+// within a group the N tiles in order and the M tiles fastest.  Units claimed one after the
+// other then share their N-tile operand, and the pairs running at one time read the
+// operands of about `group` M tiles and 74 / `group` N tiles.
+__device__ __forceinline__ void grouped_coords(int u, int num_m, int num_n, int group, int& mt,
+                                               int& nt) {
+  const int per_group = group * num_n;
+  const int grp = u / per_group;
+  const int r = u - grp * per_group;
+  const int gm = min(group, num_m - grp * group);
+  nt = r / gm;
+  mt = grp * group + (r - nt * gm);
+}
+
 // Unit u of the claim order -> kind (0: Z, 1: H, 2: W) and its two coordinates: (M tile,
 // vocabulary run) for Z, (M tile, N tile) for H and W.
 __device__ __forceinline__ int fused_unit(const BwdFusedGeom& fg, int u, int& a, int& b) {
@@ -117,13 +131,10 @@ __device__ __forceinline__ int fused_unit(const BwdFusedGeom& fg, int u, int& a,
   u -= uz;
   const int uh = fg.num_mh * fg.num_nh;
   if (u < uh) {
-    a = u / fg.num_nh;
-    b = u - a * fg.num_nh;
+    grouped_coords(u, fg.num_mh, fg.num_nh, fg.group_h, a, b);
     return 1;
   }
-  u -= uh;
-  a = u / fg.num_nw;
-  b = u - a * fg.num_nw;
+  grouped_coords(u - uh, fg.num_mw, fg.num_nw, fg.group_w, a, b);
   return 2;
 }
 

@@ -129,6 +129,7 @@ struct BwdFusedGeom {
   int kb_h;              // H K blocks (over V)
   int num_mw, num_nw;    // W units: 256-row tiles of the vocabulary x 256-column tiles of d
   int kb_w;              // W K blocks (over the chunk's rows)
+  int group_h, group_w;  // M tiles per raster group of the H and W units (M tile fastest)
   int* claim;            // next unit to claim (zero at launch)
   int* rows_done;        // [gz.num_m] finished Z units per M tile, x kFusedEpiWarps
   int* runs_done;        // [gz.units_n] finished Z units per vocabulary run, x kFusedEpiWarps

@@ -23,6 +23,14 @@ namespace {
 // Loose lockstep of the GEMMs' CTA pairs (K blocks per progress step, steps of slack; 0 K
 // blocks = off): V for the GEMMs over the vocabulary (forward, logits gradient, second
 // pass), B for the dH and dW GEMMs.
+// Raster groups of the persistent backward's dH and dW units (M tiles per group, M tile
+// fastest).  Its pairs claim units one at a time and drift out of phase, so only units
+// claimed close together share operands in L2; the groups put the units that share an
+// operand next to each other.  The separate dH and dW launches start all pairs together
+// and keep the plain row-major order.
+#ifndef SLM_GROUP_B
+#define SLM_GROUP_B 8
+#endif
 #ifndef SLM_SYNC_KB_V
 #define SLM_SYNC_KB_V 16
 #endif
@@ -38,6 +46,7 @@ namespace {
 constexpr int kPairM = 2 * kBM;                // M rows of one 2-SM tile
 constexpr int kGroupPairs = SLM_GROUP_PAIRS;   // pair M tiles per raster group
 constexpr int kMaxRuns = SLM_MAX_RUNS;         // vocabulary runs per row, at most
+constexpr int kGroupB = SLM_GROUP_B;           // M tiles per group of fused dH / dW units
 
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 

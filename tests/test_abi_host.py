@@ -41,6 +41,30 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
         _lib.load()
 
 
+def test_library_override_names_the_missing_file(tmp_path):
+    """SLM_LIBRARY points the binding at a variant build; a wrong path fails on load, naming
+    the path, and never falls back to the in-tree build."""
+    import subprocess
+    import sys
+
+    missing = str(tmp_path / "variant" / "libslm.so")
+    code = ("from lm_head_loss_streaming_b200 import _lib\n"
+            "try:\n    _lib.load()\nexcept ImportError as e:\n    print('IMPORTERROR', e)\n")
+    env = dict(os.environ, SLM_LIBRARY=missing)
+    r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, env=env, capture_output=True,
+                       text=True, timeout=120)
+    assert r.returncode == 0, r.stderr
+    assert "IMPORTERROR" in r.stdout and missing in r.stdout
+
+
+def test_variant_build_rejects_bad_definitions(tmp_path):
+    from lm_head_loss_streaming_b200.build import build
+
+    for bad in ("SLM_GROUP_B=1;rm", "A B", "X=$(y)"):
+        with pytest.raises(ValueError):
+            build(out=str(tmp_path / "libslm.so"), defines=[bad])
+
+
 def test_status_strings_and_sizes(lib):
     assert _lib.slm_version() >= 100
     for code, name in _lib.STATUS_NAMES.items():

@@ -74,10 +74,13 @@ def test_fused_backward_is_bitwise_the_three_launch_backward(kind):
 @pytest.mark.parametrize("kind,shape,chunk", [("ce", (1, 8, 50), 0), ("kl_div", (129, 64, 257), 0),
                                               ("tv", (300, 16, 4100), 128),
                                               ("ce", (2000, 128, 700), 0),
-                                              ("jsd", (513, 520, 1000), 384)])
+                                              ("jsd", (513, 520, 1000), 384),
+                                              ("kl_div", (2600, 520, 3500), 2304),
+                                              ("ce", (2600, 136, 2100), 2560)])
 def test_fused_backward_edge_shapes(kind, shape, chunk):
     """One row, fewer units than pairs, one vocabulary tile, a d of two N tiles, chunks that
-    are not multiples of 256."""
+    are not multiples of 256, and dH / dW unit grids whose last raster group of M tiles is
+    short (9 and 10 chunk M tiles, 14 and 9 vocabulary M tiles, in groups of 8)."""
     inp = synthetic.make(kind, *shape, w_std=0.1, ignore_frac=0.1 if shape[0] > 1 else 0.0,
                          seed=92)
     (h0, w0), (h1, w1) = _bwd_both(kind, inp, chunk=chunk)
