@@ -663,7 +663,8 @@ def run_ours(args):
     else:  # nothing traced (should not happen): fall back to the forward events
         dom = "fwd_gemm"
         achieved = cflops["fwd_gemm"] / (fwd_ms / 1e3) / 1e12
-    traffic = traffic_for(args.workload, kind, dom)
+    # The fused call's forward GEMM also stores the chunk's logits: its own traffic key.
+    traffic = traffic_for(args.workload, kind, dom + ("@fused" if args.fused else ""))
     out = {
         "metric": METRIC,
         "value": round(tokens_per_s, 1),
