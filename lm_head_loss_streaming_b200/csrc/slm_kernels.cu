@@ -533,6 +533,11 @@ __device__ __forceinline__ float2 mul2(float2 a, float2 b) {
   return d;
 }
 __device__ __forceinline__ float2 exp2_2(float2 a) { return make_float2(exp2f(a.x), exp2f(a.y)); }
+// log2 of a pair of sums of probabilities; a sum of 0 (both terms underflowed or masked)
+// gives -126 instead of -inf, so that the terms it multiplies stay 0.
+__device__ __forceinline__ float2 log2_2(float2 a) {
+  return make_float2(log2f(fmaxf(a.x, 1.1754944e-38f)), log2f(fmaxf(a.y, 1.1754944e-38f)));
+}
 
 // 2^x for x <= 0 on the FMA pipe instead of the MUFU pipe, for a pair of values.  The
 // epilogues' exponentials are MUFU-bound while the FMA pipe idles, so a share of them is
@@ -577,10 +582,11 @@ __device__ __forceinline__ float2 exp2_mix(int pair, int eighths, float2 x) {
 #define SLM_EXP2_FMA_CE 0
 #endif
 
-__device__ __forceinline__ void mask_tail(float (&v)[32], int64_t col0, int64_t V) {
+__device__ __forceinline__ void mask_tail(float (&v)[32], int64_t col0, int64_t V,
+                                          float fill = -INFINITY) {
 #pragma unroll
   for (int i = 0; i < 32; ++i)
-    if (col0 + i >= V) v[i] = -INFINITY;
+    if (col0 + i >= V) v[i] = fill;
 }
 
 // Fused path: this warp's 32 rows x 32 columns of fp32 logits (each lane holds its row's
@@ -964,27 +970,34 @@ struct EpiJsd {
       tmem_ld32(tb + TN + c, vp);
       tmem_ld_wait();
       if (n0 + c + 32 > p.V) {
-        mask_tail(vq, n0 + c, p.V);
-        mask_tail(vp, n0 + c, p.V);
+        // A finite fill: both exponentials of a masked column are 0 and so are its terms
+        // (a -inf logit would give 0 * -inf).
+        mask_tail(vq, n0 + c, p.V, -1e30f);
+        mask_tail(vp, n0 + c, p.V, -1e30f);
       }
+      const float2 l2 = make_float2(kLog2e, kLog2e);
+      const float2 nq = make_float2(-lq2, -lq2), np = make_float2(-lp2, -lp2);
+      float2 ap2 = make_float2(0.f, 0.f), aq2 = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const float qv = exp2f(fmaf(vq[i], kLog2e, -lq2));
-        const float pv = exp2f(fmaf(vp[i], kLog2e, -lp2));
-        const float ms = pv + qv;
-        if (ms > 0.f) {  // both 0 (masked or underflowed) contributes nothing
-          const float lm = log2f(0.5f * ms) * kLn2;
-          jp = fmaf(pv, (vp[i] - lp) - lm, jp);
-          jq = fmaf(qv, (vq[i] - lq) - lm, jq);
-        }
+      for (int i = 0; i < 32; i += 2) {
+        const float2 a = fma2(make_float2(vp[i], vp[i + 1]), l2, np);  // log2 p
+        const float2 b = fma2(make_float2(vq[i], vq[i + 1]), l2, nq);  // log2 q
+        // log2 p - log2 M = a + w and log2 q - log2 M = b + w, w = 1 - log2(p + q).
+        const float2 pv = exp2_2(a), qv = exp2_2(b);
+        const float2 w = sub2(make_float2(1.f, 1.f), log2_2(add2(pv, qv)));
+        ap2 = fma2(pv, add2(a, w), ap2);
+        aq2 = fma2(qv, add2(b, w), aq2);
       }
+      jp += ap2.x + ap2.y;
+      jq += aq2.x + aq2.y;
     }
   }
 
+  // jp and jq were summed in log2 units.
   __device__ __forceinline__ void unit_end(const Params& p, int, int slot, int) {
     if (!row_ok) return;
-    p.part[(static_cast<int64_t>(slot) * 2 + 0) * p.N + grow] = jp;
-    p.part[(static_cast<int64_t>(slot) * 2 + 1) * p.N + grow] = jq;
+    p.part[(static_cast<int64_t>(slot) * 2 + 0) * p.N + grow] = jp * kLn2;
+    p.part[(static_cast<int64_t>(slot) * 2 + 1) * p.N + grow] = jq * kLn2;
   }
 };
 
@@ -1126,30 +1139,51 @@ struct EpiDz {
           }
 #endif
         } else if (mode == 3) {
+          // alpha-based kinds: dz = ck (q - p) + cm q ([q < p] - S), two columns at a time.
+          const float2 l2 = make_float2(kLog2e, kLog2e);
+          const float2 nq = make_float2(-lq2, -lq2), np = make_float2(-lp2, -lp2);
+          const float2 ck2 = make_float2(ck, ck), cm2 = make_float2(cm, cm);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float qv = exp2f(fmaf(vq[i], kLog2e, -lq2));
-            const float pv = exp2f(fmaf(vp[i], kLog2e, -lp2));
-            const float mS = ((qv < pv) ? 1.f : 0.f) - S;
-            vq[i] = fmaf(ck, qv - pv, cm * qv * mS);
+          for (int i = 0; i < 32; i += 2) {
+            const float2 qv = exp2_2(fma2(make_float2(vq[i], vq[i + 1]), l2, nq));
+            const float2 pv = exp2_2(fma2(make_float2(vp[i], vp[i + 1]), l2, np));
+            const float2 mS = make_float2(((qv.x < pv.x) ? 1.f : 0.f) - S,
+                                          ((qv.y < pv.y) ? 1.f : 0.f) - S);
+            const float2 r = fma2(ck2, sub2(qv, pv), mul2(mul2(cm2, qv), mS));
+            vq[i] = r.x;
+            vq[i + 1] = r.y;
           }
         } else if (mode == 1) {
+          // Reverse KL: dz = ck q ((z_q - z_p) - c), two columns at a time.
+          const float2 l2 = make_float2(kLog2e, kLog2e), nq = make_float2(-lq2, -lq2);
+          const float2 ck2 = make_float2(ck, ck), cm2 = make_float2(cm, cm);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float qv = exp2f(fmaf(vq[i], kLog2e, -lq2));
-            vq[i] = ck * qv * ((vq[i] - vp[i]) - cm);
+          for (int i = 0; i < 32; i += 2) {
+            const float2 z = make_float2(vq[i], vq[i + 1]);
+            const float2 qv = exp2_2(fma2(z, l2, nq));
+            const float2 r =
+                mul2(mul2(ck2, qv), sub2(sub2(z, make_float2(vp[i], vp[i + 1])), cm2));
+            vq[i] = r.x;
+            vq[i + 1] = r.y;
           }
         } else {
+          // JSD: dz = g q ((log q - log M) / 2 - T), M = (p + q) / 2.  In log2 units, with
+          // b = log2 q: log2 q - log2 M = b + w, w = 1 - log2(p + q), so
+          // dz = q (k1 (b + w) - g T), k1 = g ln2 / 2.  Two columns at a time, no branch.
+          const float2 l2 = make_float2(kLog2e, kLog2e);
+          const float2 nq = make_float2(-lq2, -lq2), np = make_float2(-lp2, -lp2);
+          const float2 k1 = make_float2(0.5f * kLn2 * ck, 0.5f * kLn2 * ck);
+          const float2 gt = make_float2(ck * S, ck * S);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float qv = exp2f(fmaf(vq[i], kLog2e, -lq2));
-            const float pv = exp2f(fmaf(vp[i], kLog2e, -lp2));
-            float dz = 0.f;
-            if (qv > 0.f) {
-              const float lm = log2f(0.5f * (pv + qv)) * kLn2;
-              dz = ck * qv * (0.5f * ((vq[i] - lq) - lm) - S);
-            }
-            vq[i] = dz;
+          for (int i = 0; i < 32; i += 2) {
+            const float2 a = fma2(make_float2(vp[i], vp[i + 1]), l2, np);  // log2 p
+            const float2 b = fma2(make_float2(vq[i], vq[i + 1]), l2, nq);  // log2 q
+            // log2 q - log2 M = b + w, w = 1 - log2(p + q).
+            const float2 q = exp2_2(b);
+            const float2 w = sub2(make_float2(1.f, 1.f), log2_2(add2(exp2_2(a), q)));
+            const float2 r = mul2(q, sub2(mul2(k1, add2(b, w)), gt));
+            vq[i] = r.x;
+            vq[i + 1] = r.y;
           }
         }
       }

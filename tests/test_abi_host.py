@@ -171,6 +171,11 @@ def test_debug_hook_arguments(lib):
     assert _lib.slm_debug_set(-1, 0) == 2
     assert _lib.slm_debug_set(0, -1) == 2    # SLM_ERR_SHAPE: negative bound
     assert _lib.slm_debug_set(0, 0) == 0     # back to normal operation
+    for fn in (_lib.slm_debug_exp2,):
+        assert fn(None, None, None, 0, None) == 0          # nothing to do
+        assert fn(None, None, None, 5, None) == 1          # SLM_ERR_NULL
+        assert fn(None, None, None, -1, None) == 2         # SLM_ERR_SHAPE
+        assert fn(None, None, None, 1 << 31, None) == 2
 
 
 def _combo_fwd(weights, **kw):
