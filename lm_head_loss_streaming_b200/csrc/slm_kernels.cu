@@ -206,6 +206,19 @@ struct EpiStageBytes<E, decltype(void(E::kStageBytesPerWarp))> {
   static constexpr int value = E::kStageBytesPerWarp;
 };
 
+// Epilogues that set kSplitHalves take a single-buffered two-sub-tile accumulator in two
+// halves (see gemm_pair_kernel): each warpgroup drains its share of the first sub-tile,
+// releases it, then drains its share of the second.  Their tile() must accept any 32-column-aligned
+// sub-range [c0, c1) and not depend on the order in which the ranges come.
+template <class E, class = void>
+struct EpiSplit {
+  static constexpr bool value = false;
+};
+template <class E>
+struct EpiSplit<E, decltype(void(E::kSplitHalves))> {
+  static constexpr bool value = E::kSplitHalves;
+};
+
 // Epilogues with asynchronous work of their own (bulk stores) declare finish(), which the
 // kernel calls once after the epilogue's last tile.
 template <class E, class = void>
@@ -232,6 +245,14 @@ __global__ void __launch_bounds__(64 + 128 * NWG, 1)
   constexpr uint32_t kStageBytes = C::kStageBytes;
   constexpr uint32_t kAccCols = C::kAccCols;
   constexpr uint32_t kIdesc = idesc_bf16_f32(2 * kBM, BNI, A_MN, B_MN);
+  // Split accumulator (single buffer, two N sub-tiles, an epilogue that takes halves): the
+  // sub-tiles have their own "empty" barriers, so the next tile's MMAs for sub-tile 0 start
+  // while the epilogue still drains sub-tile 1.  (Halving the N = 256 MMAs of the
+  // two-operand tiles the same way measured slower: N = 128 MMAs read each A tile from
+  // shared memory twice per K step, which with the TMA writes exceeds the shared-memory
+  // port.)
+  constexpr bool kSplit = NBUF == 1 && NSUB == 2 && EpiSplit<Epi>::value;
+  static_assert(!kSplit || (!A_MN && !B_MN), "split accumulators: K-major operands");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -375,37 +396,99 @@ __global__ void __launch_bounds__(64 + 128 * NWG, 1)
           }
           tc_fence_after();
           const uint32_t dcol = tmem + b * kAccCols;
-          for (int kb = 0; kb < g.k_blocks; ++kb, ++it) {
-            const int s = it % STAGES;
-            const uint32_t ph = (it / STAGES) & 1u;
-            if (!wait_warp(&pc->full[s], ph, abort, ctl)) {
+          if constexpr (kSplit) {
+            // Sub-tile h's MMAs of one stage (first = the tile's first K block).
+            auto issue_half = [&](int st, int h, bool first) {
+              const uint32_t a_addr = smem_u32(smem + st * kStageBytes);
+              const uint32_t bs = a_addr + NUM_A * kABytes + h * kSliceBytes;
+#pragma unroll
+              for (int kk = 0; kk < kBK / 16; ++kk) {
+                const uint64_t bd = smem_desc_sw128(bs + kk * 32, 16, 1024);
+#pragma unroll
+                for (int a = 0; a < NUM_A; ++a) {
+                  const uint64_t ad = smem_desc_sw128(a_addr + a * kABytes + kk * 32, 16, 1024);
+                  umma_bf16_pair(dcol + (a * NSUB + h) * BNI, ad, bd, kIdesc,
+                                 (!first || kk != 0) ? 1u : 0u);
+                }
+              }
+            };
+            // Sub-tile 0 over the first `pre` K blocks (the stages the producer filled while
+            // the epilogue drained), then, once sub-tile 1 is free, its MMAs for those K
+            // blocks with each stage's release, then both sub-tiles per K block.
+            const int pre = min(STAGES, g.k_blocks);
+            const uint32_t it0 = it;
+            for (int kb = 0; ok && kb < pre; ++kb) {
+              const int st = (it0 + kb) % STAGES;
+              if (!wait_warp(&pc->full[st], ((it0 + kb) / STAGES) & 1u, abort, ctl)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              if (lane == 0) issue_half(st, 0, kb == 0);
+              __syncwarp();
+            }
+            if (!ok) break;
+            if (!wait_warp(&pc->tempty[1], ub ^ 1u, abort, ctl)) {
               ok = false;
               break;
             }
             tc_fence_after();
-            if (lane == 0) {
-              const uint32_t a_addr = smem_u32(smem + s * kStageBytes);
-              const uint32_t b_addr = a_addr + NUM_A * kABytes;
+            for (int kb = 0; kb < pre; ++kb) {
+              const int st = (it0 + kb) % STAGES;
+              if (lane == 0) {
+                issue_half(st, 1, kb == 0);
+                umma_commit_pair_mc(&pc->empty[st], 0x3);
+              }
+              __syncwarp();
+            }
+            it = it0 + pre;
+            for (int kb = pre; kb < g.k_blocks; ++kb, ++it) {
+              const int st = it % STAGES;
+              if (!wait_warp(&pc->full[st], (it / STAGES) & 1u, abort, ctl)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              if (lane == 0) {
+                issue_half(st, 0, false);
+                issue_half(st, 1, false);
+                umma_commit_pair_mc(&pc->empty[st], 0x3);
+              }
+              __syncwarp();
+            }
+          } else {
+            for (int kb = 0; kb < g.k_blocks; ++kb, ++it) {
+              const int s = it % STAGES;
+              const uint32_t ph = (it / STAGES) & 1u;
+              if (!wait_warp(&pc->full[s], ph, abort, ctl)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              if (lane == 0) {
+                const uint32_t a_addr = smem_u32(smem + s * kStageBytes);
+                const uint32_t b_addr = a_addr + NUM_A * kABytes;
 #pragma unroll
-              for (int kk = 0; kk < kBK / 16; ++kk) {
+                for (int kk = 0; kk < kBK / 16; ++kk) {
 #pragma unroll
-                for (int sub = 0; sub < NSUB; ++sub) {
-                  const uint32_t bs = b_addr + sub * kSliceBytes;
-                  const uint64_t bd = B_MN ? smem_desc_sw128(bs + kk * 2048, 8192, 1024)
-                                           : smem_desc_sw128(bs + kk * 32, 16, 1024);
+                  for (int sub = 0; sub < NSUB; ++sub) {
+                    const uint32_t bs = b_addr + sub * kSliceBytes;
+                    const uint64_t bd = B_MN ? smem_desc_sw128(bs + kk * 2048, 8192, 1024)
+                                             : smem_desc_sw128(bs + kk * 32, 16, 1024);
 #pragma unroll
-                  for (int a = 0; a < NUM_A; ++a) {
-                    const uint32_t aa = a_addr + a * kABytes;
-                    const uint64_t ad = A_MN ? smem_desc_sw128(aa + kk * 2048, 8192, 1024)
-                                             : smem_desc_sw128(aa + kk * 32, 16, 1024);
-                    umma_bf16_pair(dcol + (a * NSUB + sub) * BNI, ad, bd, kIdesc,
-                                   (kb | kk) != 0 ? 1u : 0u);
+                    for (int a = 0; a < NUM_A; ++a) {
+                      const uint32_t aa = a_addr + a * kABytes;
+                      const uint64_t ad = A_MN ? smem_desc_sw128(aa + kk * 2048, 8192, 1024)
+                                               : smem_desc_sw128(aa + kk * 32, 16, 1024);
+                      umma_bf16_pair(dcol + (a * NSUB + sub) * BNI, ad, bd, kIdesc,
+                                     (kb | kk) != 0 ? 1u : 0u);
+                    }
                   }
                 }
+                umma_commit_pair_mc(&pc->empty[s], 0x3);
               }
-              umma_commit_pair_mc(&pc->empty[s], 0x3);
+              __syncwarp();
             }
-            __syncwarp();
           }
           if (!ok) break;
           if (lane == 0) umma_commit_pair_mc(&pc->tfull[b], 0x3);
@@ -451,14 +534,30 @@ __global__ void __launch_bounds__(64 + 128 * NWG, 1)
           break;
         }
         tc_fence_after();
-        epi.template tile<kTileN>(ep, tmem + lane_bits + b * kAccCols, row0,
-                                  static_cast<int64_t>(nt) * kTileN, c0, c1, row);
-        tc_fence_before();
-        __syncwarp();
         // Test hook (fault == 1): withhold the release of the first accumulator, so that the
         // MMA issuer's bounded wait for it runs out and the kernel unwinds with a timeout.
         const bool withhold = ctl.fault == 1 && t == 0;
-        if (lane == 0 && !withhold) mbar_arrive_cluster(b ? tempty_leader1 : tempty_leader0);
+        if constexpr (kSplit) {
+          // This warpgroup's share of each sub-tile in turn, each released once drained.
+          constexpr int kHalf = kTileN / 2, kPer = kHalf / NWG;
+          static_assert(kPer % 32 == 0, "split epilogue share");
+#pragma unroll 1
+          for (int h = 0; h < 2; ++h) {
+            const int ch = h * kHalf + wg * kPer;
+            epi.template tile<kTileN>(ep, tmem + lane_bits, row0,
+                                      static_cast<int64_t>(nt) * kTileN, ch, ch + kPer, row);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0 && !(withhold && h == 0))
+              mbar_arrive_cluster(h ? tempty_leader1 : tempty_leader0);
+          }
+        } else {
+          epi.template tile<kTileN>(ep, tmem + lane_bits + b * kAccCols, row0,
+                                    static_cast<int64_t>(nt) * kTileN, c0, c1, row);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0 && !withhold) mbar_arrive_cluster(b ? tempty_leader1 : tempty_leader0);
+        }
       }
       if (!ok) break;
       epi.unit_end(ep, row0, j * NWG + wg, row);
@@ -624,6 +723,7 @@ __device__ __forceinline__ void finish_bulk_stores() {
 // label falls there.
 struct EpiFwdCE {
   using Params = FwdParams;
+  static constexpr bool kSplitHalves = true;
   static constexpr int kStageBytesPerWarp = 4096;
   float* stage;  // this warp's staging buffer (fused path stores)
   float m, s, zyv;
@@ -1371,6 +1471,7 @@ using EpiDwStaged = EpiDwT<true>;
 // ----------------------------------------------------------------------------------------
 struct EpiFlat {
   using Params = FwdParams;
+  static constexpr bool kSplitHalves = true;
   float m, s, s2;
   bool row_ok;
   int64_t grow;
