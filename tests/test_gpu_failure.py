@@ -17,20 +17,25 @@ from parity_util import gpu_fwd_bwd, oracle_fwd_bwd, assert_loss_close
 pytestmark = pytest.mark.gpu
 
 
-def test_wait_runs_out_reports_timeout_and_context_survives():
+# CE: the forward tile releases its accumulator in two sub-tiles (the hook withholds the
+# first); kl_div: the two-operand tile releases it at once.
+@pytest.mark.parametrize("kind", ["ce", "kl_div"])
+def test_wait_runs_out_reports_timeout_and_context_survives(kind):
     from lm_head_loss_streaming_b200.loss import device_status, lm_head_loss_fwd
-    inp = synthetic.make("ce", 512, 256, 4096, w_std=0.05, ignore_frac=0.1, seed=31)
+    inp = synthetic.make(kind, 512, 256, 4096, w_std=0.05, ignore_frac=0.1, seed=31)
     dev = torch.device("cuda", 0)
     Hq, W, lab = inp.Hq.to(dev), inp.W.to(dev), inp.labels.to(dev)
+    Hp = inp.Hp.to(dev) if inp.Hp is not None else None
     assert _lib.slm_debug_set(1, 100_000_000) == 0   # ~0.05-0.1 s per wait
     try:
-        fwd = lm_head_loss_fwd("ce", Hq, W, lab, None, inp.ignore_index)
+        fwd = lm_head_loss_fwd(kind, Hq, W, lab, Hp, inp.ignore_index)
         st = device_status(fwd)
     finally:
         assert _lib.slm_debug_set(0, 0) == 0
     assert st == 7, _lib.status_string(st)   # SLM_ERR_TIMEOUT
     # The context is usable and the next call is correct.
-    g = gpu_fwd_bwd(inp, "ce")
+    g = gpu_fwd_bwd(inp, kind)
     assert g["st_fwd"] == 0 and g["st_bwd"] == 0
-    r = oracle_fwd_bwd(inp, "ce")
-    assert_loss_close(g["loss_tok"], r["loss_tok"], g["loss_mean"], r["loss"], "after timeout")
+    r = oracle_fwd_bwd(inp, kind)
+    assert_loss_close(g["loss_tok"], r["loss_tok"], g["loss_mean"], r["loss"],
+                      f"{kind} after timeout")
