@@ -208,8 +208,8 @@ struct EpiStageBytes<E, decltype(void(E::kStageBytesPerWarp))> {
 
 // Epilogues that set kSplitHalves take a single-buffered two-sub-tile accumulator in two
 // halves (see gemm_pair_kernel): each warpgroup drains its share of the first sub-tile,
-// releases it, then drains its share of the second.  Their tile() must accept any 32-column-aligned
-// sub-range [c0, c1) and not depend on the order in which the ranges come.
+// releases it, then drains its share of the second.  Their tile() must accept any
+// 32-column-aligned sub-range [c0, c1) and not depend on the order in which ranges come.
 template <class E, class = void>
 struct EpiSplit {
   static constexpr bool value = false;
