@@ -532,8 +532,8 @@ static int launch_chunk_fused(int zkind, const CUtensorMap& tHq, const CUtensorM
   fg.num_mw = static_cast<int>(ceil_div(V, kPairM));
   fg.num_nw = static_cast<int>(ceil_div(d, kTileDw));
   fg.kb_w = static_cast<int>(ceil_div(rows, kBK));
-  fg.group_h = std::max(1, std::min(kGroupB, fg.num_mh));
-  fg.group_w = std::max(1, std::min(kGroupB, fg.num_mw));
+  fg.group_h = std::max(1, std::min(group_b(fg.num_nh), fg.num_mh));
+  fg.group_w = std::max(1, std::min(group_b(fg.num_nw), fg.num_mw));
   SLM_LAUNCH(kTrBwdFused, launch_bwd_fused(zkind < 0 ? 0 : zkind, tHq, tHp, tWk, tDzK, tWmn,
                                            tDzMn, tHmn, fg, pz, ph, pw, ctl, s));
   return SLM_OK;
